@@ -1,0 +1,79 @@
+"""Plant plausible mistakes in a copy of the oracle (on the CPU) and require
+that the pins catch every one.  A pin set that lets a dropped term, a wrong
+index or a transposed operand through would not be pinning anything."""
+import importlib.util
+import os
+
+import pytest
+
+from tests import oracle_pins
+
+ORACLE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "oracle", "vsa_oracle.py")
+
+# (name, exact source fragment, replacement)
+MUTATIONS = [
+    ("pool divides by 64", "sum(axis=2) / m", "sum(axis=2) / BLOCK"),
+    ("pool includes padding", "x[:, :, BLOCK * j:BLOCK * j + m, :].sum(axis=2)",
+     "x[:, :, BLOCK * j:BLOCK * j + BLOCK, :].sum(axis=2)"),
+    ("coarse drops scale", 'scores = scale * np.einsum("bhqd,bhkd->bhqk", qc, kc)',
+     'scores = np.einsum("bhqd,bhkd->bhqk", qc, kc)'),
+    ("coarse softmax over q", "    p = softmax_rows(scores)\n",
+     "    p = softmax_rows(scores.swapaxes(-1, -2)).swapaxes(-1, -2)\n"),
+    ("coarse output uses kc", 'out_c = np.einsum("bhqk,bhkd->bhqd", p, vc)',
+     'out_c = np.einsum("bhqk,bhkd->bhqd", p, kc)'),
+    ("topk ties to higher index", "order = np.lexsort((cols, -scores[b, h, a]))",
+     "order = np.lexsort((-cols, -scores[b, h, a]))"),
+    ("topk keeps rank order", "chosen = np.sort(order[:k])", "chosen = order[:k]"),
+    ("topk picks smallest", "order = np.lexsort((cols, -scores[b, h, a]))",
+     "order = np.lexsort((cols, scores[b, h, a]))"),
+    ("sparse attends padded keys",
+     "key_rows.append(np.arange(BLOCK * c, BLOCK * c + int(kv_block_sizes[c])))",
+     "key_rows.append(np.arange(BLOCK * c, BLOCK * c + BLOCK))"),
+    ("sparse drops scale", "logits = scale * (qa @ k[b, h, rows, :].T)",
+     "logits = (qa @ k[b, h, rows, :].T)"),
+    ("sparse uses k as values", "p @ v[b, h, rows, :]", "p @ k[b, h, rows, :]"),
+    ("sparse ignores q block size", "mq = int(q_block_sizes[a])", "mq = BLOCK"),
+    ("combine gate not transposed", "g = None if gate is None else _f64(gate).transpose(0, 2, 1, 3)",
+     "g = None if gate is None else _f64(gate).reshape(o_s.shape)"),
+    ("combine gates the sparse branch", "out[:, :, sl, :] = oc * g[:, :, sl, :] + o_s[:, :, sl, :]",
+     "out[:, :, sl, :] = oc + g[:, :, sl, :] * o_s[:, :, sl, :]"),
+    ("combine shifts coarse block", "oc = out_c[:, :, a:a + 1, :]",
+     "oc = out_c[:, :, max(a - 1, 0):max(a - 1, 0) + 1, :]"),
+    ("varlen rebase drops offset", 'out[h, row, :nn] = local + layout["kvoff"][i]',
+     "out[h, row, :nn] = local"),
+    ("varlen pack not block aligned", "                row = [-1] * BLOCK\n",
+     "                row = [-1] * s\n"),
+    ("metadata column-major in tile",
+     "                for t in range(bt * tt, min(T, bt * tt + tt)):\n"
+     "                    for h in range(bh * th, min(Hh, bh * th + th)):\n"
+     "                        for w in range(bw * tw, min(W, bw * tw + tw)):\n",
+     "                for w in range(bw * tw, min(W, bw * tw + tw)):\n"
+     "                    for h in range(bh * th, min(Hh, bh * th + th)):\n"
+     "                        for t in range(bt * tt, min(T, bt * tt + tt)):\n"),
+    ("metadata reverse is forward", "reverse[perm] = np.arange(len(perm), dtype=np.int64)",
+     "reverse[:] = perm"),
+    ("metadata pads every tile to the end", "non_pad.extend(range(vol * j, vol * j + s))",
+     "non_pad.extend(range(vol * j + vol - s, vol * j + vol))"),
+]
+
+
+def _mutant(old, new):
+    src = open(ORACLE).read()
+    assert src.count(old) == 1, f"mutation anchor not unique/present: {old!r}"
+    spec = importlib.util.spec_from_loader("oracle_mutant", loader=None)
+    mod = importlib.util.module_from_spec(spec)
+    exec(compile(src.replace(old, new), ORACLE + " (mutant)", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_mutation(name, old, new):
+    mod = _mutant(old, new)
+    caught = []
+    for check in oracle_pins.ALL_CHECKS:
+        try:
+            check(mod)
+        except Exception as e:  # noqa: BLE001 - any failure counts as caught
+            caught.append((check.__name__, type(e).__name__))
+    assert caught, f"no pin caught the planted mistake '{name}'"
