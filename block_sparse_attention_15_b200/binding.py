@@ -1,0 +1,344 @@
+"""Thin ctypes binding over libvsa.so (the C ABI declared in include/vsa.h).
+
+Argument marshalling only: torch allocates device memory for outputs and
+workspaces and supplies the current CUDA stream; every step of the VSA
+forward runs in the library's CUDA kernels.  There is no CPU fallback: if the
+shared library is missing or a call fails, these functions raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvsa.so")
+
+VSA_OK = 0
+VSA_MAX_BLOCKS = 2048
+STATUS_NAMES = {
+    0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_SHAPE", 3: "VSA_ERR_UNSUPPORTED",
+    4: "VSA_ERR_CUDA", 5: "VSA_ERR_DEVICE_TIMEOUT", 6: "VSA_ERR_INDEX_RANGE",
+    7: "VSA_ERR_WORKSPACE", 8: "VSA_ERR_BLOCK_SIZE",
+}
+
+_c_void_p = ctypes.c_void_p
+_c_int = ctypes.c_int
+_c_int64 = ctypes.c_int64
+_c_size_t = ctypes.c_size_t
+_c_float = ctypes.c_float
+_P32 = ctypes.POINTER(ctypes.c_int32)
+_P64 = ctypes.POINTER(ctypes.c_int64)
+
+# name -> (restype, argtypes); mirrors include/vsa.h
+SIGNATURES = {
+    "vsa_status_string": (ctypes.c_char_p, [_c_int]),
+    "vsa_abi_version": (_c_int, []),
+    "vsa_get_device_status": (_c_int, [_c_void_p]),
+    "vsa_forward_workspace_size": (_c_size_t, [_c_int] * 5),
+    "vsa_forward": (_c_int, [_c_void_p] * 4 + [_c_void_p, _c_void_p] + [_c_int] * 6 +
+                    [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p,
+                     _c_size_t, _c_void_p]),
+    "block_sparse_attn_from_indices": (_c_int, [_c_void_p] * 7 + [_c_int] * 6 +
+                                       [_c_float, _c_void_p, _c_void_p]),
+    "block_sparse_attn_varlen_workspace_size": (_c_size_t, [_c_int] * 3),
+    "block_sparse_attn_varlen": (_c_int, [_c_void_p] * 3 + [_P32, _P32, _P32, _P32, _P32, _P32] +
+                                 [_c_int] * 3 + [_c_void_p, _c_void_p, _c_int, _c_float,
+                                                 _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                                 _c_void_p, _c_size_t, _c_void_p]),
+    "build_vsa_metadata": (_c_int, [_c_int] * 6 + [_P64, _P64, _P32, _P64, _P64, _P32]),
+    "vsa_gather_tokens": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int64, _c_int64, _c_int64,
+                                   _c_int, _c_void_p]),
+    "vsa_scatter_tokens": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int64, _c_int64,
+                                    _c_int64, _c_int, _c_void_p]),
+    "vsa_selftest_umma": (_c_int, [_c_int, _c_int, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+}
+
+_LIB = None
+
+
+class VSAError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load libvsa.so (built in-tree); raise if it is missing."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m block_sparse_attention_15_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = h
+    return _LIB
+
+
+def _check(fn: str, code: int):
+    if code != VSA_OK:
+        raise VSAError(fn, code)
+
+
+def _ptr(t):
+    return None if t is None else _c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return _c_void_p(s.cuda_stream)
+
+
+def _require(t, dtype, name, device=True):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _block_sizes_tensor(bs, n, device):
+    if bs is None:
+        return None
+    if not isinstance(bs, torch.Tensor):
+        bs = torch.tensor(list(bs), dtype=torch.int32)
+    bs = bs.to(device=device, dtype=torch.int32).contiguous()
+    if bs.numel() != n:
+        raise ValueError(f"expected {n} block sizes, got {bs.numel()}")
+    return bs
+
+
+def get_device_status(stream=None) -> int:
+    """Synchronise the stream, then read and clear the device status word."""
+    return lib().vsa_get_device_status(_stream(stream))
+
+
+def check_device_status(stream=None):
+    code = get_device_status(stream)
+    if code != VSA_OK:
+        raise VSAError("device status", code)
+
+
+def vsa_forward(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=None, *, topk: int,
+                scale: float | None = None, idx_stride: int | None = None, out=None,
+                return_out_c: bool = False, return_pooled: bool = False, workspace=None,
+                stream=None):
+    """Full VSA forward through ``vsa_forward`` (see include/vsa.h).
+
+    q: [B, H, Sq_pad, D] bf16; k, v: [B, H, Skv_pad, D]; gate: [B, Sq_pad, H, D]
+    or None.  Returns ``(out, q2k_idx, q2k_num)`` plus ``out_c`` and the pooled
+    (qc, kc, vc) when asked.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, torch.bfloat16, n)
+    B, H, Sq, D = q.shape
+    Skv = k.shape[2]
+    if k.shape != (B, H, Skv, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H, Skv_pad, D] matching q")
+    if gate is not None:
+        _require(gate, torch.bfloat16, "gate")
+        if gate.shape != (B, Sq, H, D):
+            raise ValueError(f"gate must be [B, Sq_pad, H, D] = {(B, Sq, H, D)}, got {tuple(gate.shape)}")
+    nq, nkv = Sq // 64, Skv // 64
+    k_eff = min(int(topk), nkv)
+    stride = k_eff if idx_stride is None else int(idx_stride)
+    dev = q.device
+    qbs = _block_sizes_tensor(q_block_sizes, nq, dev)
+    kbs = _block_sizes_tensor(kv_block_sizes, nkv, dev)
+    if out is None:
+        out = torch.empty_like(q)
+    q2k_idx = torch.empty((B, H, nq, stride), dtype=torch.int32, device=dev)
+    q2k_num = torch.empty((B, H, nq), dtype=torch.int32, device=dev)
+    out_c = torch.empty((B, H, nq, D), dtype=torch.float32, device=dev) if return_out_c else None
+    L = lib()
+    ws_bytes = L.vsa_forward_workspace_size(B, H, nq, nkv, D)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    _check("vsa_forward", L.vsa_forward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(qbs), _ptr(kbs), B, H, Sq, Skv, D, int(topk),
+        float(scale) if scale is not None else 0.0, _ptr(out), _ptr(q2k_idx), _ptr(q2k_num), stride,
+        _ptr(out_c), _ptr(workspace), workspace.numel(), _stream(stream)))
+    res = [out, q2k_idx, q2k_num]
+    if return_out_c:
+        res.append(out_c)
+    if return_pooled:
+        res.append(pooled_views(workspace, B, H, nq, nkv, D))
+    return tuple(res)
+
+
+def pooled_views(workspace, B, H, nq, nkv, D):
+    """(qc, kc, vc) fp32 views of a vsa_forward workspace (its documented order)."""
+    g = B * H * D * 4
+
+    def a256(x):
+        return (x + 255) // 256 * 256
+
+    offs = [0, a256(g * nq), a256(g * nq) + a256(g * nkv)]
+    shapes = [(B, H, nq, D), (B, H, nkv, D), (B, H, nkv, D)]
+    views = []
+    for off, shp in zip(offs, shapes):
+        n = int(np.prod(shp))
+        views.append(workspace[off:off + 4 * n].view(torch.float32).view(shp))
+    return tuple(views)
+
+
+def block_sparse_attn_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes=None,
+                                   kv_block_sizes=None, *, scale: float | None = None, out=None,
+                                   stream=None):
+    """Block-sparse attention over the listed tiles (``block_sparse_attn_from_indices``)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, torch.bfloat16, n)
+    _require(q2k_idx, torch.int32, "q2k_idx")
+    _require(q2k_num, torch.int32, "q2k_num")
+    B, H, Sq, D = q.shape
+    Skv = k.shape[2]
+    nq, nkv = Sq // 64, Skv // 64
+    if q2k_idx.dim() != 4 or q2k_idx.shape[:3] != (B, H, nq) or q2k_num.shape != (B, H, nq):
+        raise ValueError("q2k_idx must be [B, H, n_q_blocks, stride], q2k_num [B, H, n_q_blocks]")
+    dev = q.device
+    qbs = _block_sizes_tensor(q_block_sizes, nq, dev)
+    kbs = _block_sizes_tensor(kv_block_sizes, nkv, dev)
+    if out is None:
+        out = torch.empty_like(q)
+    _check("block_sparse_attn_from_indices", lib().block_sparse_attn_from_indices(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(q2k_idx), _ptr(q2k_num), _ptr(qbs), _ptr(kbs), B, H, Sq,
+        Skv, D, q2k_idx.shape[3], float(scale) if scale is not None else 0.0, _ptr(out),
+        _stream(stream)))
+    return out
+
+
+def _host_i32(xs):
+    arr = np.ascontiguousarray(np.asarray(xs, dtype=np.int32))
+    return arr, arr.ctypes.data_as(_P32)
+
+
+def block_sparse_attn_varlen(q, k, v, cu_seqlens_q, cu_seqlens_kv, q2k_idx, q2k_num, *,
+                             scale: float | None = None, q_block_sizes_list=None,
+                             kv_block_sizes_list=None, return_aux: bool = False, out=None,
+                             stream=None):
+    """Varlen block-sparse attention (``block_sparse_attn_varlen``).
+
+    q: [H, total_q, D]; k, v: [H, total_kv, D]; cu_seqlens_*: host sequences
+    of n+1 ints; q2k_idx: [H, total_q_blocks, stride] with per-sequence local
+    indices.  With ``return_aux`` also returns (pack_index_q, pack_index_kv,
+    q2k_idx_rebased).
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, torch.bfloat16, n)
+    _require(q2k_idx, torch.int32, "q2k_idx")
+    _require(q2k_num, torch.int32, "q2k_num")
+    H, total_q, D = q.shape
+    cq, cq_p = _host_i32(cu_seqlens_q)
+    ck, ck_p = _host_i32(cu_seqlens_kv)
+    n = len(cq) - 1
+    keep = [cq, ck]
+
+    def sizes(lst):
+        if lst is None:
+            return None, None, None
+        flat = [int(s) for seq in lst for s in seq]
+        cub = [0]
+        for seq in lst:
+            cub.append(cub[-1] + len(seq))
+        a, ap = _host_i32(flat)
+        b, bp = _host_i32(cub)
+        keep.extend([a, b])
+        return ap, bp, len(flat)
+
+    qs_p, qcb_p, nqb = sizes(q_block_sizes_list)
+    ks_p, kcb_p, nkb = sizes(kv_block_sizes_list)
+    if nqb is None:
+        nqb = sum(-(-(int(cq[i + 1]) - int(cq[i])) // 64) for i in range(n))
+    if nkb is None:
+        nkb = sum(-(-(int(ck[i + 1]) - int(ck[i])) // 64) for i in range(n))
+    dev = q.device
+    if out is None:
+        out = torch.zeros_like(q)
+    L = lib()
+    ws_bytes = L.block_sparse_attn_varlen_workspace_size(max(n, 1), max(nqb, 1), max(nkb, 1))
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    aux = None
+    if return_aux:
+        aux = (torch.empty(64 * nqb, dtype=torch.int64, device=dev),
+               torch.empty(64 * nkb, dtype=torch.int64, device=dev),
+               torch.empty_like(q2k_idx))
+    stride = q2k_idx.shape[-1]
+    _check("block_sparse_attn_varlen", L.block_sparse_attn_varlen(
+        _ptr(q), _ptr(k), _ptr(v), cq_p, ck_p, qs_p, qcb_p, ks_p, kcb_p, n, H, D, _ptr(q2k_idx),
+        _ptr(q2k_num), stride, float(scale) if scale is not None else 0.0, _ptr(out),
+        _ptr(aux[0]) if aux else None, _ptr(aux[1]) if aux else None,
+        _ptr(aux[2]) if aux else None, _ptr(ws), ws.numel(), _stream(stream)))
+    del keep
+    return (out, *aux) if return_aux else out
+
+
+def build_vsa_metadata(T: int, Hh: int, W: int, tile=(4, 4, 4)) -> dict:
+    """Tile metadata from the library's host routine (numpy arrays)."""
+    L = lib()
+    n_tiles = ctypes.c_int32(0)
+    _check("build_vsa_metadata", L.build_vsa_metadata(T, Hh, W, *tile, None, None, None, None, None,
+                                                      ctypes.byref(n_tiles)))
+    N = T * Hh * W
+    vol = int(np.prod(tile))
+    nt = n_tiles.value
+    perm = np.empty(N, dtype=np.int64)
+    rev = np.empty(N, dtype=np.int64)
+    vbs = np.empty(nt, dtype=np.int32)
+    npi = np.empty(N, dtype=np.int64)
+    slot = np.empty(nt * vol, dtype=np.int64)
+    _check("build_vsa_metadata", L.build_vsa_metadata(
+        T, Hh, W, *tile, perm.ctypes.data_as(_P64), rev.ctypes.data_as(_P64),
+        vbs.ctypes.data_as(_P32), npi.ctypes.data_as(_P64), slot.ctypes.data_as(_P64),
+        ctypes.byref(n_tiles)))
+    return dict(tile_partition_indices=perm, reverse_tile_partition_indices=rev,
+                variable_block_sizes=vbs, non_pad_index=npi, slot_token=slot, n_tiles=nt,
+                max_block_size=vol)
+
+
+def gather_tokens(x, slot_token, *, stream=None):
+    """[G, N, D] tokens -> [G, n_slots, D] padded block layout (zeros in pads)."""
+    _require(x, torch.bfloat16, "x")
+    _require(slot_token, torch.int64, "slot_token")
+    G, N, D = x.shape
+    ns = slot_token.numel()
+    dst = torch.empty((G, ns, D), dtype=x.dtype, device=x.device)
+    _check("vsa_gather_tokens", lib().vsa_gather_tokens(_ptr(x), _ptr(dst), _ptr(slot_token), N, ns,
+                                                        G, D, _stream(stream)))
+    return dst
+
+
+def scatter_tokens(x_pad, slot_token, n_tokens: int, *, stream=None):
+    """Inverse of :func:`gather_tokens` on the real tokens."""
+    _require(x_pad, torch.bfloat16, "x_pad")
+    _require(slot_token, torch.int64, "slot_token")
+    G, ns, D = x_pad.shape
+    dst = torch.empty((G, n_tokens, D), dtype=x_pad.dtype, device=x_pad.device)
+    _check("vsa_scatter_tokens", lib().vsa_scatter_tokens(_ptr(x_pad), _ptr(dst), _ptr(slot_token),
+                                                          n_tokens, ns, G, D, _stream(stream)))
+    return dst
+
+
+def selftest_umma(mode: int, a, b, *, stream=None):
+    """Run one tensor-core product of the sparse kernel on global operands."""
+    _require(a, torch.bfloat16, "a")
+    _require(b, torch.bfloat16, "b")
+    D = a.shape[1]
+    rows = 128 if mode == 0 else D
+    c = torch.empty((rows, 64), dtype=torch.float32, device=a.device)
+    _check("vsa_selftest_umma", lib().vsa_selftest_umma(mode, D, _ptr(a), _ptr(b), _ptr(c),
+                                                        _stream(stream)))
+    return c
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

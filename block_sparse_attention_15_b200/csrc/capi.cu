@@ -1,0 +1,417 @@
+// C ABI of libvsa.so: argument checks, workspace carving, host-side block
+// metadata, and the launch sequence of every entry point declared in vsa.h.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <vector>
+
+#include "vsa.h"
+#include "vsa_launch.h"
+
+namespace vsa {
+
+// Device status word: kernels record the first error of a launch sequence.
+__device__ int g_device_status = 0;
+
+int* device_status_ptr() {
+  static int* cached[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cached[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_device_status) != cudaSuccess) return nullptr;
+    cached[dev] = static_cast<int*>(ptr);
+  }
+  return cached[dev];
+}
+
+static inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static inline bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+static inline float resolve_scale(float scale, int D) {
+  return scale > 0.f ? scale : 1.0f / sqrtf((float)D);
+}
+
+}  // namespace vsa
+
+using namespace vsa;
+
+extern "C" {
+
+const char* vsa_status_string(int status) {
+  switch (status) {
+    case VSA_OK: return "ok";
+    case VSA_ERR_INVALID_ARG: return "invalid argument";
+    case VSA_ERR_SHAPE: return "inconsistent shape";
+    case VSA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case VSA_ERR_CUDA: return "CUDA error";
+    case VSA_ERR_DEVICE_TIMEOUT: return "device barrier wait timed out";
+    case VSA_ERR_INDEX_RANGE: return "block index out of range";
+    case VSA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case VSA_ERR_BLOCK_SIZE: return "block size outside [1, 64]";
+    default: return "unknown status";
+  }
+}
+
+int vsa_abi_version(void) { return (1 << 16) | 0; }
+
+int vsa_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return VSA_ERR_CUDA;
+  int value = 0;
+  if (cudaMemcpyFromSymbol(&value, g_device_status, sizeof(int)) != cudaSuccess) return VSA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return VSA_ERR_CUDA;
+  return value;
+}
+
+// ---------------------------------------------------------------------------
+// vsa_forward
+// ---------------------------------------------------------------------------
+size_t vsa_forward_workspace_size(int B, int H, int n_q_blocks, int n_kv_blocks, int D) {
+  if (B <= 0 || H <= 0 || n_q_blocks <= 0 || n_kv_blocks <= 0 || D <= 0) return 0;
+  const size_t g = (size_t)B * H * D * sizeof(float);
+  return align256(g * n_q_blocks) * 2 + align256(g * n_kv_blocks) * 2;
+}
+
+int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
+                const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B, int H,
+                int Sq_pad, int Skv_pad, int D, int topk, float scale, void* out,
+                int32_t* q2k_idx, int32_t* q2k_num, int idx_stride, float* out_c,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !out || !q2k_idx || !q2k_num) return VSA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || topk < 1 || !(scale == scale))
+    return VSA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
+  if (Sq_pad % 64 || Skv_pad % 64) return VSA_ERR_SHAPE;
+  const int nq = Sq_pad / 64, nkv = Skv_pad / 64;
+  if (nq > VSA_MAX_BLOCKS || nkv > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
+  const int k_eff = topk < nkv ? topk : nkv;
+  if (idx_stride < k_eff) return VSA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (gate && !aligned16(gate)) || (out_c && !aligned16(out_c)))
+    return VSA_ERR_INVALID_ARG;
+  const size_t need = vsa_forward_workspace_size(B, H, nq, nkv, D);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return VSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = device_status_ptr();
+  if (!status) return VSA_ERR_CUDA;
+
+  const size_t g = (size_t)B * H * D * sizeof(float);
+  char* ws = static_cast<char*>(workspace);
+  float* qc = reinterpret_cast<float*>(ws);
+  ws += align256(g * nq);
+  float* kc = reinterpret_cast<float*>(ws);
+  ws += align256(g * nkv);
+  float* vc = reinterpret_cast<float*>(ws);
+  ws += align256(g * nkv);
+  float* oc = out_c ? out_c : reinterpret_cast<float*>(ws);
+
+  PoolParams pp;
+  pp.q = static_cast<const __nv_bfloat16*>(q);
+  pp.k = static_cast<const __nv_bfloat16*>(k);
+  pp.v = static_cast<const __nv_bfloat16*>(v);
+  pp.q_bs = q_block_sizes;
+  pp.kv_bs = kv_block_sizes;
+  pp.groups = B * H;
+  pp.nq = nq;
+  pp.nkv = nkv;
+  pp.qc = qc;
+  pp.kc = kc;
+  pp.vc = vc;
+  pp.status = status;
+  int rc = launch_pool(pp, D, st);
+  if (rc != VSA_OK) return rc;
+
+  const float sc = resolve_scale(scale, D);
+  CoarseParams cp;
+  cp.qc = qc;
+  cp.kc = kc;
+  cp.vc = vc;
+  cp.groups = B * H;
+  cp.nq = nq;
+  cp.nkv = nkv;
+  cp.scale = sc;
+  cp.topk = k_eff;
+  cp.idx_stride = idx_stride;
+  cp.q2k_idx = q2k_idx;
+  cp.q2k_num = q2k_num;
+  cp.out_c = oc;
+  rc = launch_coarse_topk(cp, D, st);
+  if (rc != VSA_OK) return rc;
+
+  SparseParams sp;
+  memset(&sp, 0, sizeof(sp));
+  sp.out = static_cast<__nv_bfloat16*>(out);
+  sp.gate = static_cast<const __nv_bfloat16*>(gate);
+  sp.out_c = oc;
+  sp.q2k_idx = q2k_idx;
+  sp.q2k_num = q2k_num;
+  sp.idx_stride = idx_stride;
+  sp.q_bs = q_block_sizes;
+  sp.kv_bs = kv_block_sizes;
+  sp.B = B;
+  sp.H = H;
+  sp.nq = nq;
+  sp.nkv = nkv;
+  sp.q_rows_per_group = Sq_pad;
+  sp.kv_rows_per_group = Skv_pad;
+  sp.gate_seq = Sq_pad;
+  sp.scale_log2 = sc * 1.4426950408889634f;
+  sp.varlen = 0;
+  sp.status = status;
+  return launch_sparse(sp, q, k, v, (long long)B * H * Sq_pad, (long long)B * H * Skv_pad, D,
+                       /*combine=*/true, /*gated=*/gate != nullptr, st);
+}
+
+// ---------------------------------------------------------------------------
+// block_sparse_attn_from_indices
+// ---------------------------------------------------------------------------
+int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
+                                   const int32_t* q2k_idx, const int32_t* q2k_num,
+                                   const int32_t* q_block_sizes, const int32_t* kv_block_sizes,
+                                   int B, int H, int Sq_pad, int Skv_pad, int D, int idx_stride,
+                                   float scale, void* out, void* stream) {
+  if (!q || !k || !v || !out || !q2k_idx || !q2k_num) return VSA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || idx_stride < 1 || !(scale == scale))
+    return VSA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
+  if (Sq_pad % 64 || Skv_pad % 64) return VSA_ERR_SHAPE;
+  const int nq = Sq_pad / 64, nkv = Skv_pad / 64;
+  if (idx_stride > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return VSA_ERR_INVALID_ARG;
+  int* status = device_status_ptr();
+  if (!status) return VSA_ERR_CUDA;
+  const float sc = resolve_scale(scale, D);
+  SparseParams sp;
+  memset(&sp, 0, sizeof(sp));
+  sp.out = static_cast<__nv_bfloat16*>(out);
+  sp.q2k_idx = q2k_idx;
+  sp.q2k_num = q2k_num;
+  sp.idx_stride = idx_stride;
+  sp.q_bs = q_block_sizes;
+  sp.kv_bs = kv_block_sizes;
+  sp.B = B;
+  sp.H = H;
+  sp.nq = nq;
+  sp.nkv = nkv;
+  sp.q_rows_per_group = Sq_pad;
+  sp.kv_rows_per_group = Skv_pad;
+  sp.scale_log2 = sc * 1.4426950408889634f;
+  sp.status = status;
+  return launch_sparse(sp, q, k, v, (long long)B * H * Sq_pad, (long long)B * H * Skv_pad, D,
+                       false, false, static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// block_sparse_attn_varlen
+// ---------------------------------------------------------------------------
+size_t block_sparse_attn_varlen_workspace_size(int n_seqs, int total_q_blocks,
+                                               int total_kv_blocks) {
+  if (n_seqs <= 0 || total_q_blocks <= 0 || total_kv_blocks <= 0) return 0;
+  return align256(sizeof(int32_t) * (4 * (size_t)total_q_blocks + 2 * (size_t)total_kv_blocks));
+}
+
+// Resolve one side's blocks: per block first token row and size.
+static int resolve_blocks(const int32_t* cu, const int32_t* sizes, const int32_t* cu_blocks,
+                          int n, std::vector<int32_t>& tok, std::vector<int32_t>& len,
+                          std::vector<int32_t>& first_block) {
+  first_block.assign(n + 1, 0);
+  if (cu[0] != 0) return VSA_ERR_SHAPE;
+  for (int i = 0; i < n; ++i) {
+    const long long L = (long long)cu[i + 1] - cu[i];
+    if (L <= 0) return VSA_ERR_SHAPE;  // zero-token sequences are rejected
+    if (sizes) {
+      if (!cu_blocks) return VSA_ERR_INVALID_ARG;
+      if (cu_blocks[0] != 0 || cu_blocks[i + 1] <= cu_blocks[i]) return VSA_ERR_SHAPE;
+      long long t = cu[i];
+      for (int j = cu_blocks[i]; j < cu_blocks[i + 1]; ++j) {
+        const int s = sizes[j];
+        if (s < 1 || s > 64) return VSA_ERR_BLOCK_SIZE;
+        tok.push_back((int32_t)t);
+        len.push_back(s);
+        t += s;
+      }
+      if (t != cu[i + 1]) return VSA_ERR_SHAPE;  // block sizes must cover the sequence
+    } else {
+      for (long long t = cu[i]; t < cu[i + 1]; t += 64) {
+        tok.push_back((int32_t)t);
+        len.push_back((int32_t)((cu[i + 1] - t) < 64 ? (cu[i + 1] - t) : 64));
+      }
+    }
+    first_block[i + 1] = (int32_t)tok.size();
+  }
+  return VSA_OK;
+}
+
+int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
+                             const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv,
+                             const int32_t* q_block_sizes, const int32_t* cu_q_blocks,
+                             const int32_t* kv_block_sizes, const int32_t* cu_kv_blocks,
+                             int n_seqs, int H, int D, const int32_t* q2k_idx,
+                             const int32_t* q2k_num, int idx_stride, float scale, void* out,
+                             int64_t* pack_index_q, int64_t* pack_index_kv,
+                             int32_t* q2k_idx_rebased, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  if (!q || !k || !v || !out || !q2k_idx || !q2k_num || !cu_seqlens_q || !cu_seqlens_kv)
+    return VSA_ERR_INVALID_ARG;
+  if (n_seqs <= 0) return VSA_ERR_SHAPE;  // empty batch
+  if (H <= 0 || idx_stride < 1 || !(scale == scale)) return VSA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
+  if (idx_stride > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return VSA_ERR_INVALID_ARG;
+  std::vector<int32_t> qtok, qlen, qfirst, ktok, klen, kfirst;
+  int rc = resolve_blocks(cu_seqlens_q, q_block_sizes, cu_q_blocks, n_seqs, qtok, qlen, qfirst);
+  if (rc != VSA_OK) return rc;
+  rc = resolve_blocks(cu_seqlens_kv, kv_block_sizes, cu_kv_blocks, n_seqs, ktok, klen, kfirst);
+  if (rc != VSA_OK) return rc;
+  const int nqb = (int)qtok.size(), nkvb = (int)ktok.size();
+  std::vector<int32_t> table(4 * (size_t)nqb + 2 * (size_t)nkvb);
+  int32_t* t_qtok = table.data();
+  int32_t* t_qlen = t_qtok + nqb;
+  int32_t* t_kvbase = t_qlen + nqb;
+  int32_t* t_kvcount = t_kvbase + nqb;
+  int32_t* t_ktok = t_kvcount + nqb;
+  int32_t* t_klen = t_ktok + nkvb;
+  for (int i = 0; i < n_seqs; ++i) {
+    for (int a = qfirst[i]; a < qfirst[i + 1]; ++a) {
+      t_qtok[a] = qtok[a];
+      t_qlen[a] = qlen[a];
+      t_kvbase[a] = kfirst[i];
+      t_kvcount[a] = kfirst[i + 1] - kfirst[i];
+    }
+  }
+  memcpy(t_ktok, ktok.data(), sizeof(int32_t) * nkvb);
+  memcpy(t_klen, klen.data(), sizeof(int32_t) * nkvb);
+  const size_t need = block_sparse_attn_varlen_workspace_size(n_seqs, nqb, nkvb);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return VSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* dtab = static_cast<int32_t*>(workspace);
+  // Pageable source: the runtime stages it before returning, so `table` may
+  // be released right after the call.
+  if (cudaMemcpyAsync(dtab, table.data(), sizeof(int32_t) * table.size(), cudaMemcpyHostToDevice,
+                      st) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  int* status = device_status_ptr();
+  if (!status) return VSA_ERR_CUDA;
+  const int32_t* d_qtok = dtab;
+  const int32_t* d_qlen = d_qtok + nqb;
+  const int32_t* d_kvbase = d_qlen + nqb;
+  const int32_t* d_kvcount = d_kvbase + nqb;
+  const int32_t* d_ktok = d_kvcount + nqb;
+  const int32_t* d_klen = d_ktok + nkvb;
+  if (pack_index_q && (rc = launch_varlen_aux(d_qtok, d_qlen, nqb, pack_index_q, st)) != VSA_OK)
+    return rc;
+  if (pack_index_kv && (rc = launch_varlen_aux(d_ktok, d_klen, nkvb, pack_index_kv, st)) != VSA_OK)
+    return rc;
+  if (q2k_idx_rebased &&
+      (rc = launch_rebase(q2k_idx, q2k_num, d_kvbase, d_kvcount, H, nqb, idx_stride,
+                          q2k_idx_rebased, status, st)) != VSA_OK)
+    return rc;
+  const long long total_q = cu_seqlens_q[n_seqs], total_kv = cu_seqlens_kv[n_seqs];
+  const float sc = resolve_scale(scale, D);
+  SparseParams sp;
+  memset(&sp, 0, sizeof(sp));
+  sp.out = static_cast<__nv_bfloat16*>(out);
+  sp.q2k_idx = q2k_idx;
+  sp.q2k_num = q2k_num;
+  sp.idx_stride = idx_stride;
+  sp.q_bs = d_qlen;
+  sp.kv_bs = d_klen;
+  sp.q_tok = d_qtok;
+  sp.kv_tok = d_ktok;
+  sp.q_kv_base = d_kvbase;
+  sp.q_kv_count = d_kvcount;
+  sp.B = 1;
+  sp.H = H;
+  sp.nq = nqb;
+  sp.nkv = nkvb;
+  sp.q_rows_per_group = total_q;
+  sp.kv_rows_per_group = total_kv;
+  sp.scale_log2 = sc * 1.4426950408889634f;
+  sp.varlen = 1;
+  sp.status = status;
+  return launch_sparse(sp, q, k, v, (long long)H * total_q, (long long)H * total_kv, D, false,
+                       false, st);
+}
+
+// ---------------------------------------------------------------------------
+// build_vsa_metadata (host) and the device gather / scatter
+// ---------------------------------------------------------------------------
+int build_vsa_metadata(int T, int Hh, int W, int tT, int tH, int tW,
+                       int64_t* tile_partition_indices, int64_t* reverse_tile_partition_indices,
+                       int32_t* variable_block_sizes, int64_t* non_pad_index,
+                       int64_t* slot_token, int32_t* n_tiles) {
+  if (T <= 0 || Hh <= 0 || W <= 0 || tT <= 0 || tH <= 0 || tW <= 0) return VSA_ERR_INVALID_ARG;
+  const int vol = tT * tH * tW;
+  if (vol > 64) return VSA_ERR_INVALID_ARG;
+  const int nT = (T + tT - 1) / tT, nH = (Hh + tH - 1) / tH, nW = (W + tW - 1) / tW;
+  const long long ntiles = (long long)nT * nH * nW;
+  if (ntiles > 0x7FFFFFFFLL) return VSA_ERR_UNSUPPORTED;
+  if (n_tiles) *n_tiles = (int32_t)ntiles;
+  long long pos = 0;
+  long long tile = 0;
+  for (int bt = 0; bt < nT; ++bt) {
+    for (int bh = 0; bh < nH; ++bh) {
+      for (int bw = 0; bw < nW; ++bw, ++tile) {
+        int count = 0;
+        const int t1 = (bt + 1) * tT < T ? (bt + 1) * tT : T;
+        const int h1 = (bh + 1) * tH < Hh ? (bh + 1) * tH : Hh;
+        const int w1 = (bw + 1) * tW < W ? (bw + 1) * tW : W;
+        for (int t = bt * tT; t < t1; ++t) {
+          for (int h = bh * tH; h < h1; ++h) {
+            for (int w = bw * tW; w < w1; ++w) {
+              const int64_t token = ((int64_t)t * Hh + h) * W + w;
+              const int64_t slot = tile * vol + count;
+              if (tile_partition_indices) tile_partition_indices[pos] = token;
+              if (reverse_tile_partition_indices) reverse_tile_partition_indices[token] = pos;
+              if (non_pad_index) non_pad_index[pos] = slot;
+              if (slot_token) slot_token[slot] = token;
+              ++pos;
+              ++count;
+            }
+          }
+        }
+        if (variable_block_sizes) variable_block_sizes[tile] = count;
+        if (slot_token) {
+          for (int s = count; s < vol; ++s) slot_token[tile * vol + s] = -1;
+        }
+      }
+    }
+  }
+  return VSA_OK;
+}
+
+int vsa_gather_tokens(const void* src, void* dst, const int64_t* slot_token, int64_t n_tokens,
+                      int64_t n_slots, int64_t groups, int D, void* stream) {
+  if (!src || !dst || !slot_token || n_tokens < 0 || n_slots < 0 || groups < 0)
+    return VSA_ERR_INVALID_ARG;
+  if (D <= 0 || D % 8) return VSA_ERR_UNSUPPORTED;
+  if (!aligned16(src) || !aligned16(dst)) return VSA_ERR_INVALID_ARG;
+  return launch_gather_tokens(src, dst, slot_token, n_tokens, n_slots, groups, D, false,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int vsa_scatter_tokens(const void* src, void* dst, const int64_t* slot_token, int64_t n_tokens,
+                       int64_t n_slots, int64_t groups, int D, void* stream) {
+  if (!src || !dst || !slot_token || n_tokens < 0 || n_slots < 0 || groups < 0)
+    return VSA_ERR_INVALID_ARG;
+  if (D <= 0 || D % 8) return VSA_ERR_UNSUPPORTED;
+  if (!aligned16(src) || !aligned16(dst)) return VSA_ERR_INVALID_ARG;
+  return launch_gather_tokens(src, dst, slot_token, n_tokens, n_slots, groups, D, true,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int vsa_selftest_umma(int mode, int D, const void* a, const void* b, float* c, void* stream) {
+  if (!a || !b || !c || (mode != 0 && mode != 1)) return VSA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
+  return launch_selftest_umma(mode, D, a, b, c, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,287 @@
+/*
+ * vsa.h -- C ABI of the B200 (sm_100a) Video Sparse Attention forward library
+ * (libvsa.so).
+ *
+ * The library computes the VSA forward pass described by the FastVideo pages:
+ *   a1 mean-pool q, k, v over 64-slot blocks;
+ *   a2 coarse attention among the pooled blocks (out_c, block resolution);
+ *   a3 per query block, the top-k KV blocks by coarse logit (q2k_idx, q2k_num);
+ *   a4 softmax attention restricted to the selected 64x64 tiles (out_s);
+ *   a5 the combine out = out_c * gate + out_s, out_c broadcast inside a block;
+ *   a6 a varlen entry over block-aligned packed sequences with rebased indices;
+ *   a7 host metadata for 3-D video tiles plus the device token gather/scatter.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Element type "bf16" is IEEE bfloat16 (2 bytes); all activations are bf16.
+ * - Layout "BHSD": [batch][head][sequence slot][head dim], contiguous, with the
+ *   sequence padded to 64 slots per block: block j occupies slots 64j..64j+63,
+ *   its real tokens first.  Padded slots must hold finite values (zeros are
+ *   what the packing helpers write); they are never attended to.
+ * - Block sizes ("variable_block_sizes") are int32, one per block, each in
+ *   [1, 64]; NULL means every block is full (64).  Shared by all batches and
+ *   heads.  Sizes outside [1, 64] found on the device set VSA_ERR_BLOCK_SIZE
+ *   in the device status word (see vsa_get_device_status).
+ * - Head dim D is 64 or 128.
+ * - `scale` <= 0 selects 1/sqrt(D).
+ * - Pointers documented "device" must point to memory of the current CUDA
+ *   device; "host" pointers to ordinary host memory.  The caller owns every
+ *   buffer; the library allocates and frees nothing.  Scratch comes from the
+ *   caller's `workspace` (size from the matching *_workspace_size call,
+ *   256-byte aligned).
+ * - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *   asynchronous on that stream and never synchronise it, except
+ *   vsa_get_device_status.
+ * - Every call returns a vsa status code.  Argument problems detectable on
+ *   the host are returned before anything is launched.  Problems found inside
+ *   kernels (an out-of-range index, a bad block size, a barrier wait that ran
+ *   out) are recorded in a per-device status word read by
+ *   vsa_get_device_status.  No C++ exception crosses this interface.
+ *
+ * Page references are to the FastVideo pages: "[kernel] Add varlen support
+ * for block-sparse attention" (PR #1319), "[perf] avoid full-sequence
+ * materialization in VSA coarse/sparse combine" (PR #1813), "[chore] release
+ * fastvideo-kernel 0.3.0" (PR #1478), "[kernel] Extract VSA utility functions
+ * into fastvideo_kernel" (PR #1408) and the fastvideo-kernel README.
+ */
+#ifndef VSA_H_
+#define VSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------- */
+#define VSA_OK 0
+#define VSA_ERR_INVALID_ARG 1    /* null pointer, negative size, bad scale  */
+#define VSA_ERR_SHAPE 2          /* inconsistent sizes (e.g. S not 64*n)    */
+#define VSA_ERR_UNSUPPORTED 3    /* valid but not built (e.g. D = 96)       */
+#define VSA_ERR_CUDA 4           /* a CUDA runtime/driver call failed        */
+#define VSA_ERR_DEVICE_TIMEOUT 5 /* a kernel's bounded barrier wait ran out  */
+#define VSA_ERR_INDEX_RANGE 6    /* q2k_idx entry outside [0, n_kv_blocks)   */
+#define VSA_ERR_WORKSPACE 7      /* workspace missing, small or misaligned   */
+#define VSA_ERR_BLOCK_SIZE 8     /* a block size outside [1, 64]             */
+
+/* Largest supported number of KV blocks per sequence and of index entries
+ * per query block (the coarse stage keeps a full score row on chip). */
+#define VSA_MAX_BLOCKS 2048
+
+/* Human-readable name of a status code (static string). */
+const char* vsa_status_string(int status);
+
+/* Library ABI version: (major << 16) | minor. */
+int vsa_abi_version(void);
+
+/*
+ * Read and clear the device status word of the current device.
+ * Synchronises `stream` first, so it reports every kernel issued before it.
+ * Returns VSA_OK or the first error code a kernel recorded since the last
+ * read; returns VSA_ERR_CUDA if the synchronisation itself failed.
+ */
+int vsa_get_device_status(void* stream);
+
+/* ======================================================================== *
+ * a1-a5: full VSA forward
+ * ======================================================================== */
+
+/*
+ * Workspace bytes vsa_forward needs for these sizes (pooled q/k/v and the
+ * coarse output when `out_c` is not supplied, fp32).
+ */
+size_t vsa_forward_workspace_size(int B, int H, int n_q_blocks, int n_kv_blocks, int D);
+
+/*
+ * vsa_forward -- pool, coarse attention, top-k, block-sparse attention and
+ * the gated combine, in three kernel launches on `stream`.
+ *
+ * Defined by: README "Usage" (`video_sparse_attn(q, k, v, block_sizes,
+ * block_sizes, topk=5)`); PR #1813 "Problem"/"Change" for the combine
+ * out = out_c * gate + out_s with out_c kept at block resolution
+ * [B, H, n_blocks, 1, D] and the gate ("compress_attn_weight") laid out
+ * [B, S, H, D]; release 0.3.0 "Block-sparse / VSA attention improvements"
+ * for q2k_idx / q2k_num.  Readings the pages leave open: coarse softmax
+ * scale equals the fine one; top-k ranks scaled coarse logits, ties to the
+ * lower KV index, each q2k_idx row ascending with -1 after q2k_num entries;
+ * padded query rows of `out` are written as 0.
+ *
+ * q        device bf16 [B, H, Sq_pad, D]   (Sq_pad = 64 * n_q_blocks)
+ * k, v     device bf16 [B, H, Skv_pad, D]  (Skv_pad = 64 * n_kv_blocks)
+ * gate     device bf16 [B, Sq_pad, H, D], or NULL for the ungated combine
+ *          out = out_c + out_s
+ * q_block_sizes   device int32 [Sq_pad/64] or NULL (all 64)
+ * kv_block_sizes  device int32 [Skv_pad/64] or NULL (all 64)
+ * topk     KV blocks kept per query block, >= 1; clamped to n_kv_blocks
+ * out      device bf16 [B, H, Sq_pad, D]
+ * q2k_idx  device int32 [B, H, n_q_blocks, idx_stride], written
+ * q2k_num  device int32 [B, H, n_q_blocks], written (= min(topk, n_kv))
+ * idx_stride  row pitch of q2k_idx, >= min(topk, n_kv_blocks)
+ * out_c    device fp32 [B, H, n_q_blocks, D] to receive the coarse output,
+ *          or NULL (kept in the workspace)
+ * workspace   device, >= vsa_forward_workspace_size(...) bytes, 256-aligned
+ *
+ * Limits: n_q_blocks, n_kv_blocks in [1, VSA_MAX_BLOCKS]; D in {64, 128}.
+ */
+int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
+                const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B, int H,
+                int Sq_pad, int Skv_pad, int D, int topk, float scale, void* out,
+                int32_t* q2k_idx, int32_t* q2k_num, int idx_stride, float* out_c,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* ======================================================================== *
+ * a4: block-sparse attention from indices
+ * ======================================================================== */
+
+/*
+ * block_sparse_attn_from_indices -- out_s = softmax attention of every real
+ * query row of block a over the real keys of the KV blocks listed in
+ * q2k_idx[b, h, a, 0 : q2k_num[b, h, a]] (a block listed twice counts
+ * twice; q2k_num = 0 gives 0).  Padded query rows are written as 0.
+ *
+ * Defined by: release 0.3.0, "Block-sparse / VSA attention improvements":
+ * `block_sparse_attn_from_indices(q, k, v, q2k_idx, q2k_num,
+ * variable_block_sizes)`, the index-native block-sparse API.
+ *
+ * q, k, v, q_block_sizes, kv_block_sizes, Sq_pad, Skv_pad, D, scale: as in
+ *          vsa_forward
+ * q2k_idx  device int32 [B, H, n_q_blocks, idx_stride]; entries past
+ *          q2k_num are ignored.  An entry outside [0, n_kv_blocks) is
+ *          skipped and sets VSA_ERR_INDEX_RANGE in the device status word.
+ * q2k_num  device int32 [B, H, n_q_blocks], each in [0, idx_stride]
+ * idx_stride  1 .. VSA_MAX_BLOCKS
+ * out      device bf16 [B, H, Sq_pad, D]
+ */
+int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
+                                   const int32_t* q2k_idx, const int32_t* q2k_num,
+                                   const int32_t* q_block_sizes, const int32_t* kv_block_sizes,
+                                   int B, int H, int Sq_pad, int Skv_pad, int D, int idx_stride,
+                                   float scale, void* out, void* stream);
+
+/* ======================================================================== *
+ * a6: varlen block-sparse attention
+ * ======================================================================== */
+
+/* Workspace bytes for block_sparse_attn_varlen (device block tables). */
+size_t block_sparse_attn_varlen_workspace_size(int n_seqs, int total_q_blocks,
+                                               int total_kv_blocks);
+
+/*
+ * block_sparse_attn_varlen -- block-sparse attention over several sequences
+ * of different lengths in one launch.
+ *
+ * Defined by: PR #1319 "How it works": sequences are packed block-aligned
+ * (each block takes 64 slots), each sequence's q2k_idx is rebased to global
+ * block offsets, one block-sparse call covers the whole batch, and the output
+ * is unpacked per sequence; Q and KV lengths may differ (release 0.3.0,
+ * "Varlen block-sparse attention").  Here the packing is virtual: a device
+ * block table gives each packed block's first token, so the kernel reads the
+ * token-packed inputs in place and writes only real rows of `out`.
+ *
+ * q        device bf16 [H, total_q, D], sequences back to back
+ * k, v     device bf16 [H, total_kv, D]
+ * cu_seqlens_q, cu_seqlens_kv  host int32 [n_seqs + 1], non-decreasing,
+ *          starting at 0; total_q = cu_seqlens_q[n_seqs]
+ * q_block_sizes   host int32, the blocks of every sequence concatenated
+ *          (each in [1, 64], per sequence summing to its length), or NULL:
+ *          64-token blocks with a partial last block
+ * cu_q_blocks     host int32 [n_seqs + 1]: first block of each sequence in
+ *          q_block_sizes; required iff q_block_sizes is given
+ * kv_block_sizes, cu_kv_blocks  the same for K/V
+ * q2k_idx  device int32 [H, total_q_blocks, idx_stride]: rows of sequence i
+ *          hold indices local to sequence i's KV blocks
+ * q2k_num  device int32 [H, total_q_blocks]
+ * out      device bf16 [H, total_q, D]; only real token rows are written
+ * pack_index_q   device int64 [64 * total_q_blocks] or NULL: for each packed
+ *          slot the token row of q it holds, -1 for padding
+ * pack_index_kv  device int64 [64 * total_kv_blocks] or NULL: same for k/v
+ * q2k_idx_rebased  device int32 [H, total_q_blocks, idx_stride] or NULL:
+ *          q2k_idx plus each sequence's first packed KV block, -1 tails
+ * workspace  device, >= block_sparse_attn_varlen_workspace_size(...) bytes
+ *
+ * Host checks return VSA_ERR_SHAPE for an empty batch, a sequence with zero
+ * tokens, or block sizes whose count or sum disagrees with the lengths (the
+ * PR #1319 review notes).
+ */
+int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
+                             const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv,
+                             const int32_t* q_block_sizes, const int32_t* cu_q_blocks,
+                             const int32_t* kv_block_sizes, const int32_t* cu_kv_blocks,
+                             int n_seqs, int H, int D, const int32_t* q2k_idx,
+                             const int32_t* q2k_num, int idx_stride, float scale, void* out,
+                             int64_t* pack_index_q, int64_t* pack_index_kv,
+                             int32_t* q2k_idx_rebased, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* ======================================================================== *
+ * a7: video tile metadata (host) and token gather / scatter (device)
+ * ======================================================================== */
+
+/*
+ * build_vsa_metadata -- tile partition of a T x Hh x W latent (tokens
+ * numbered row-major over (t, h, w)) into tT x tH x tW tiles.
+ *
+ * Defined by: PR #1408 "Summary"/"Design decisions": one call builds
+ * tile_partition_indices, reverse_tile_partition_indices, the variable block
+ * sizes (tokens per tile, at most the tile volume, tile size a parameter)
+ * and the non-pad index (get_non_pad_index(variable_block_sizes,
+ * max_block_size)).  The pages name these but not the order; this library
+ * visits tiles in row-major (t, h, w) tile order, tokens inside a tile in
+ * row-major (t, h, w) order, and clips edge tiles.
+ *
+ * All pointers are host memory.  Outputs may be NULL to skip them; call
+ * first with all outputs NULL except n_tiles to size the arrays.
+ * tile_partition_indices          int64 [T*Hh*W]: token at tiled position j
+ * reverse_tile_partition_indices  int64 [T*Hh*W]: tiled position of token i
+ * variable_block_sizes            int32 [n_tiles]
+ * non_pad_index                   int64 [T*Hh*W]: padded slot of tiled
+ *                                 position j (tile volume slots per tile)
+ * slot_token                      int64 [n_tiles * tT*tH*tW]: token held by
+ *                                 each padded slot, -1 for padding
+ * n_tiles                         int32 [1]
+ * Returns VSA_ERR_INVALID_ARG for non-positive sizes or a tile volume above
+ * 64.
+ */
+int build_vsa_metadata(int T, int Hh, int W, int tT, int tH, int tW,
+                       int64_t* tile_partition_indices, int64_t* reverse_tile_partition_indices,
+                       int32_t* variable_block_sizes, int64_t* non_pad_index,
+                       int64_t* slot_token, int32_t* n_tiles);
+
+/*
+ * vsa_gather_tokens -- dst[g, s, :] = src[g, slot_token[s], :], or 0 where
+ * slot_token[s] < 0: places tokens into the tiled, padded block layout.
+ * src device bf16 [groups, n_tokens, D]; dst device bf16 [groups, n_slots, D];
+ * slot_token device int64 [n_slots] with entries < n_tokens.
+ * (PR #1408: the tile permutation plus non-pad placement the metadata
+ * describes.)
+ */
+int vsa_gather_tokens(const void* src, void* dst, const int64_t* slot_token, int64_t n_tokens,
+                      int64_t n_slots, int64_t groups, int D, void* stream);
+
+/*
+ * vsa_scatter_tokens -- dst[g, slot_token[s], :] = src[g, s, :] for every
+ * slot with slot_token[s] >= 0: the inverse of vsa_gather_tokens on the real
+ * tokens.  Same argument meanings; dst is [groups, n_tokens, D].
+ */
+int vsa_scatter_tokens(const void* src, void* dst, const int64_t* slot_token, int64_t n_tokens,
+                       int64_t n_slots, int64_t groups, int D, void* stream);
+
+/* ======================================================================== *
+ * diagnostics
+ * ======================================================================== */
+
+/*
+ * vsa_selftest_umma -- run the two tensor-core products of the sparse kernel
+ * once on operands in global memory, to check shared-memory layouts in
+ * isolation.  mode 0: c[128][64] = a[128][D] * b[64][D]^T (fp32), the
+ * transposed-score product; mode 1: c[D][64] = a[128][D]^T * b[128][64], the
+ * transposed-output product.  a, b device bf16; c device fp32.  D 64 or 128.
+ */
+int vsa_selftest_umma(int mode, int D, const void* a, const void* b, float* c, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H_ */

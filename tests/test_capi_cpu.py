@@ -1,0 +1,144 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/vsa.h declares, rejects bad arguments on the host before launching
+anything, and its host metadata routine matches the oracle bit for bit."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vsa.h")
+
+
+def _lib():
+    from block_sparse_attention_15_b200 import binding
+    if not os.path.exists(binding.LIB_PATH):
+        from block_sparse_attention_15_b200 import build
+        build.build()
+    return binding.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+char\s*\*|int|size_t)\s+([a-z_0-9]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("vsa_forward", "block_sparse_attn_from_indices", "block_sparse_attn_varlen",
+                     "build_vsa_metadata", "vsa_forward_workspace_size", "vsa_get_device_status"):
+        assert required in names
+
+
+@pytest.mark.parametrize("name", declared_functions())
+def test_symbol_exported(name):
+    lib = _lib()
+    assert hasattr(lib, name), f"{name} declared in vsa.h but not exported"
+
+
+def test_exports_are_c_symbols():
+    _lib()
+    from block_sparse_attention_15_b200 import binding
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in declared_functions():
+        assert name in exported, f"{name} is not an unmangled exported symbol"
+
+
+def test_binding_signatures_cover_header():
+    from block_sparse_attention_15_b200 import binding
+    assert set(declared_functions()) == set(binding.SIGNATURES)
+
+
+def test_status_strings():
+    lib = _lib()
+    assert lib.vsa_status_string(0) == b"ok"
+    assert b"range" in lib.vsa_status_string(6)
+    assert lib.vsa_abi_version() >> 16 == 1
+
+
+def _fwd(lib, **kw):
+    args = dict(q=1, k=1, v=1, gate=None, qbs=None, kbs=None, B=1, H=1, Sq=64, Skv=64, D=128,
+                topk=1, scale=0.0, out=1, idx=1, num=1, stride=1, out_c=None, ws=None, wsb=0,
+                stream=None)
+    args.update(kw)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.vsa_forward(v(args["q"]), v(args["k"]), v(args["v"]), v(args["gate"]), v(args["qbs"]),
+                           v(args["kbs"]), args["B"], args["H"], args["Sq"], args["Skv"], args["D"],
+                           args["topk"], args["scale"], v(args["out"]), v(args["idx"]),
+                           v(args["num"]), args["stride"], v(args["out_c"]), v(args["ws"]),
+                           args["wsb"], None)
+
+
+def test_forward_host_argument_checks():
+    """Bad arguments come back as status codes before any CUDA call."""
+    lib = _lib()
+    fake = 1 << 20  # never dereferenced: every case fails on the host
+    base = dict(q=fake, k=fake, v=fake, out=fake, idx=fake, num=fake)
+    assert _fwd(lib, **{**base, "q": None}) == 1                       # null input
+    assert _fwd(lib, **base, D=96) == 3                                 # unsupported head dim
+    assert _fwd(lib, **base, Sq=100) == 2                               # not 64 * n
+    assert _fwd(lib, **base, topk=0) == 1                               # topk >= 1
+    assert _fwd(lib, **base, Sq=64 * 4, Skv=64 * 4, topk=3, stride=2) == 2  # stride < k
+    assert _fwd(lib, **base, B=0) == 1                                  # empty batch
+    assert _fwd(lib, **base, Sq=64 * 4096) == 3                         # above VSA_MAX_BLOCKS
+    assert _fwd(lib, **{**base, "q": fake + 2}) == 1                    # misaligned
+    assert _fwd(lib, **base) == 7                                       # no workspace
+    assert _fwd(lib, **base, ws=fake + 64, wsb=1 << 30) == 7            # misaligned workspace
+
+
+def test_varlen_host_argument_checks():
+    lib = _lib()
+    from block_sparse_attention_15_b200.binding import _P32
+    fake = ctypes.c_void_p(1 << 20)
+
+    def call(cu_q, cu_kv, n, qs=None, qcb=None):
+        a = np.asarray(cu_q, np.int32)
+        b = np.asarray(cu_kv, np.int32)
+        qs_a = None if qs is None else np.asarray(qs, np.int32)
+        qcb_a = None if qcb is None else np.asarray(qcb, np.int32)
+        p = lambda x: None if x is None else x.ctypes.data_as(_P32)
+        return lib.block_sparse_attn_varlen(fake, fake, fake, p(a), p(b), p(qs_a), p(qcb_a), None,
+                                            None, n, 2, 128, fake, fake, 4, 0.0, fake, None, None,
+                                            None, None, 0, None)
+
+    assert call([0], [0], 0) == 2                                 # empty batch
+    assert call([0, 64, 64], [0, 64, 128], 2) == 2                # zero-token sequence
+    assert call([1, 64], [0, 64], 1) == 2                         # cu_seqlens must start at 0
+    assert call([0, 100], [0, 64], 1, qs=[64, 30], qcb=[0, 2]) == 2   # sizes must sum to length
+    assert call([0, 100], [0, 64], 1, qs=[64, 36, 0], qcb=[0, 3]) == 8  # size 0 not allowed
+    assert call([0, 100], [0, 64], 1, qs=[64, 36]) == 1           # sizes need per-seq counts
+    assert call([0, 100], [0, 64], 1) == 7                        # valid, but no workspace
+
+
+@pytest.mark.parametrize("shape,tile", [((9, 30, 52), (4, 4, 4)), ((5, 5, 5), (4, 4, 4)),
+                                        ((8, 4, 12), (4, 4, 4)), ((3, 7, 10), (2, 4, 8)),
+                                        ((1, 1, 1), (4, 4, 4))])
+def test_metadata_matches_oracle(shape, tile):
+    from block_sparse_attention_15_b200 import build_vsa_metadata
+    from oracle import vsa_oracle as O
+    got = build_vsa_metadata(*shape, tile=tile)
+    want = O.build_vsa_metadata(*shape, tile=tile)
+    for key in ("tile_partition_indices", "reverse_tile_partition_indices",
+                "variable_block_sizes", "non_pad_index"):
+        assert np.array_equal(got[key], want[key]), key
+    assert got["n_tiles"] == want["n_tiles"]
+    # the slot map is the non-pad scatter of the partition
+    slot = np.full(want["n_tiles"] * want["max_block_size"], -1, dtype=np.int64)
+    slot[want["non_pad_index"]] = want["tile_partition_indices"]
+    assert np.array_equal(got["slot_token"], slot)
+
+
+def test_metadata_rejects_bad_tiles():
+    lib = _lib()
+    n = ctypes.c_int32(0)
+    assert lib.build_vsa_metadata(4, 4, 4, 8, 4, 4, None, None, None, None, None,
+                                  ctypes.byref(n)) == 1          # tile volume 128 > 64
+    assert lib.build_vsa_metadata(0, 4, 4, 4, 4, 4, None, None, None, None, None,
+                                  ctypes.byref(n)) == 1
