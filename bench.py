@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""VSA forward benchmark on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload h3]
+    python bench.py --impl reference ...        # the CPU oracle, as a baseline
+
+One step = one whole VSA forward (pool -> coarse attention + top-k ->
+block-sparse attention with the fused gated combine) over one batch of seeded
+synthetic bf16 inputs already resident in HBM.  Default workload: the
+H3-like shape B=1, H=56, D=128, S=15488 (242 blocks of 64), top 20% = 48 KV
+blocks per query block, gated.  Metric: effective TFLOP/s over the selected
+64x64 tiles (4 * 64 * 64 * D FLOPs per tile) and ms per forward.
+
+With N GPUs (torchrun, one process per GPU) every rank runs its own copy of
+the workload (the forward has no exchange step: heads, batches and sequences
+are independent), so per-GPU work is fixed and the scaling is weak; the time
+is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_15_b200 import inputs as I  # noqa: E402
+
+METRIC = "VSA fwd ms & effective TFLOPS (selected tiles) at H=56,D=128,S=15488,topk 20%"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2**20
+SPARSE_SOURCES = ["block_sparse_attention_15_b200/csrc/sparse_fwd.cu",
+                  "block_sparse_attention_15_b200/csrc/vsa_device.cuh"]
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+def make_workload(name: str) -> I.Workload:
+    if name == "tiny":
+        return I.workload_tiny()
+    if name == "h3":
+        return I.workload_h3()
+    m = re.fullmatch(r"long(\d+)(-ungated)?", name)
+    if m:
+        return I.workload_long(int(m.group(1)) / 100.0, gated=m.group(2) is None)
+    if name == "video":
+        from block_sparse_attention_15_b200 import binding
+        meta = binding.build_vsa_metadata(9, 30, 52)
+        sizes = [int(s) for s in meta["variable_block_sizes"]]
+        wl = I.Workload("video-tiled: 9x30x52 latent (14040 tokens) in 4x4x4 tiles, B1 H12 D128, "
+                        "top 25% gated", 1, 12, 128, sizes, sizes,
+                        I.topk_count(0.25, len(sizes)), True, 1002)
+        wl.extra["meta"] = meta
+        return wl
+    raise ValueError(f"unknown workload {name}")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the block-sparse kernel from the committed ncu
+    summary, if the kernel sources still hash to what was profiled."""
+    path = os.path.join(ROOT, "profiles", "sparse_fwd_h3.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_t = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    m_h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    if not (m_t and m_h):
+        return None
+    h = hashlib.sha256()
+    for rel in SPARSE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return int(m_t.group(1)) if h.hexdigest() == m_h.group(1) else None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", ident], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except Exception:  # noqa: BLE001 - clocks are best effort
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.06)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons, power = [], [], set(), []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count() or 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def oracle_sample(wl: I.Workload, q, k, v, gate, head: int, n_items: int):
+    """Run the oracle's whole forward for one head restricted to the first
+    n_items query blocks; return (seconds, selected-tile FLOPs)."""
+    from oracle import vsa_oracle as O
+    t0 = time.perf_counter()
+    qn = q[:, head:head + 1].float().numpy()
+    kn = k[:, head:head + 1].float().numpy()
+    vn = v[:, head:head + 1].float().numpy()
+    gn = None if gate is None else gate[:, :, head:head + 1].float().numpy()
+    items = [(0, 0, a) for a in range(min(n_items, wl.nq))]
+    O.vsa_forward(qn, kn, vn, gn, wl.q_block_sizes, wl.kv_block_sizes, wl.topk, items=items)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * 64 * 64 * wl.D * min(wl.topk, wl.nkv) * len(items)
+    return dt, flops
+
+
+def cpu_baseline(wl, q, k, v, gate, budget_s=15.0):
+    total_t, total_f, heads, items = 0.0, 0.0, 0, 0
+    h = 0
+    while total_t < budget_s and h < wl.H:
+        dt, fl = oracle_sample(wl, q, k, v, gate, h, wl.nq)
+        total_t += dt
+        total_f += fl
+        heads += 1
+        items += wl.nq
+        h += 1
+    return {"value": total_f / total_t / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 numpy oracle, whole forward of {heads} head(s) x {wl.nq} query blocks "
+                      f"of this workload ({total_t:.1f} s on the host cores)"}
+
+
+# ---------------------------------------------------------------------------
+# inputs
+# ---------------------------------------------------------------------------
+def host_inputs(wl: I.Workload):
+    Sq, Skv = 64 * wl.nq, 64 * wl.nkv
+    if "meta" in wl.extra:
+        meta = wl.extra["meta"]
+        N = int(sum(wl.q_block_sizes))
+        slot = torch.from_numpy(meta["slot_token"])
+        toks = [I.normal_bf16((wl.B, wl.H, N, wl.D), wl.seed, s) for s in range(3)]
+        padded = []
+        for t in toks:
+            x = torch.zeros((wl.B, wl.H, Sq, wl.D), dtype=torch.bfloat16)
+            real = slot >= 0
+            x[:, :, real] = t[:, :, slot[real]]
+            padded.append(x)
+        q, k, v = padded
+    else:
+        q = I.padded_normal_bhsd(wl.B, wl.H, wl.q_block_sizes, wl.D, wl.seed, I.STREAM_Q)
+        k = I.padded_normal_bhsd(wl.B, wl.H, wl.kv_block_sizes, wl.D, wl.seed, I.STREAM_K)
+        v = I.padded_normal_bhsd(wl.B, wl.H, wl.kv_block_sizes, wl.D, wl.seed, I.STREAM_V)
+    gate = I.gate_bf16((wl.B, Sq, wl.H, wl.D), wl.seed) if wl.gated else None
+    return q, k, v, gate
+
+
+def config_of(wl: I.Workload, flushed: bool) -> dict:
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "D": wl.D, "seq_q_slots": 64 * wl.nq,
+            "seq_kv_slots": 64 * wl.nkv, "q_blocks": wl.nq, "kv_blocks": wl.nkv,
+            "topk": min(wl.topk, wl.nkv), "gated": wl.gated,
+            "selected_tiles_per_gpu": wl.selected_tiles,
+            "l2": "L2 flushed between steps" if flushed else
+                  "inputs larger than L2 (126 MB) every step", "per_gpu_work": "fixed (weak)"}
+
+
+# ---------------------------------------------------------------------------
+# the two arms
+# ---------------------------------------------------------------------------
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    q, k, v, gate = host_inputs(wl)
+    items = max(1, args.ref_items)
+    for _ in range(args.warmup):
+        oracle_sample(wl, q, k, v, gate, 0, items)
+    times, flops = [], 0.0
+    for s in range(args.steps):
+        dt, fl = oracle_sample(wl, q, k, v, gate, s % wl.H, items)
+        times.append(dt)
+        flops += fl
+    total = sum(times)
+    val = flops / total / 1e12
+    sample = (f"fp64 numpy oracle on the host cores: per step, one head's pool + coarse + top-k "
+              f"and the sparse attention + combine of its first {items} query blocks")
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(wl, False),
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": _blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, wl):
+    import torch.distributed as dist
+    from block_sparse_attention_15_b200 import binding as vsa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    q_h, k_h, v_h, g_h = host_inputs(wl)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    gate = None if g_h is None else g_h.to(dev)
+    in_bytes = sum(t.numel() * 2 for t in (q, k, v) + ((gate,) if gate is not None else ()))
+    flush = None
+    if 2 * in_bytes < 2 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    qbs = None if all(s == 64 for s in wl.q_block_sizes) else torch.tensor(wl.q_block_sizes, dtype=torch.int32, device=dev)
+    kbs = None if all(s == 64 for s in wl.kv_block_sizes) else torch.tensor(wl.kv_block_sizes, dtype=torch.int32, device=dev)
+    k_eff = min(wl.topk, wl.nkv)
+    out = torch.empty_like(q)
+    ws_bytes = vsa.lib().vsa_forward_workspace_size(wl.B, wl.H, wl.nq, wl.nkv, wl.D)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        if flush is not None:
+            flush.fill_(1)
+        vsa.vsa_forward(q, k, v, gate, qbs, kbs, topk=wl.topk, out=out, workspace=ws)
+
+    for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
+        step()
+    torch.cuda.synchronize(dev)
+    vsa.check_device_status()
+
+    # timed region: per-step events plus events around each kernel
+    K = args.steps
+    ev_step = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    ev_k = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local)
+    ev_step[0].record(stream)
+    for i in range(K):
+        vsa.set_profile_events(ev_k[i])
+        step()
+    ev_step[K].record(stream)
+    vsa.set_profile_events(None)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    status = vsa.get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+    total_ms = ev_step[0].elapsed_time(ev_step[K])
+    k_pool = sum(e[0].elapsed_time(e[1]) for e in ev_k) / K
+    k_coarse = sum(e[1].elapsed_time(e[2]) for e in ev_k) / K
+    k_sparse = sum(e[2].elapsed_time(e[3]) for e in ev_k) / K
+    t = torch.tensor([total_ms, k_sparse], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, k_sparse_max = float(t[0]), float(t[1])
+    ms_per_step = total_ms / K
+    flops_gpu = wl.flops
+    value = world * flops_gpu / (ms_per_step * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers (pinned)
+    E = max(1, min(K, args.e2e_steps))
+    pin = [x.pin_memory() for x in (q_h, k_h, v_h) + ((g_h,) if g_h is not None else ())]
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dg = None if gate is None else torch.empty_like(gate)
+
+    def e2e_step():
+        dq.copy_(pin[0], non_blocking=True)
+        dk.copy_(pin[1], non_blocking=True)
+        dv.copy_(pin[2], non_blocking=True)
+        if dg is not None:
+            dg.copy_(pin[3], non_blocking=True)
+        vsa.vsa_forward(dq, dk, dv, dg, qbs, kbs, topk=wl.topk, out=out, workspace=ws)
+        out_h.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    te = torch.tensor([e0.elapsed_time(e1) / E], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te[0])
+    h2d = sum(x.numel() * x.element_size() for x in pin)
+    d2h = out_h.numel() * out_h.element_size()
+    vsa.check_device_status()
+
+    if rank == 0:
+        peaks, peak_kind = load_peaks()
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        achieved = flops_gpu / (k_sparse * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_of(wl, flush is not None),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": profiled_traffic(),
+                         "kernel": "sparse_fwd_kernel (block-sparse attention + fused gated combine)",
+                         "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS)",
+                         "frac_of_sustained": achieved / sustained},
+            "kernels_ms": {"pool": k_pool, "coarse_topk": k_coarse, "sparse_combine": k_sparse,
+                           "sparse_combine_max_over_ranks": k_sparse_max},
+            "forward_frac_of_peak": (flops_gpu / (ms_per_step * 1e-3) / 1e12) / peak,
+            "e2e": {"value": world * flops_gpu / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 3 * K,
+            "clocks": clocks,
+        }
+        # pooling streams q, k and v once: algorithmic bytes = their real tokens
+        pool_bytes = 2 * wl.B * wl.H * wl.D * (sum(wl.q_block_sizes) + 2 * sum(wl.kv_block_sizes))
+        line["pool_gbs"] = pool_bytes / (k_pool * 1e-3) / 1e9
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, q_h, k_h, v_h, g_h, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="h3")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-items", type=int, default=24,
+                    help="query blocks per reference-arm step (bounded CPU sample)")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (smaller cases for profiler captures)")
+    args = ap.parse_args(argv)
+    wl = make_workload(args.workload)
+    if args.heads > 0:
+        wl.H = args.heads
+        wl.name += f" [H overridden to {args.heads}]"
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

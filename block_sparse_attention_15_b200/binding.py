@@ -56,6 +56,7 @@ SIGNATURES = {
     "vsa_scatter_tokens": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int64, _c_int64,
                                     _c_int64, _c_int, _c_void_p]),
     "vsa_selftest_umma": (_c_int, [_c_int, _c_int, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "vsa_set_profile_events": (_c_int, [ctypes.POINTER(_c_void_p)]),
 }
 
 _LIB = None
@@ -338,6 +339,17 @@ def selftest_umma(mode: int, a, b, *, stream=None):
     _check("vsa_selftest_umma", lib().vsa_selftest_umma(mode, D, _ptr(a), _ptr(b), _ptr(c),
                                                         _stream(stream)))
     return c
+
+
+def set_profile_events(events):
+    """Record four torch.cuda.Event objects around vsa_forward's kernels
+    (before pool, after pool, after coarse/top-k, after block-sparse), or
+    switch the hook off with None."""
+    if events is None:
+        _check("vsa_set_profile_events", lib().vsa_set_profile_events(None))
+        return
+    arr = (_c_void_p * 4)(*[e.cuda_event for e in events])
+    _check("vsa_set_profile_events", lib().vsa_set_profile_events(arr))
 
 
 def default_scale(D: int) -> float:

@@ -33,6 +33,14 @@ static inline bool aligned16(const void* p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
 
+// Optional timing events recorded around the kernels of vsa_forward.
+static cudaEvent_t g_prof_events[4] = {nullptr, nullptr, nullptr, nullptr};
+static bool g_prof_on = false;
+
+static inline void prof_record(int i, cudaStream_t st) {
+  if (g_prof_on) cudaEventRecord(g_prof_events[i], st);
+}
+
 static inline float resolve_scale(float scale, int D) {
   return scale > 0.f ? scale : 1.0f / sqrtf((float)D);
 }
@@ -125,8 +133,10 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
   pp.kc = kc;
   pp.vc = vc;
   pp.status = status;
+  prof_record(0, st);
   int rc = launch_pool(pp, D, st);
   if (rc != VSA_OK) return rc;
+  prof_record(1, st);
 
   const float sc = resolve_scale(scale, D);
   CoarseParams cp;
@@ -144,6 +154,7 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
   cp.out_c = oc;
   rc = launch_coarse_topk(cp, D, st);
   if (rc != VSA_OK) return rc;
+  prof_record(2, st);
 
   SparseParams sp;
   memset(&sp, 0, sizeof(sp));
@@ -165,8 +176,11 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
   sp.scale_log2 = sc * 1.4426950408889634f;
   sp.varlen = 0;
   sp.status = status;
-  return launch_sparse(sp, q, k, v, (long long)B * H * Sq_pad, (long long)B * H * Skv_pad, D,
-                       /*combine=*/true, /*gated=*/gate != nullptr, st);
+  rc = launch_sparse(sp, q, k, v, (long long)B * H * Sq_pad, (long long)B * H * Skv_pad, D,
+                     /*combine=*/true, /*gated=*/gate != nullptr, st);
+  if (rc != VSA_OK) return rc;
+  prof_record(3, st);
+  return VSA_OK;
 }
 
 // ---------------------------------------------------------------------------
@@ -406,6 +420,19 @@ int vsa_scatter_tokens(const void* src, void* dst, const int64_t* slot_token, in
   if (!aligned16(src) || !aligned16(dst)) return VSA_ERR_INVALID_ARG;
   return launch_gather_tokens(src, dst, slot_token, n_tokens, n_slots, groups, D, true,
                               static_cast<cudaStream_t>(stream));
+}
+
+int vsa_set_profile_events(void* const* events) {
+  if (!events) {
+    g_prof_on = false;
+    return VSA_OK;
+  }
+  for (int i = 0; i < 4; ++i) {
+    if (!events[i]) return VSA_ERR_INVALID_ARG;
+  }
+  for (int i = 0; i < 4; ++i) g_prof_events[i] = static_cast<cudaEvent_t>(events[i]);
+  g_prof_on = true;
+  return VSA_OK;
 }
 
 int vsa_selftest_umma(int mode, int D, const void* a, const void* b, float* c, void* stream) {

@@ -272,6 +272,17 @@ int vsa_scatter_tokens(const void* src, void* dst, const int64_t* slot_token, in
  * ======================================================================== */
 
 /*
+ * vsa_set_profile_events -- timing hook for vsa_forward.  `events` points to
+ * four cudaEvent_t handles (host array) or is NULL to switch the hook off.
+ * While set, every vsa_forward call records events[0] on its stream before
+ * the pooling kernel, events[1] after it, events[2] after the coarse/top-k
+ * kernel and events[3] after the block-sparse kernel, so a caller can time
+ * each kernel with cudaEventElapsedTime.  The handles are copied; the setting
+ * is process-wide and not thread-safe.
+ */
+int vsa_set_profile_events(void* const* events);
+
+/*
  * vsa_selftest_umma -- run the two tensor-core products of the sparse kernel
  * once on operands in global memory, to check shared-memory layouts in
  * isolation.  mode 0: c[128][64] = a[128][D] * b[64][D]^T (fp32), the
