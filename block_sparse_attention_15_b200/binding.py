@@ -348,6 +348,9 @@ def set_profile_events(events):
     if events is None:
         _check("vsa_set_profile_events", lib().vsa_set_profile_events(None))
         return
+    for e in events:
+        if not e.cuda_event:  # torch creates the handle on first record
+            e.record()
     arr = (_c_void_p * 4)(*[e.cuda_event for e in events])
     _check("vsa_set_profile_events", lib().vsa_set_profile_events(arr))
 
