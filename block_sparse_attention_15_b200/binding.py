@@ -43,6 +43,9 @@ SIGNATURES = {
     "vsa_forward": (_c_int, [_c_void_p] * 4 + [_c_void_p, _c_void_p] + [_c_int] * 6 +
                     [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p,
                      _c_size_t, _c_void_p]),
+    "vsa_forward_noalloc": (_c_int, [_c_void_p] * 4 + [_c_void_p, _c_void_p] + [_c_int] * 6 +
+                            [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p,
+                             _c_void_p]),
     "block_sparse_attn_from_indices": (_c_int, [_c_void_p] * 7 + [_c_int] * 6 +
                                        [_c_float, _c_void_p, _c_void_p]),
     "block_sparse_attn_varlen_workspace_size": (_c_size_t, [_c_int] * 3),

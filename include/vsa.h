@@ -130,6 +130,40 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
                 int32_t* q2k_idx, int32_t* q2k_num, int idx_stride, float* out_c,
                 void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * vsa_forward_noalloc -- vsa_forward for callers that cannot allocate device
+ * memory while they run (a serving loop under a fixed memory budget, where a
+ * cudaMalloc can synchronise the device and stall every stream; a plugin
+ * whose host application owns all device memory).  The pages have no
+ * counterpart to this entry point; it exists for such callers only.
+ *
+ * Same arguments, results and launches as vsa_forward, minus the workspace:
+ * the scratch (pooled q/k/v and, when out_c is NULL, the coarse output, all
+ * fp32) lives in one fixed array of VSA_NOALLOC_SCRATCH_BYTES that the
+ * library's device image defines.  Every GPU that uses the library holds that
+ * array until the process exits.  The call allocates and frees nothing.
+ *
+ * - Sizes whose scratch exceeds the array, i.e. when
+ *     4*B*H*D*(n_q_blocks + n_kv_blocks) * 2 (each term rounded up to 256 B)
+ *   is above VSA_NOALLOC_SCRATCH_BYTES, return VSA_ERR_WORKSPACE before
+ *   anything is launched.  (The H3-like shape B=1, H=56, D=128, 242 + 242
+ *   blocks needs 27.8 MB and fits.)
+ * - The first call on each device looks the array's device address up and
+ *   may load the library's device image there; make that first call before
+ *   any stream capture.
+ * - All calls on a device share the one array.  Every region of it is
+ *   written in full before it is read within a call, so nothing has to be
+ *   cleared between calls, but two calls whose kernels overlap on the GPU
+ *   (different streams, or different host threads) race on the array and
+ *   give wrong results: serialise them, e.g. on one stream.
+ */
+#define VSA_NOALLOC_SCRATCH_BYTES (32u << 20) /* 32 MiB */
+int vsa_forward_noalloc(const void* q, const void* k, const void* v, const void* gate,
+                        const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B, int H,
+                        int Sq_pad, int Skv_pad, int D, int topk, float scale, void* out,
+                        int32_t* q2k_idx, int32_t* q2k_num, int idx_stride, float* out_c,
+                        void* stream);
+
 /* ======================================================================== *
  * a4: block-sparse attention from indices
  * ======================================================================== */
