@@ -8,25 +8,30 @@
 // q2k_idx[a][0 : q2k_num[a]], then out = out_c[a] * gate + out_s with out_c
 // held per block and never expanded.
 //
-// How (sm_100a): one CTA per (query block, head, batch), 6 warps.
-//   warp 0      TMA producer: Q once, then the selected K/V tiles two at a
-//               time into a 2-stage ring (128-byte swizzle, no multicast).
-//   warp 1      TMEM owner and MMA issuer (one thread).
-//   warps 2-5   softmax, then the epilogue.
-// Each step takes a PAIR of selected KV tiles so that both tensor-core
-// products run at M = 128 although a query block has only 64 rows:
+// How (sm_100a).  A query block has 64 rows but tcgen05 runs at full rate
+// with M = 128, so every step takes a PAIR of selected KV tiles and both
+// products are transposed:
 //   S^T[128 kv][64 q] = K2[128 kv][D] . Q[64 q][D]^T           (K-major A, B)
 //   O^T[D][64 q]     += V2[128 kv][D]^T . P^T[128 kv][64 q]      (MN-major A, B)
-// S^T and O^T live in TMEM (fp32).  TMEM lane = KV row for S^T, so the
-// softmax thread of lane L owns one key row and all 64 query columns; the
-// per-query running max m[q] is kept identical in every softmax thread and
-// only refreshed (exact column max across lanes) on the first pair and when
-// some logit exceeds it by more than 2^8 -- rare, and then O^T and the row
-// sums are rescaled.  Row sums l[q] are accumulated per lane and reduced
-// across lanes once at the end.  P^T is written to shared memory in bf16 as
-// the B operand of the second product.  S^T is double-buffered in TMEM so the
-// tensor core computes S(i+1) and PV(i-1) while the softmax warps work on
-// S(i).
+// TMEM lane = key row of S^T (softmax needs no cross-thread work per
+// element) and lane = head dim of O^T.  S^T is double-buffered in TMEM and
+// O^T too, so the epilogue of one work item overlaps the next item's loop.
+//
+// Persistent grid: one CTA per SM walks the work items (query block, head,
+// batch) b-major, h, a-minor with stride gridDim.x.  512 threads:
+//   warp 0       K producer: Q of each item (2 buffers) and K tile pairs into
+//                a 3-stage ring, with each pair's key counts (TMA, 128-byte
+//                swizzle, no multicast)
+//   warp 1       TMEM owner and MMA issuer (one thread)
+//   warp 2       V producer: V tile pairs into a 2-stage ring
+//   warp 3       idle
+//   warps 4-7    softmax for query columns 0..31
+//   warps 8-11   softmax for query columns 32..63
+//   warps 12-15  epilogue: O^T / l, the gated combine, bf16 stores
+// The running max per query column is exact after an item's first pair
+// (column reduction across lanes) and refreshed only when a logit exceeds it
+// by more than 2^8 (warp vote), then O^T and the partial sums are rescaled.
+// Row sums are accumulated per lane and reduced across lanes once per item.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -38,47 +43,54 @@
 
 namespace vsa {
 
-constexpr int kSparseThreads = 192;
-constexpr int kMaxSel = VSA_MAX_BLOCKS;
-constexpr uint32_t kTmemCols = 256;   // S buffers at 0 and 64, O^T at 128
+constexpr int kThreads = 512;
+constexpr uint32_t kTmemCols = 256;   // S^T buffers at 0 and 64, O^T buffers at 128 and 192
 constexpr uint32_t kTmemO = 128;
 
 template <int D>
-struct SparseSmem {
-  static constexpr int DH = D / 64;                         // 64-element d halves
-  static constexpr uint32_t kQBytes = 64u * D * 2u;         // one 64-row tile
-  static constexpr uint32_t kTileBytes = 64u * D * 2u;
-  static constexpr uint32_t kKBytes = 2u * kTileBytes;      // two tiles, M = 128
-  static constexpr uint32_t kStageBytes = 2u * kKBytes;     // K2 + V2
-  static constexpr uint32_t kPBytes = 128u * 64u * 2u;      // P^T, bf16
+struct Layout {
+  static constexpr int DH = D / 64;                        // 64-element head-dim halves
+  static constexpr int NK = 3;                             // K ring stages (tile pairs)
+  static constexpr int NV = 2;                             // V ring stages
+  static constexpr uint32_t kQ = 64u * D * 2u;             // one 64-row Q tile
+  static constexpr uint32_t kK2 = 2u * 64u * D * 2u;       // a pair of K tiles (M = 128)
+  static constexpr uint32_t kV2 = kK2;
+  static constexpr uint32_t kP = 128u * 64u * 2u;          // P^T in bf16
   static constexpr uint32_t kQOff = 0;
-  static constexpr uint32_t kStageOff = kQBytes;
-  static constexpr uint32_t kPOff = kStageOff + 2u * kStageBytes;
-  static constexpr uint32_t kSelRowOff = kPOff + 2u * kPBytes;
-  static constexpr uint32_t kSelLenOff = kSelRowOff + 4u * kMaxSel;
-  static constexpr uint32_t kRedOff = kSelLenOff + kMaxSel;     // [4][64] f32
-  static constexpr uint32_t kFinOff = kRedOff + 4u * 64u * 4u;  // [64] f32
-  static constexpr uint32_t kMOff = kFinOff + 64u * 4u;        // [64] running max (log2 units)
+  static constexpr uint32_t kKOff = kQOff + 2u * kQ;
+  static constexpr uint32_t kVOff = kKOff + NK * kK2;
+  static constexpr uint32_t kPOff = kVOff + NV * kV2;
+  static constexpr uint32_t kRedOff = kPOff + kP;               // [2 groups][4 warps][32] f32
+  static constexpr uint32_t kFinOff = kRedOff + 2u * 4u * 32u * 4u;  // [64] f32
+  static constexpr uint32_t kMOff = kFinOff + 64u * 4u;         // [64] running max (log2 units)
   static constexpr uint32_t kAlphaOff = kMOff + 64u * 4u;       // [64] rescale factors
-  static constexpr uint32_t kInvLOff = kAlphaOff + 64u * 4u;    // [64] 1 / row sum
-  static constexpr uint32_t kFlagOff = kInvLOff + 64u * 4u;     // [2][4] int
-  static constexpr uint32_t kBarOff = kFlagOff + 64u;           // mbarriers
-  static constexpr uint32_t kNumBars = 13;
-  static constexpr uint32_t kMiscOff = kBarOff + 8u * kNumBars;  // tmem addr, abort
+  static constexpr uint32_t kInvLOff = kAlphaOff + 64u * 4u;    // [2][64] 1 / row sum per O buffer
+  static constexpr uint32_t kFlagOff = kInvLOff + 2u * 64u * 4u;  // [2 groups][2][4] int
+  static constexpr uint32_t kKMetaOff = kFlagOff + 64u;         // [NK] int2: key counts of a pair
+  static constexpr uint32_t kBarOff = kKMetaOff + 32u;
+  // barriers
+  static constexpr int kQFull = 0, kQEmpty = 2, kKFull = 4, kKEmpty = kKFull + NK,
+                       kVFull = kKEmpty + NK, kVEmpty = kVFull + NV, kSFull = kVEmpty + NV,
+                       kSEmpty = kSFull + 2, kPFull = kSEmpty + 2, kPEmpty = kPFull + 1,
+                       kOFull = kPEmpty + 1, kOEmpty = kOFull + 2, kLFull = kOEmpty + 2,
+                       kNumBars = kLFull + 2;
+  static constexpr uint32_t kMiscOff = kBarOff + 8u * kNumBars;  // tmem address, abort flag
   static constexpr uint32_t kBytes = kMiscOff + 16u;
-  static constexpr uint32_t kAlloc = kBytes + 1024u;            // room to align to 1 KB
-  static_assert(kQOff % 1024 == 0 && kStageOff % 1024 == 0 && kPOff % 1024 == 0, "align");
-  static_assert(2u * kStageBytes >= 64u * D * 4u, "epilogue tile reuses the stage ring");
+  static constexpr uint32_t kAlloc = kBytes + 1024u;             // slack to align to 1 KB
+  static_assert(kKOff % 1024 == 0 && kVOff % 1024 == 0 && kPOff % 1024 == 0, "1 KB atoms");
+  static_assert(kAlloc <= 227u * 1024u, "shared memory");
 };
 
-// K2 tile layout: [dh][2 tiles][64 rows][128 B]; V2: [2 tiles][dh][64 rows][128 B].
+// Pair layouts inside a stage.  K2: [dh][2 tiles][64 rows][128 B] (rows of
+// the two tiles contiguous, so the pair is one M = 128 operand).
+// V2: [2 tiles][dh][64 rows][128 B].
 template <int D>
 __device__ __forceinline__ uint32_t k_slot_off(int dh, int tile) {
   return uint32_t(dh) * 16384u + uint32_t(tile) * 8192u;
 }
 template <int D>
 __device__ __forceinline__ uint32_t v_slot_off(int tile, int dh) {
-  return uint32_t(tile) * uint32_t(SparseSmem<D>::DH) * 8192u + uint32_t(dh) * 8192u;
+  return uint32_t(tile) * uint32_t(D / 64) * 8192u + uint32_t(dh) * 8192u;
 }
 
 // S^T[128][64] = K2 . Q^T: M = 128 key rows, N = 64 query rows, K = D.
@@ -121,139 +133,147 @@ __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t chunk) {
   return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
-// Reduce 64 per-thread values column-wise across the 128 softmax threads into
-// fin[0..63] (shared memory, visible to all 128 threads on return).  Warp
-// stage: recursive halving with shuffles, after which lane l holds columns 2l
-// and 2l+1; then the four warps combine through shared memory.
 template <bool IsMax>
 __device__ __forceinline__ float red_op(float a, float b) {
   return IsMax ? fmaxf(a, b) : a + b;
 }
 
+// Column-wise reduction of 32 per-thread values over the 128 threads of one
+// softmax group; the 32 results land in fin[0..31] (shared memory, visible to
+// the group on return).  Warp stage: recursive halving with shuffles, after
+// which lane l holds column l; then the four warps combine through `red`.
 template <bool IsMax>
-__device__ __forceinline__ void col_reduce64(const float (&v)[64], float* red, float* fin, int wq,
-                                             int lane, int t128) {
-  float a[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const bool hi = lane & 16;
-    const float keep = hi ? v[j + 32] : v[j];
-    const float send = hi ? v[j] : v[j + 32];
-    a[j] = red_op<IsMax>(keep, __shfl_xor_sync(0xffffffffu, send, 16));
-  }
-  float b[16];
+__device__ __forceinline__ void col_reduce32(const float (&v)[32], float* red, float* fin, int wq,
+                                             int lane, int t128, uint32_t bar_id) {
+  float a[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    const bool hi = lane & 8;
-    const float keep = hi ? a[j + 16] : a[j];
-    const float send = hi ? a[j] : a[j + 16];
-    b[j] = red_op<IsMax>(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+    const bool hi = lane & 16;
+    a[j] = red_op<IsMax>(hi ? v[j + 16] : v[j],
+                         __shfl_xor_sync(0xffffffffu, hi ? v[j] : v[j + 16], 16));
   }
-  float c[8];
+  float b[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    const bool hi = lane & 4;
-    const float keep = hi ? b[j + 8] : b[j];
-    const float send = hi ? b[j] : b[j + 8];
-    c[j] = red_op<IsMax>(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+    const bool hi = lane & 8;
+    b[j] = red_op<IsMax>(hi ? a[j + 8] : a[j], __shfl_xor_sync(0xffffffffu, hi ? a[j] : a[j + 8], 8));
   }
-  float d[4];
+  float c[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const bool hi = lane & 2;
-    const float keep = hi ? c[j + 4] : c[j];
-    const float send = hi ? c[j] : c[j + 4];
-    d[j] = red_op<IsMax>(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+    const bool hi = lane & 4;
+    c[j] = red_op<IsMax>(hi ? b[j + 4] : b[j], __shfl_xor_sync(0xffffffffu, hi ? b[j] : b[j + 4], 4));
   }
-  float e[2];
+  float d[2];
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
-    const bool hi = lane & 1;
-    const float keep = hi ? d[j + 2] : d[j];
-    const float send = hi ? d[j] : d[j + 2];
-    e[j] = red_op<IsMax>(keep, __shfl_xor_sync(0xffffffffu, send, 1));
+    const bool hi = lane & 2;
+    d[j] = red_op<IsMax>(hi ? c[j + 2] : c[j], __shfl_xor_sync(0xffffffffu, hi ? c[j] : c[j + 2], 2));
   }
-  *reinterpret_cast<float2*>(red + wq * 64 + 2 * lane) = make_float2(e[0], e[1]);
-  named_barrier_sync(2, 128);
-  if (t128 < 64) {
-    fin[t128] = red_op<IsMax>(red_op<IsMax>(red[t128], red[64 + t128]),
-                              red_op<IsMax>(red[128 + t128], red[192 + t128]));
+  const bool hi = lane & 1;
+  const float e = red_op<IsMax>(hi ? d[1] : d[0], __shfl_xor_sync(0xffffffffu, hi ? d[0] : d[1], 1));
+  red[wq * 32 + lane] = e;
+  named_barrier_sync(bar_id, 128);
+  if (t128 < 32) {
+    fin[t128] = red_op<IsMax>(red_op<IsMax>(red[t128], red[32 + t128]),
+                              red_op<IsMax>(red[64 + t128], red[96 + t128]));
   }
-  named_barrier_sync(2, 128);
+  named_barrier_sync(bar_id, 128);
+}
+
+// One work item: query block a of head h of batch b.
+struct Item {
+  int a, h, b;
+  long long group;     // b * H + h
+  int num;             // selected entries, clamped to [0, idx_stride]
+  int q_len;           // real query rows
+  long long q_tok;     // first token row of the block within its group
+  int kv_base, kv_count;
+};
+
+__device__ __forceinline__ Item load_item(const SparseParams& p, long long it) {
+  Item x;
+  x.a = (int)(it % p.nq);
+  const long long t = it / p.nq;
+  x.h = (int)(t % p.H);
+  x.b = (int)(t / p.H);
+  x.group = t;
+  const int num = p.q2k_num[t * p.nq + x.a];
+  x.num = num < 0 ? 0 : (num > p.idx_stride ? p.idx_stride : num);
+  x.q_tok = p.q_tok ? (long long)p.q_tok[x.a] : 64LL * x.a;
+  const int ql = p.q_bs ? p.q_bs[x.a] : 64;
+  x.q_len = ql < 1 ? 0 : (ql > 64 ? 64 : ql);
+  x.kv_base = p.q_kv_base ? p.q_kv_base[x.a] : 0;
+  x.kv_count = p.q_kv_count ? p.q_kv_count[x.a] : p.nkv;
+  return x;
+}
+
+// Report a work item whose count or query block size is out of range.
+__device__ __forceinline__ void check_item(const SparseParams& p, long long it) {
+  const long long t = it / p.nq;
+  const int a = (int)(it % p.nq);
+  const int num = p.q2k_num[t * p.nq + a];
+  if (num < 0 || num > p.idx_stride) set_status(p.status, VSA_ERR_INDEX_RANGE);
+  const int ql = p.q_bs ? p.q_bs[a] : 64;
+  if (ql < 1 || ql > 64) set_status(p.status, VSA_ERR_BLOCK_SIZE);
+}
+
+// Producer helper: for entry j of an item's selection, the row of its first
+// token within the group and its key count (0 for an invalid entry, which is
+// reported and then masked out).
+__device__ __forceinline__ void resolve_entry(const SparseParams& p, const Item& x,
+                                              const int32_t* idx_row, int j, int& row, int& len) {
+  row = 0;
+  len = 0;
+  if (j >= x.num) return;
+  const int c = idx_row[j];
+  if (c < 0 || c >= x.kv_count) {
+    set_status(p.status, VSA_ERR_INDEX_RANGE);
+    return;
+  }
+  const int cg = c + x.kv_base;
+  row = p.kv_tok ? p.kv_tok[cg] : 64 * cg;
+  len = p.kv_bs ? p.kv_bs[cg] : 64;
+  if (len < 1 || len > 64) {
+    set_status(p.status, VSA_ERR_BLOCK_SIZE);
+    len = 0;
+  }
 }
 
 template <int D, bool COMBINE, bool GATED>
-__global__ void __launch_bounds__(kSparseThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const SparseParams p) {
-  using L = SparseSmem<D>;
+  using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  int32_t* sel_row = reinterpret_cast<int32_t*>(smem + L::kSelRowOff);
-  uint8_t* sel_len = smem + L::kSelLenOff;
-  float* red = reinterpret_cast<float*>(smem + L::kRedOff);
-  float* fin = reinterpret_cast<float*>(smem + L::kFinOff);
+  float* red_all = reinterpret_cast<float*>(smem + L::kRedOff);
+  float* fin_all = reinterpret_cast<float*>(smem + L::kFinOff);
   float* m_s = reinterpret_cast<float*>(smem + L::kMOff);
   float* alpha_s = reinterpret_cast<float*>(smem + L::kAlphaOff);
-  float* inv_l_s = reinterpret_cast<float*>(smem + L::kInvLOff);
+  float* inv_l = reinterpret_cast<float*>(smem + L::kInvLOff);
   volatile int* flags = reinterpret_cast<volatile int*>(smem + L::kFlagOff);
+  int2* kmeta = reinterpret_cast<int2*>(smem + L::kKMetaOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* bar_q = bars + 0;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* s_empty = bars + 7;   // [2]
-  uint64_t* p_full = bars + 9;    // [2]
-  uint64_t* pv_done = bars + 11;  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
   const int tid = threadIdx.x;
   const int warp = tid / 32, lane = tid % 32;
-  const int a = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const long long group = (long long)b * p.H + h;
+  const long long n_items = (long long)p.B * p.H * p.nq;
+  const long long it0 = blockIdx.x, it_step = gridDim.x;
 
-  // ---- work item geometry and the selected tiles -------------------------
-  int num = p.q2k_num[group * p.nq + a];
-  if (num < 0 || num > p.idx_stride) {
-    if (tid == 0) set_status(p.status, VSA_ERR_INDEX_RANGE);
-    num = num < 0 ? 0 : p.idx_stride;
-  }
-  const long long q_tok = p.q_tok ? (long long)p.q_tok[a] : 64LL * a;
-  int q_len = p.q_bs ? p.q_bs[a] : 64;
-  if (q_len < 1 || q_len > 64) {
-    if (tid == 0) set_status(p.status, VSA_ERR_BLOCK_SIZE);
-    q_len = q_len < 1 ? 0 : 64;
-  }
-  const int kv_base = p.q_kv_base ? p.q_kv_base[a] : 0;
-  const int kv_count = p.q_kv_count ? p.q_kv_count[a] : p.nkv;
-  const int32_t* idx_row = p.q2k_idx + (group * p.nq + a) * (long long)p.idx_stride;
-  for (int j = tid; j < num; j += kSparseThreads) {
-    const int c = idx_row[j];
-    int row = 0, len = 0;
-    if (c < 0 || c >= kv_count) {
-      set_status(p.status, VSA_ERR_INDEX_RANGE);
-    } else {
-      const int cg = c + kv_base;
-      row = p.kv_tok ? p.kv_tok[cg] : 64 * cg;
-      len = p.kv_bs ? p.kv_bs[cg] : 64;
-      if (len < 1 || len > 64) {
-        set_status(p.status, VSA_ERR_BLOCK_SIZE);
-        len = 0;
-      }
-    }
-    sel_row[j] = row;
-    sel_len[j] = (uint8_t)len;
-  }
   if (tid == 0) {
-    // s_empty and p_full collect one arrival per softmax warp; the rest one
-    // arrival (TMA expect_tx or a tcgen05 commit).
-    for (int i = 0; i < (int)L::kNumBars; ++i) {
-      const bool per_warp = (bars + i == s_empty) || (bars + i == s_empty + 1) ||
-                            (bars + i == p_full) || (bars + i == p_full + 1);
-      mbar_init(bars + i, per_warp ? 4u : 1u);
+    for (int i = 0; i < L::kNumBars; ++i) {
+      uint32_t count = 1;
+      if (i == L::kSEmpty || i == L::kSEmpty + 1 || i == L::kPFull || i == L::kLFull ||
+          i == L::kLFull + 1)
+        count = 8;  // one arrival per softmax warp
+      if (i >= L::kKEmpty && i < L::kKEmpty + L::NK) count = 9;  // MMA commit + 8 softmax warps
+      if (i == L::kOEmpty || i == L::kOEmpty + 1) count = 4;   // epilogue warps
+      mbar_init(bars + i, count);
     }
     *abort_flag = 0;
     mbar_fence_init();
@@ -268,243 +288,337 @@ __global__ void __launch_bounds__(kSparseThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
-  const int npairs = (num + 1) / 2;
-  const uint32_t q_smem = sbase + L::kQOff;
 
-  if (warp == 0) {
-    // ===================== TMA producer =====================
-    if (lane == 0 && npairs > 0) {
-      const uint64_t pol_q = l2_policy_evict_first();
-      const uint64_t pol_kv = l2_policy_evict_last();
-      const int q_row = (int)(group * p.q_rows_per_group + q_tok);
-      mbar_arrive_expect_tx(bar_q, L::kQBytes);
+  if (warp == 0 || warp == 2) {
+    // ===================== producers (whole warp) =====================
+    const bool is_k = (warp == 0);
+    const uint64_t pol_q = l2_policy_evict_first();
+    const uint64_t pol_kv = l2_policy_evict_last();
+    long long gp = 0;  // pair counter over this CTA's items
+    bool ok = true;
+    long long n = 0;
+    for (long long it = it0; ok && it < n_items; it += it_step, ++n) {
+      const Item x = load_item(p, it);
+      const int o = (int)(n & 1);
+      if (is_k) {
+        if (lane == 0) {
+          check_item(p, it);
+          if (n >= 2)
+            ok = mbar_wait(bars + L::kQEmpty + o, (uint32_t)(((n - 2) >> 1) & 1), abort_flag, p.status);
+          if (ok) {
+            mbar_arrive_expect_tx(bars + L::kQFull + o, L::kQ);
+            const int q_row = (int)(x.group * p.q_rows_per_group + x.q_tok);
 #pragma unroll
-      for (int dh = 0; dh < L::DH; ++dh)
-        tma_load_2d(smem + L::kQOff + dh * 8192, &tm_q, bar_q, dh * 64, q_row, pol_q);
-      const long long kv_row0 = group * p.kv_rows_per_group;
-      for (int i = 0; i < npairs; ++i) {
-        const int s = i & 1;
-        if (i >= 2 && !mbar_wait(kv_empty + s, ((i - 2) >> 1) & 1, abort_flag, p.status)) break;
-        const int j0 = 2 * i;
-        const int j1 = (2 * i + 1 < num) ? 2 * i + 1 : 2 * i;
-        const int r0 = (int)(kv_row0 + sel_row[j0]);
-        const int r1 = (int)(kv_row0 + sel_row[j1]);
-        uint8_t* kst = smem + L::kStageOff + s * L::kStageBytes;
-        uint8_t* vst = kst + L::kKBytes;
-        mbar_arrive_expect_tx(kv_full + s, L::kStageBytes);
-#pragma unroll
-        for (int dh = 0; dh < L::DH; ++dh) {
-          tma_load_2d(kst + k_slot_off<D>(dh, 0), &tm_k, kv_full + s, dh * 64, r0, pol_kv);
-          tma_load_2d(kst + k_slot_off<D>(dh, 1), &tm_k, kv_full + s, dh * 64, r1, pol_kv);
+            for (int dh = 0; dh < L::DH; ++dh)
+              tma_load_2d(smem + L::kQOff + o * L::kQ + dh * 8192, &tm_q, bars + L::kQFull + o,
+                          dh * 64, q_row, pol_q);
+          }
         }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      }
+      const int32_t* idx_row = p.q2k_idx + (x.group * p.nq + x.a) * (long long)p.idx_stride;
+      const int np = (x.num + 1) / 2;
+      const long long kv_row0 = x.group * p.kv_rows_per_group;
+      for (int j0 = 0; ok && j0 < x.num; j0 += 32) {
+        int row, len;
+        resolve_entry(p, x, idx_row, j0 + lane, row, len);
+        const int i_end = min(np, (j0 + 32) / 2);
+        for (int i = j0 / 2; i < i_end; ++i) {
+          const int r0 = __shfl_sync(0xffffffffu, row, 2 * i - j0);
+          const int l0 = __shfl_sync(0xffffffffu, len, 2 * i - j0);
+          int r1 = __shfl_sync(0xffffffffu, row, 2 * i + 1 - j0);
+          int l1 = __shfl_sync(0xffffffffu, len, 2 * i + 1 - j0);
+          if (2 * i + 1 >= x.num) { r1 = r0; l1 = 0; }
+          if (lane == 0) {
+            if (is_k) {
+              const int ks = (int)(gp % L::NK);
+              const long long u = gp / L::NK;
+              if (u >= 1) ok = mbar_wait(bars + L::kKEmpty + ks, (uint32_t)((u - 1) & 1), abort_flag, p.status);
+              if (ok) {
+                kmeta[ks] = make_int2(l0, l1);
+                uint8_t* dst = smem + L::kKOff + ks * L::kK2;
+                mbar_arrive_expect_tx(bars + L::kKFull + ks, L::kK2);
 #pragma unroll
-        for (int dh = 0; dh < L::DH; ++dh) {
-          tma_load_2d(vst + v_slot_off<D>(0, dh), &tm_v, kv_full + s, dh * 64, r0, pol_kv);
-          tma_load_2d(vst + v_slot_off<D>(1, dh), &tm_v, kv_full + s, dh * 64, r1, pol_kv);
+                for (int dh = 0; dh < L::DH; ++dh) {
+                  tma_load_2d(dst + k_slot_off<D>(dh, 0), &tm_k, bars + L::kKFull + ks, dh * 64,
+                              (int)(kv_row0 + r0), pol_kv);
+                  tma_load_2d(dst + k_slot_off<D>(dh, 1), &tm_k, bars + L::kKFull + ks, dh * 64,
+                              (int)(kv_row0 + r1), pol_kv);
+                }
+              }
+            } else {
+              const int vs = (int)(gp % L::NV);
+              const long long u = gp / L::NV;
+              if (u >= 1) ok = mbar_wait(bars + L::kVEmpty + vs, (uint32_t)((u - 1) & 1), abort_flag, p.status);
+              if (ok) {
+                uint8_t* dst = smem + L::kVOff + vs * L::kV2;
+                mbar_arrive_expect_tx(bars + L::kVFull + vs, L::kV2);
+#pragma unroll
+                for (int dh = 0; dh < L::DH; ++dh) {
+                  tma_load_2d(dst + v_slot_off<D>(0, dh), &tm_v, bars + L::kVFull + vs, dh * 64,
+                              (int)(kv_row0 + r0), pol_kv);
+                  tma_load_2d(dst + v_slot_off<D>(1, dh), &tm_v, bars + L::kVFull + vs, dh * 64,
+                              (int)(kv_row0 + r1), pol_kv);
+                }
+              }
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          ++gp;
         }
       }
     }
   } else if (warp == 1) {
     // ===================== MMA issuer =====================
-    if (lane == 0 && npairs > 0) {
-      bool ok = mbar_wait(bar_q, 0, abort_flag, p.status);
-      for (int i = 0; ok && i <= npairs; ++i) {
-        if (i < npairs) {
-          const int s = i & 1;
-          if (!mbar_wait(kv_full + s, (i >> 1) & 1, abort_flag, p.status)) break;
-          if (i >= 2 && !mbar_wait(s_empty + s, ((i - 2) >> 1) & 1, abort_flag, p.status)) break;
+    if (lane == 0) {
+      // total pairs and items of this CTA: commits that nobody would wait for
+      // are not issued, so no asynchronous arrival outlives the CTA
+      long long total = 0, n_mine = 0;
+      for (long long it = it0; it < n_items; it += it_step, ++n_mine) {
+        const Item x = load_item(p, it);
+        total += (x.num + 1) / 2;
+      }
+      long long gp = 0, n = 0;
+      bool ok = true;
+      // the PV product runs one step behind the score product
+      long long pv_g = -1, pv_n = 0;
+      int pv_o = 0;
+      bool pv_first = false, pv_last = false;
+      auto issue_pv = [&]() -> bool {
+        const int vs = (int)(pv_g % L::NV);
+        if (!mbar_wait(bars + L::kVFull + vs, (uint32_t)((pv_g / L::NV) & 1), abort_flag, p.status)) return false;
+        if (!mbar_wait(bars + L::kPFull, (uint32_t)(pv_g & 1), abort_flag, p.status)) return false;
+        if (pv_first && pv_n >= 2 &&
+            !mbar_wait(bars + L::kOEmpty + pv_o, (uint32_t)(((pv_n - 2) >> 1) & 1), abort_flag, p.status))
+          return false;
+        tc_fence_after_sync();
+        issue_pv_mma<D>(tmem_base + kTmemO + 64u * pv_o, sbase + L::kVOff + vs * L::kV2,
+                        sbase + L::kPOff, !pv_first);
+        if (pv_g + 1 < total) umma_commit(bars + L::kPEmpty);
+        if (pv_g + L::NV < total) umma_commit(bars + L::kVEmpty + vs);
+        if (pv_last) umma_commit(bars + L::kOFull + pv_o);
+        pv_g = -1;
+        return true;
+      };
+      for (long long it = it0; ok && it < n_items; it += it_step, ++n) {
+        const Item x = load_item(p, it);
+        const int o = (int)(n & 1);
+        const int np = (x.num + 1) / 2;
+        if (!mbar_wait(bars + L::kQFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
+        for (int i = 0; i < np; ++i, ++gp) {
+          const int sb = (int)(gp & 1);
+          const int ks = (int)(gp % L::NK);
+          if (!mbar_wait(bars + L::kKFull + ks, (uint32_t)((gp / L::NK) & 1), abort_flag, p.status)) { ok = false; break; }
+          if (gp >= 2 && !mbar_wait(bars + L::kSEmpty + sb, (uint32_t)(((gp - 2) >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
           tc_fence_after_sync();
-          issue_score_mma<D>(tmem_base + uint32_t(s) * 64u,
-                             sbase + L::kStageOff + s * L::kStageBytes, q_smem);
-          umma_commit(s_full + s);
+          issue_score_mma<D>(tmem_base + 64u * sb, sbase + L::kKOff + ks * L::kK2,
+                             sbase + L::kQOff + o * L::kQ);
+          umma_commit(bars + L::kSFull + sb);
+          if (gp + L::NK < total) umma_commit(bars + L::kKEmpty + ks);
+          if (i == np - 1 && n + 2 < n_mine) umma_commit(bars + L::kQEmpty + o);
+          if (pv_g >= 0 && !issue_pv()) { ok = false; break; }
+          pv_g = gp; pv_n = n; pv_o = o; pv_first = (i == 0); pv_last = (i == np - 1);
         }
-        if (i >= 1) {
-          const int j = i - 1, sj = j & 1;
-          if (!mbar_wait(p_full + sj, (j >> 1) & 1, abort_flag, p.status)) break;
-          tc_fence_after_sync();
-          issue_pv_mma<D>(tmem_base + kTmemO,
-                          sbase + L::kStageOff + sj * L::kStageBytes + L::kKBytes,
-                          sbase + L::kPOff + sj * L::kPBytes, j > 0);
-          umma_commit(pv_done + sj);
-          // the producer only waits for stages it will refill
-          if (j + 2 < npairs) umma_commit(kv_empty + sj);
+        if (!ok) break;
+        if (np == 0) {
+          // empty selection: no products; still hand the O buffer to the
+          // epilogue in order (it writes out_c * gate for this block)
+          if (pv_g >= 0 && !issue_pv()) { ok = false; break; }
+          if (n >= 2 && !mbar_wait(bars + L::kOEmpty + o, (uint32_t)(((n - 2) >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
+          umma_commit(bars + L::kOFull + o);
+          if (n + 2 < n_mine) umma_commit(bars + L::kQEmpty + o);
         }
       }
+      if (ok && pv_g >= 0) issue_pv();
     }
-  } else {
-    // ===================== softmax + epilogue (warps 2..5) =====================
-    const int wq = warp & 3;             // TMEM lane quarter of this warp
-    const int t128 = tid - 64;           // 0..127
-    const int Lr = wq * 32 + lane;       // TMEM lane: key row of S^T, d of O^T
+  } else if (warp >= 4 && warp < 12) {
+    // ===================== softmax (two groups of 4 warps) =====================
+    const int grp = (warp - 4) / 4;              // query columns 32*grp .. 32*grp+31
+    const int wq = warp & 3;                     // TMEM lane quarter
+    const int t128 = (warp - 4 - 4 * grp) * 32 + lane;
+    const int Lr = wq * 32 + lane;               // TMEM lane: key row of S^T, head dim of O^T
     const int half = Lr >> 6, r = Lr & 63;
+    const uint32_t col0 = 32u * grp;
     const uint32_t t_lane = tmem_base + (uint32_t(wq * 32) << 16);
+    const uint32_t bar_flag = 1 + 2 * grp, bar_red = 2 + 2 * grp;
+    float* red = red_all + grp * 128;
+    float* fin = fin_all + col0;
+    volatile int* gflags = flags + grp * 8;
+    float* m_g = m_s + col0;
+    float* a_g = alpha_s + col0;
     const float c = p.scale_log2;
-    float lp[64];
-#pragma unroll
-    for (int q = 0; q < 64; ++q) lp[q] = 0.f;
+    long long gp = 0, n = 0;
     bool ok = true;
-    for (int i = 0; i < npairs; ++i) {
-      const int s = i & 1;
-      if (!mbar_wait(s_full + s, (i >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-      tc_fence_after_sync();
-      uint32_t sr[64];
-      tmem_ld64(t_lane + uint32_t(s) * 64u, sr);
+    for (long long it = it0; ok && it < n_items; it += it_step, ++n) {
+      const Item x = load_item(p, it);
+      const int o = (int)(n & 1);
+      const int np = (x.num + 1) / 2;
+      float lp[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) lp[q] = 0.f;
+      for (int i = 0; i < np; ++i, ++gp) {
+        const int sb = (int)(gp & 1);
+        const int ks = (int)(gp % L::NK);
+        if (!mbar_wait(bars + L::kSFull + sb, (uint32_t)((gp >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
+        // the K stage's barrier also publishes the pair's key counts; the
+        // stage cannot be refilled before this group's arrival below
+        if (!mbar_wait(bars + L::kKFull + ks, (uint32_t)((gp / L::NK) & 1), abort_flag, p.status)) { ok = false; break; }
+        const int2 lens = kmeta[ks];
+        const bool valid = r < (half ? lens.y : lens.x);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + L::kKEmpty + ks);
+        tc_fence_after_sync();
+        uint32_t sr[32];
+        tmem_ld32(t_lane + 64u * sb + col0, sr);
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + L::kSEmpty + sb);
+        bool rescale = (i == 0);
+        if (i > 0) {
+          float worst = -INFINITY;
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 32; q += 4) {
+              const float4 mm = *reinterpret_cast<const float4*>(m_g + q);
+              worst = fmaxf(worst, fmaf(__uint_as_float(sr[q]), c, -mm.x));
+              worst = fmaxf(worst, fmaf(__uint_as_float(sr[q + 1]), c, -mm.y));
+              worst = fmaxf(worst, fmaf(__uint_as_float(sr[q + 2]), c, -mm.z));
+              worst = fmaxf(worst, fmaf(__uint_as_float(sr[q + 3]), c, -mm.w));
+            }
+          }
+          const int need = __any_sync(0xffffffffu, worst > 8.f) ? 1 : 0;
+          if (lane == 0) gflags[(gp & 1) * 4 + wq] = need;
+          named_barrier_sync(bar_flag, 128);
+          rescale = (gflags[(gp & 1) * 4 + 0] | gflags[(gp & 1) * 4 + 1] |
+                     gflags[(gp & 1) * 4 + 2] | gflags[(gp & 1) * 4 + 3]) != 0;
+        }
+        if (rescale) {
+          {
+            float masked[32];
+#pragma unroll
+            for (int q = 0; q < 32; ++q) masked[q] = valid ? __uint_as_float(sr[q]) * c : -INFINITY;
+            col_reduce32<true>(masked, red, fin, wq, lane, t128, bar_red);
+          }
+          if (t128 < 32) {
+            const float f = fin[t128];
+            if (i == 0) {
+              m_g[t128] = (f == -INFINITY) ? 0.f : f;
+            } else {
+              const float old = m_g[t128];
+              const float nm = fmaxf(old, f);
+              a_g[t128] = fast_exp2(old - nm);
+              m_g[t128] = nm;
+            }
+          }
+          named_barrier_sync(bar_red, 128);
+          if (i > 0) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) lp[q] *= a_g[q];
+            // O^T holds this item's PV products up to the previous pair:
+            // wait for the last one, then rescale this lane's columns.
+            if (!mbar_wait(bars + L::kPEmpty, (uint32_t)((gp - 1) & 1), abort_flag, p.status)) { ok = false; break; }
+            tc_fence_after_sync();
+            uint32_t ov[32];
+            tmem_ld32(t_lane + kTmemO + 64u * o + col0, ov);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * a_g[q]);
+            tmem_st32(t_lane + kTmemO + 64u * o + col0, ov);
+            tc_fence_before_sync();
+          }
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int q = 0; q < 32; q += 4) {
+          const float4 mm = *reinterpret_cast<const float4*>(m_g + q);
+          float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+          if (valid) {
+            p0 = fast_exp2(fmaf(__uint_as_float(sr[q]), c, -mm.x));
+            p1 = fast_exp2(fmaf(__uint_as_float(sr[q + 1]), c, -mm.y));
+            p2 = fast_exp2(fmaf(__uint_as_float(sr[q + 2]), c, -mm.z));
+            p3 = fast_exp2(fmaf(__uint_as_float(sr[q + 3]), c, -mm.w));
+          }
+          lp[q] += p0;
+          lp[q + 1] += p1;
+          lp[q + 2] += p2;
+          lp[q + 3] += p3;
+          pk[q / 2] = pack_bf16x2(p0, p1);
+          pk[q / 2 + 1] = pack_bf16x2(p2, p3);
+        }
+        // the single P^T buffer is free once the previous PV product is done
+        if (gp >= 1 && !mbar_wait(bars + L::kPEmpty, (uint32_t)((gp - 1) & 1), abort_flag, p.status)) { ok = false; break; }
+        uint8_t* pbuf = smem + L::kPOff;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          *reinterpret_cast<uint4*>(pbuf + sw128_off(Lr, 4 * grp + ch)) =
+              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + L::kPFull);
+      }
+      if (!ok) break;
+      // end of item: 1 / row sums for the epilogue
+      if (n >= 2 && !mbar_wait(bars + L::kOEmpty + o, (uint32_t)(((n - 2) >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
+      col_reduce32<false>(lp, red, fin, wq, lane, t128, bar_red);
+      if (t128 < 32) inv_l[o * 64 + col0 + t128] = fin[t128] > 0.f ? 1.f / fin[t128] : 0.f;
+      named_barrier_sync(bar_red, 128);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + L::kLFull + o);
+    }
+  } else if (warp >= 12) {
+    // ===================== epilogue =====================
+    const int wq = warp & 3;
+    const int d = wq * 32 + lane;                // TMEM lane = head dim of O^T
+    const uint32_t t_lane = tmem_base + (uint32_t(wq * 32) << 16);
+    long long n = 0;
+    for (long long it = it0; it < n_items; it += it_step, ++n) {
+      const Item x = load_item(p, it);
+      const int o = (int)(n & 1);
+      if (!mbar_wait(bars + L::kOFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status)) break;
+      if (!mbar_wait(bars + L::kLFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status)) break;
+      float ov[64];
+      if (wq * 32 < D && x.num > 0) {
+        tc_fence_after_sync();
+        uint32_t raw[32];
+        tmem_ld32(t_lane + kTmemO + 64u * o, raw);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) ov[q] = __uint_as_float(raw[q]) * inv_l[o * 64 + q];
+        tmem_ld32(t_lane + kTmemO + 64u * o + 32u, raw);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) ov[32 + q] = __uint_as_float(raw[q]) * inv_l[o * 64 + 32 + q];
+      } else {
+#pragma unroll
+        for (int q = 0; q < 64; ++q) ov[q] = 0.f;
+      }
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_empty + s);
-      const int jsel = 2 * i + half;
-      const int len = (jsel < num) ? (int)sel_len[jsel] : 0;
-      const bool valid = r < len;
-      bool rescale = (i == 0);
-      if (i > 0) {
-        // does any logit of this pair exceed the running max by more than 2^8?
-        float worst = -INFINITY;
-        if (valid) {
+      if (lane == 0) mbar_arrive(bars + L::kOEmpty + o);
+      if (wq * 32 >= D) continue;
+      float oc = 0.f;
+      if (COMBINE) oc = p.out_c[(x.group * p.nq + x.a) * (long long)D + d];
+      const long long orow0 = x.group * p.q_rows_per_group + x.q_tok;
+      const long long grow0 = ((long long)x.b * p.gate_seq + x.q_tok) * p.H + x.h;
 #pragma unroll
-          for (int q = 0; q < 64; q += 4) {
-            const float4 mm = *reinterpret_cast<const float4*>(m_s + q);
-            worst = fmaxf(worst, fmaf(__uint_as_float(sr[q]), c, -mm.x));
-            worst = fmaxf(worst, fmaf(__uint_as_float(sr[q + 1]), c, -mm.y));
-            worst = fmaxf(worst, fmaf(__uint_as_float(sr[q + 2]), c, -mm.z));
-            worst = fmaxf(worst, fmaf(__uint_as_float(sr[q + 3]), c, -mm.w));
+      for (int q = 0; q < 64; ++q) {
+        __nv_bfloat16 val;
+        if (q < x.q_len) {
+          float v = ov[q];
+          if (COMBINE) {
+            if (GATED) {
+              const float g = __bfloat162float(p.gate[(grow0 + (long long)q * p.H) * D + d]);
+              v = fmaf(oc, g, v);
+            } else {
+              v += oc;
+            }
           }
+          val = __float2bfloat16_rn(v);
+        } else {
+          if (p.varlen) continue;
+          val = __float2bfloat16_rn(0.f);
         }
-        const int need = __any_sync(0xffffffffu, worst > 8.f) ? 1 : 0;
-        if (lane == 0) flags[(i & 1) * 4 + wq] = need;
-        named_barrier_sync(1, 128);
-        rescale = (flags[(i & 1) * 4 + 0] | flags[(i & 1) * 4 + 1] | flags[(i & 1) * 4 + 2] |
-                   flags[(i & 1) * 4 + 3]) != 0;
+        p.out[(orow0 + q) * D + d] = val;
       }
-      if (rescale) {
-        {
-          float masked[64];
-#pragma unroll
-          for (int q = 0; q < 64; ++q) masked[q] = valid ? __uint_as_float(sr[q]) * c : -INFINITY;
-          col_reduce64<true>(masked, red, fin, wq, lane, t128);
-        }
-        if (t128 < 64) {
-          const float f = fin[t128];
-          if (i == 0) {
-            m_s[t128] = (f == -INFINITY) ? 0.f : f;
-          } else {
-            const float old = m_s[t128];
-            const float nm = fmaxf(old, f);
-            alpha_s[t128] = fast_exp2(old - nm);
-            m_s[t128] = nm;
-          }
-        }
-        named_barrier_sync(2, 128);
-        if (i > 0) {
-#pragma unroll
-          for (int q = 0; q < 64; ++q) lp[q] *= alpha_s[q];
-          // O^T already holds PV(0..i-1): wait for the last one, then rescale
-          // this thread's lane (one head-dim row, all 64 query columns).
-          const int j = i - 1;
-          if (!mbar_wait(pv_done + (j & 1), (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-          tc_fence_after_sync();
-          uint32_t o[64];
-          tmem_ld64(t_lane + kTmemO, o);
-#pragma unroll
-          for (int q = 0; q < 64; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha_s[q]);
-          tmem_st64(t_lane + kTmemO, o);
-          tc_fence_before_sync();
-        }
-      }
-      // probabilities (bf16) for this key row
-      uint32_t pk[32];
-#pragma unroll
-      for (int q = 0; q < 64; q += 4) {
-        const float4 mm = *reinterpret_cast<const float4*>(m_s + q);
-        float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-        if (valid) {
-          p0 = fast_exp2(fmaf(__uint_as_float(sr[q]), c, -mm.x));
-          p1 = fast_exp2(fmaf(__uint_as_float(sr[q + 1]), c, -mm.y));
-          p2 = fast_exp2(fmaf(__uint_as_float(sr[q + 2]), c, -mm.z));
-          p3 = fast_exp2(fmaf(__uint_as_float(sr[q + 3]), c, -mm.w));
-        }
-        lp[q] += p0;
-        lp[q + 1] += p1;
-        lp[q + 2] += p2;
-        lp[q + 3] += p3;
-        pk[q / 2] = pack_bf16x2(p0, p1);
-        pk[q / 2 + 1] = pack_bf16x2(p2, p3);
-      }
-      if (i >= 2 && !mbar_wait(pv_done + s, ((i - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-      uint8_t* pbuf = smem + L::kPOff + s * L::kPBytes;
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        *reinterpret_cast<uint4*>(pbuf + sw128_off(Lr, ch)) =
-            make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full + s);
-    }
-
-    // ---- epilogue --------------------------------------------------------
-    float* tile = reinterpret_cast<float*>(smem + L::kStageOff);  // [64][D] fp32
-    col_reduce64<false>(lp, red, fin, wq, lane, t128);
-    if (t128 < 64) inv_l_s[t128] = fin[t128] > 0.f ? 1.f / fin[t128] : 0.f;
-    named_barrier_sync(2, 128);
-    bool have_o = ok && npairs > 0;
-    if (have_o) {
-      const int jl = npairs - 1;
-      if (npairs >= 2 && !mbar_wait(pv_done + ((jl - 1) & 1), ((jl - 1) >> 1) & 1, abort_flag, p.status)) have_o = false;
-      if (have_o && !mbar_wait(pv_done + (jl & 1), (jl >> 1) & 1, abort_flag, p.status)) have_o = false;
-    }
-    if (Lr < D) {
-      if (have_o) {
-        tc_fence_after_sync();
-        uint32_t o[64];
-        tmem_ld64(t_lane + kTmemO, o);
-#pragma unroll
-        for (int q = 0; q < 64; ++q) tile[q * D + Lr] = __uint_as_float(o[q]) * inv_l_s[q];
-      } else {
-#pragma unroll
-        for (int q = 0; q < 64; ++q) tile[q * D + Lr] = 0.f;
-      }
-    } else if (have_o) {
-      // D = 64: lanes 64..127 hold nothing of use; the warp still takes
-      // part in the collective TMEM load.
-      tc_fence_after_sync();
-      uint32_t o[64];
-      tmem_ld64(t_lane + kTmemO, o);
-    }
-    tc_fence_before_sync();
-    named_barrier_sync(1, 128);
-    // cooperative combine + store: 4 consecutive d per thread, coalesced rows
-    constexpr int TPR = D / 4;            // threads per row
-    constexpr int RPI = 128 / TPR;        // rows per iteration
-    const int d0 = (t128 % TPR) * 4;
-    const float* oc = COMBINE ? p.out_c + (group * p.nq + a) * (long long)D : nullptr;
-    float4 ocv = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (COMBINE) ocv = *reinterpret_cast<const float4*>(oc + d0);
-    for (int q = t128 / TPR; q < 64; q += RPI) {
-      const long long orow = group * p.q_rows_per_group + q_tok + q;
-      uint2 packed;
-      if (q < q_len) {
-        const float4 o = *reinterpret_cast<const float4*>(tile + q * D + d0);
-        float v0 = o.x, v1 = o.y, v2 = o.z, v3 = o.w;
-        if (COMBINE) {
-          if (GATED) {
-            const long long grow = ((long long)b * p.gate_seq + q_tok + q) * p.H + h;
-            const uint2 graw = *reinterpret_cast<const uint2*>(p.gate + grow * D + d0);
-            const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&graw.x));
-            const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&graw.y));
-            v0 = fmaf(ocv.x, g01.x, v0);
-            v1 = fmaf(ocv.y, g01.y, v1);
-            v2 = fmaf(ocv.z, g23.x, v2);
-            v3 = fmaf(ocv.w, g23.y, v3);
-          } else {
-            v0 += ocv.x; v1 += ocv.y; v2 += ocv.z; v3 += ocv.w;
-          }
-        }
-        packed = make_uint2(pack_bf16x2(v0, v1), pack_bf16x2(v2, v3));
-      } else {
-        if (p.varlen) continue;
-        packed = make_uint2(0u, 0u);
-      }
-      *reinterpret_cast<uint2*>(p.out + orow * D + d0) = packed;
     }
   }
 
@@ -522,7 +636,6 @@ __global__ void __launch_bounds__(kSparseThreads, 1)
 template <int D>
 __global__ void __launch_bounds__(128, 1)
     selftest_umma_kernel(int mode, const __nv_bfloat16* a, const __nv_bfloat16* bm, float* cm) {
-  using L = SparseSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -592,7 +705,6 @@ __global__ void __launch_bounds__(128, 1)
     tc_fence_after_sync();
     tmem_dealloc(tmem_base, 128);
   }
-  (void)L::kBytes;
 }
 
 // ---------------------------------------------------------------------------
@@ -631,16 +743,30 @@ static bool make_tile_map(CUtensorMap* map, const void* base, long long rows, in
   return r == CUDA_SUCCESS;
 }
 
+static int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 template <int D, bool COMBINE, bool GATED>
 static int launch_sparse_t(const SparseParams& p, const CUtensorMap& mq, const CUtensorMap& mk,
                            const CUtensorMap& mv, cudaStream_t stream) {
-  using L = SparseSmem<D>;
+  using L = Layout<D>;
   auto kern = sparse_fwd_kernel<D, COMBINE, GATED>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc) !=
       cudaSuccess)
     return VSA_ERR_CUDA;
-  dim3 grid(p.nq, p.H, p.B);
-  kern<<<grid, kSparseThreads, L::kAlloc, stream>>>(mq, mk, mv, p);
+  const long long n_items = (long long)p.B * p.H * p.nq;
+  const long long grid = n_items < sm_count() ? n_items : sm_count();
+  kern<<<(unsigned)grid, kThreads, L::kAlloc, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
@@ -648,7 +774,6 @@ int launch_sparse(const SparseParams& p, const void* q, const void* k, const voi
                   long long q_rows_total, long long kv_rows_total, int D, bool combine,
                   bool gated, cudaStream_t stream) {
   if (p.nq <= 0 || p.H <= 0 || p.B <= 0) return VSA_OK;
-  if (p.H > 65535 || p.B > 65535) return VSA_ERR_UNSUPPORTED;
   if (q_rows_total + 64 > 0x7FFFFFFFLL || kv_rows_total + 64 > 0x7FFFFFFFLL)
     return VSA_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
   CUtensorMap mq, mk, mv;

@@ -243,6 +243,19 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Load / store 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  VSA_TMEM_LD16(taddr + 0, r, 0);
+  VSA_TMEM_LD16(taddr + 16, r, 16);
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  VSA_TMEM_ST16(taddr + 0, r, 0);
+  VSA_TMEM_ST16(taddr + 16, r, 16);
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // 2^x on the special-function unit (PTX ex2.approx, flush-to-zero).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;

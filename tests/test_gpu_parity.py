@@ -88,6 +88,37 @@ def test_sparse_from_indices(case):
     assert np.all(got[:, :, pad] == 0.0), "padded query rows must be written as 0"
 
 
+@pytest.mark.parametrize("D", [128, 64])
+def test_sparse_many_items_mixed_counts(D):
+    """More work items than SMs, so each CTA of the persistent grid walks
+    several items: selection counts vary per item (0, odd, longer than the
+    K/V rings), blocks are ragged, entries repeat."""
+    B, H = 1, 8
+    qs = [64] * 63 + [17]
+    ks = [64] * 10 + [5, 64, 64, 33, 64, 64]
+    width = 13
+    rng = np.random.default_rng(77 + D)
+    q = _bhsd(B, H, qs, D, 16, 0)
+    k = _bhsd(B, H, ks, D, 16, 1, pad_value=2.0)
+    v = _bhsd(B, H, ks, D, 16, 2, pad_value=-2.0)
+    idx = np.full((B, H, len(qs), width), -1, dtype=np.int32)
+    num = rng.integers(0, width + 1, size=(B, H, len(qs))).astype(np.int32)
+    for b in range(B):
+        for h in range(H):
+            for a in range(len(qs)):
+                idx[b, h, a, :num[b, h, a]] = rng.integers(0, len(ks), size=num[b, h, a])
+    out = vsa.block_sparse_attn_from_indices(
+        q.to(DEV), k.to(DEV), v.to(DEV), torch.from_numpy(idx).to(DEV), torch.from_numpy(num).to(DEV),
+        qs, ks)
+    vsa.check_device_status()
+    want = O.block_sparse_attention(P.to_np(q), P.to_np(k), P.to_np(v), idx, num, qs, ks,
+                                    O.default_scale(D))
+    got = P.to_np(out)
+    rr = P.real_rows(qs)
+    P.assert_outputs_close(got[:, :, rr], want[:, :, rr])
+    assert np.all(got[:, :, np.setdiff1d(np.arange(got.shape[2]), rr)] == 0.0)
+
+
 def test_sparse_edge_cases():
     """q2k_num = 0, a single one-token KV block, repeated entries, odd counts."""
     B, H, D = 1, 2, 128
