@@ -18,20 +18,24 @@
 // O^T too, so the epilogue of one work item overlaps the next item's loop.
 //
 // Persistent grid: one CTA per SM walks the work items (query block, head,
-// batch) b-major, h, a-minor with stride gridDim.x.  512 threads:
-//   warp 0       K producer: Q of each item (2 buffers) and K tile pairs into
-//                a 3-stage ring, with each pair's key counts (TMA, 128-byte
+// batch) b-major, h, a-minor with stride gridDim.x.  512 threads, four
+// warpgroups:
+//   warp 0       K producer: the item's Q tile and K tile pairs into a
+//                3-stage ring with each pair's key counts (TMA, 128-byte
 //                swizzle, no multicast)
-//   warp 1       TMEM owner and MMA issuer (one thread)
+//   warp 1       TMEM owner; issues the score products S^T into four TMEM
+//                buffers, running ahead of the softmax
 //   warp 2       V producer: V tile pairs into a 2-stage ring
-//   warp 3       idle
+//   warp 3       issues the PV products into two TMEM output buffers
 //   warps 4-7    softmax for query columns 0..31
 //   warps 8-11   softmax for query columns 32..63
 //   warps 12-15  epilogue: O^T / l, the gated combine, bf16 stores
-// The running max per query column is exact after an item's first pair
-// (column reduction across lanes) and refreshed only when a logit exceeds it
-// by more than 2^8 (warp vote), then O^T and the partial sums are rescaled.
-// Row sums are accumulated per lane and reduced across lanes once per item.
+// P^T is double-buffered in shared memory, so the softmax of pair g only
+// waits for the PV product of pair g - 2.  The running max per query column
+// is exact after an item's first pair (column reduction across lanes) and
+// refreshed only when a logit exceeds it by more than 2^8 (barrier vote),
+// then O^T and the partial sums are rescaled.  Row sums are accumulated per
+// lane and reduced across lanes once per item.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -44,35 +48,50 @@
 namespace vsa {
 
 constexpr int kThreads = 512;
-constexpr uint32_t kTmemCols = 256;   // S^T buffers at 0 and 64, O^T buffers at 128 and 192
-constexpr uint32_t kTmemO = 128;
+constexpr uint32_t kRegsProducer = 64, kRegsSoftmax = 192, kRegsEpilogue = 64;
+static_assert(128u * (kRegsProducer + 2u * kRegsSoftmax + kRegsEpilogue) <= 512u * 128u,
+              "register split exceeds the launch's 128 registers per thread");
+#ifndef VSA_KLEAD
+#define VSA_KLEAD 4
+#endif
+constexpr int kKLead = VSA_KLEAD;      // K requests run at most this many pairs ahead of V
+constexpr int kNS = 4;                 // S^T buffers in TMEM
+constexpr int kNP = 2;                 // P^T buffers in shared memory
+constexpr uint32_t kTmemCols = 512;    // S^T buffers at 64*i (i < 4), O^T buffers at 256, 320
+constexpr uint32_t kTmemO = 256;
 
 template <int D>
 struct Layout {
   static constexpr int DH = D / 64;                        // 64-element head-dim halves
-  static constexpr int NK = 3;                             // K ring stages (tile pairs)
-  static constexpr int NV = 2;                             // V ring stages
+#ifndef VSA_NK
+#define VSA_NK 3
+#endif
+#ifndef VSA_NV
+#define VSA_NV 2
+#endif
+  static constexpr int NK = VSA_NK;                        // K ring stages (tile pairs)
+  static constexpr int NV = VSA_NV;                        // V ring stages
   static constexpr uint32_t kQ = 64u * D * 2u;             // one 64-row Q tile
   static constexpr uint32_t kK2 = 2u * 64u * D * 2u;       // a pair of K tiles (M = 128)
   static constexpr uint32_t kV2 = kK2;
   static constexpr uint32_t kP = 128u * 64u * 2u;          // P^T in bf16
   static constexpr uint32_t kQOff = 0;
-  static constexpr uint32_t kKOff = kQOff + 2u * kQ;
+  static constexpr uint32_t kKOff = kQOff + kQ;
   static constexpr uint32_t kVOff = kKOff + NK * kK2;
   static constexpr uint32_t kPOff = kVOff + NV * kV2;
-  static constexpr uint32_t kRedOff = kPOff + kP;               // [2 groups][4 warps][32] f32
+  static constexpr uint32_t kStageOff = kPOff + kNP * kP;       // epilogue tile [16][D] f32
+  static constexpr uint32_t kRedOff = kStageOff + 16u * D * 4u; // [2 groups][4 warps][32] f32
   static constexpr uint32_t kFinOff = kRedOff + 2u * 4u * 32u * 4u;  // [64] f32
-  static constexpr uint32_t kMOff = kFinOff + 64u * 4u;         // [64] running max (log2 units)
-  static constexpr uint32_t kAlphaOff = kMOff + 64u * 4u;       // [64] rescale factors
+  static constexpr uint32_t kAlphaOff = kFinOff + 64u * 4u;     // [64] rescale factors
   static constexpr uint32_t kInvLOff = kAlphaOff + 64u * 4u;    // [2][64] 1 / row sum per O buffer
-  static constexpr uint32_t kFlagOff = kInvLOff + 2u * 64u * 4u;  // [2 groups][2][4] int
-  static constexpr uint32_t kKMetaOff = kFlagOff + 64u;         // [NK] int2: key counts of a pair
-  static constexpr uint32_t kBarOff = kKMetaOff + 32u;
+  static constexpr uint32_t kKMetaOff = kInvLOff + 2u * 64u * 4u;  // [NK] int2: key counts
+  static constexpr uint32_t kVIssuedOff = kKMetaOff + 32u;        // V pairs requested so far
+  static constexpr uint32_t kBarOff = kVIssuedOff + 16u;
   // barriers
-  static constexpr int kQFull = 0, kQEmpty = 2, kKFull = 4, kKEmpty = kKFull + NK,
+  static constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + NK,
                        kVFull = kKEmpty + NK, kVEmpty = kVFull + NV, kSFull = kVEmpty + NV,
-                       kSEmpty = kSFull + 2, kPFull = kSEmpty + 2, kPEmpty = kPFull + 1,
-                       kOFull = kPEmpty + 1, kOEmpty = kOFull + 2, kLFull = kOEmpty + 2,
+                       kSEmpty = kSFull + kNS, kPFull = kSEmpty + kNS, kPEmpty = kPFull + kNP,
+                       kOFull = kPEmpty + kNP, kOEmpty = kOFull + 2, kLFull = kOEmpty + 2,
                        kNumBars = kLFull + 2;
   static constexpr uint32_t kMiscOff = kBarOff + 8u * kNumBars;  // tmem address, abort flag
   static constexpr uint32_t kBytes = kMiscOff + 16u;
@@ -94,37 +113,47 @@ __device__ __forceinline__ uint32_t v_slot_off(int tile, int dh) {
 }
 
 // S^T[128][64] = K2 . Q^T: M = 128 key rows, N = 64 query rows, K = D.
+// a_desc / b_desc describe the K2 pair and the Q tile at their first byte;
+// each K = 16 step advances the start address (in 16-byte units) inside the
+// 128-byte swizzle atom, and by one 64-column region every 4 steps.
 template <int D>
-__device__ __forceinline__ void issue_score_mma(uint32_t tmem_d, uint32_t k_base, uint32_t q_base) {
+__device__ __forceinline__ void issue_score_desc(uint32_t tmem_d, uint64_t a_desc, uint64_t b_desc) {
   constexpr uint32_t idesc = make_idesc_bf16(128, 64, false, false);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const int dh = kk / 4;
-    const uint32_t koff = uint32_t(kk % 4) * 32u;
-    const uint64_t a = make_sdesc_sw128(k_base + k_slot_off<D>(dh, 0) + koff, 16u, 1024u);
-    const uint64_t b = make_sdesc_sw128(q_base + uint32_t(dh) * 8192u + koff, 16u, 1024u);
+    const uint64_t a = a_desc + (uint64_t)((k_slot_off<D>(kk / 4, 0) + (kk % 4) * 32) >> 4);
+    const uint64_t b = b_desc + (uint64_t)(((kk / 4) * 8192 + (kk % 4) * 32) >> 4);
     umma_bf16(tmem_d, a, b, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
 // O^T[128][64] (+)= V2^T . P^T: M = 128 head-dim rows, N = 64 query rows,
-// K = 128 key rows.  Both operands MN-major.  The second 64-row atom of A
-// (head dims 64..127) sits 8 KB after the first.  For D = 64 that atom is
-// other, in-bounds shared memory: TMEM lanes 64..127 then hold values that no
-// one reads (row m of the product depends on row m of A only).
+// K = 128 key rows.  Both operands MN-major; each K = 16 step moves 16 key
+// rows (2 KB) down.  The second 64-row atom of A (head dims 64..127) sits
+// 8 KB after the first (LBO).  For D = 64 that atom is other, in-bounds
+// shared memory: TMEM lanes 64..127 then hold values that no one reads (row m
+// of the product depends on row m of A only).
+template <int D>
+__device__ __forceinline__ void issue_pv_desc(uint32_t tmem_o, uint64_t a_desc, uint64_t b_desc,
+                                              bool accumulate) {
+  constexpr uint32_t idesc = make_idesc_bf16(128, 64, true, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t a = a_desc + (uint64_t)((v_slot_off<D>(kk / 4, 0) + (kk % 4) * 2048) >> 4);
+    const uint64_t b = b_desc + (uint64_t)((kk * 2048) >> 4);
+    umma_bf16(tmem_o, a, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_score_mma(uint32_t tmem_d, uint32_t k_base, uint32_t q_base) {
+  issue_score_desc<D>(tmem_d, make_sdesc_sw128(k_base, 16u, 1024u), make_sdesc_sw128(q_base, 16u, 1024u));
+}
 template <int D>
 __device__ __forceinline__ void issue_pv_mma(uint32_t tmem_o, uint32_t v_base, uint32_t p_base,
                                              bool accumulate) {
-  constexpr uint32_t idesc = make_idesc_bf16(128, 64, true, true);
-  constexpr uint32_t lbo = 8192u;
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const int tile = kk / 4;
-    const uint32_t roff = uint32_t(kk % 4) * 16u * 128u;
-    const uint64_t a = make_sdesc_sw128(v_base + v_slot_off<D>(tile, 0) + roff, lbo, 1024u);
-    const uint64_t b = make_sdesc_sw128(p_base + uint32_t(kk) * 2048u, 8192u, 1024u);
-    umma_bf16(tmem_o, a, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
-  }
+  issue_pv_desc<D>(tmem_o, make_sdesc_sw128(v_base, 8192u, 1024u),
+                   make_sdesc_sw128(p_base, 8192u, 1024u), accumulate);
 }
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled
@@ -179,6 +208,27 @@ __device__ __forceinline__ void col_reduce32(const float (&v)[32], float* red, f
                               red_op<IsMax>(red[64 + t128], red[96 + t128]));
   }
   named_barrier_sync(bar_id, 128);
+}
+
+// Probabilities of one key row for 32 query columns: p = 2^x (0 for a
+// masked row), added to the row-sum partials and written as bf16 into this
+// row's half of the swizzled P^T tile.
+__device__ __forceinline__ void write_probs(const uint32_t (&x)[32], bool valid, float (&lp)[32],
+                                            uint8_t* pbuf, int row, int grp) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int q = 0; q < 32; q += 2) {
+    const float p0 = valid ? fast_exp2(__uint_as_float(x[q])) : 0.f;
+    const float p1 = valid ? fast_exp2(__uint_as_float(x[q + 1])) : 0.f;
+    lp[q] += p0;
+    lp[q + 1] += p1;
+    pk[q / 2] = pack_bf16x2(p0, p1);
+  }
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    *reinterpret_cast<uint4*>(pbuf + sw128_off(row, 4 * grp + ch)) =
+        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+  }
 }
 
 // One work item: query block a of head h of batch b.
@@ -251,10 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   float* red_all = reinterpret_cast<float*>(smem + L::kRedOff);
   float* fin_all = reinterpret_cast<float*>(smem + L::kFinOff);
-  float* m_s = reinterpret_cast<float*>(smem + L::kMOff);
-  float* alpha_s = reinterpret_cast<float*>(smem + L::kAlphaOff);
   float* inv_l = reinterpret_cast<float*>(smem + L::kInvLOff);
-  volatile int* flags = reinterpret_cast<volatile int*>(smem + L::kFlagOff);
   int2* kmeta = reinterpret_cast<int2*>(smem + L::kKMetaOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
@@ -267,15 +314,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < L::kNumBars; ++i) {
-      uint32_t count = 1;
-      if (i == L::kSEmpty || i == L::kSEmpty + 1 || i == L::kPFull || i == L::kLFull ||
-          i == L::kLFull + 1)
+      uint32_t count = 1;  // TMA transaction arrival or one tcgen05.commit
+      if ((i >= L::kSEmpty && i < L::kSEmpty + kNS) || (i >= L::kPFull && i < L::kPFull + kNP) ||
+          i == L::kLFull || i == L::kLFull + 1)
         count = 8;  // one arrival per softmax warp
-      if (i >= L::kKEmpty && i < L::kKEmpty + L::NK) count = 9;  // MMA commit + 8 softmax warps
+      if (i >= L::kKEmpty && i < L::kKEmpty + L::NK) count = 9;  // score commit + 8 softmax warps
       if (i == L::kOEmpty || i == L::kOEmpty + 1) count = 4;   // epilogue warps
       mbar_init(bars + i, count);
     }
     *abort_flag = 0;
+    *reinterpret_cast<volatile int*>(smem + L::kVIssuedOff) = 0;
     mbar_fence_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
@@ -289,150 +337,172 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0 || warp == 2) {
-    // ===================== producers (whole warp) =====================
-    const bool is_k = (warp == 0);
-    const uint64_t pol_q = l2_policy_evict_first();
-    const uint64_t pol_kv = l2_policy_evict_last();
-    long long gp = 0;  // pair counter over this CTA's items
-    bool ok = true;
-    long long n = 0;
-    for (long long it = it0; ok && it < n_items; it += it_step, ++n) {
-      const Item x = load_item(p, it);
-      const int o = (int)(n & 1);
-      if (is_k) {
-        if (lane == 0) {
-          check_item(p, it);
-          if (n >= 2)
-            ok = mbar_wait(bars + L::kQEmpty + o, (uint32_t)(((n - 2) >> 1) & 1), abort_flag, p.status);
-          if (ok) {
-            mbar_arrive_expect_tx(bars + L::kQFull + o, L::kQ);
-            const int q_row = (int)(x.group * p.q_rows_per_group + x.q_tok);
-#pragma unroll
-            for (int dh = 0; dh < L::DH; ++dh)
-              tma_load_2d(smem + L::kQOff + o * L::kQ + dh * 8192, &tm_q, bars + L::kQFull + o,
-                          dh * 64, q_row, pol_q);
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      }
-      const int32_t* idx_row = p.q2k_idx + (x.group * p.nq + x.a) * (long long)p.idx_stride;
-      const int np = (x.num + 1) / 2;
-      const long long kv_row0 = x.group * p.kv_rows_per_group;
-      for (int j0 = 0; ok && j0 < x.num; j0 += 32) {
-        int row, len;
-        resolve_entry(p, x, idx_row, j0 + lane, row, len);
-        const int i_end = min(np, (j0 + 32) / 2);
-        for (int i = j0 / 2; i < i_end; ++i) {
-          const int r0 = __shfl_sync(0xffffffffu, row, 2 * i - j0);
-          const int l0 = __shfl_sync(0xffffffffu, len, 2 * i - j0);
-          int r1 = __shfl_sync(0xffffffffu, row, 2 * i + 1 - j0);
-          int l1 = __shfl_sync(0xffffffffu, len, 2 * i + 1 - j0);
-          if (2 * i + 1 >= x.num) { r1 = r0; l1 = 0; }
+  // Register split by warpgroup: producers/MMA and the epilogue give
+  // registers to the two softmax warpgroups.  The launch reserves 128 per
+  // thread (512 x 128 = 65536); the split needs 128 x (64 + 192 + 192 + 64).
+  if (warp < 4) {
+    regs_dec<kRegsProducer>();
+    if (warp == 0 || warp == 2) {
+      // ===================== producers (whole warp) =====================
+      const bool is_k = (warp == 0);
+      const uint64_t pol_q = l2_policy_evict_first();
+      const uint64_t pol_kv = l2_policy_evict_last();
+      long long gp = 0;  // pair counter over this CTA's items
+      bool ok = true;
+      long long n = 0;
+      for (long long it = it0; ok && it < n_items; it += it_step, ++n) {
+        const Item x = load_item(p, it);
+        if (is_k) {
           if (lane == 0) {
-            if (is_k) {
-              const int ks = (int)(gp % L::NK);
-              const long long u = gp / L::NK;
-              if (u >= 1) ok = mbar_wait(bars + L::kKEmpty + ks, (uint32_t)((u - 1) & 1), abort_flag, p.status);
-              if (ok) {
-                kmeta[ks] = make_int2(l0, l1);
-                uint8_t* dst = smem + L::kKOff + ks * L::kK2;
-                mbar_arrive_expect_tx(bars + L::kKFull + ks, L::kK2);
+            check_item(p, it);
+            if (n >= 1)
+              ok = mbar_wait(bars + L::kQEmpty, (uint32_t)((n - 1) & 1), abort_flag, p.status);
+            if (ok) {
+              mbar_arrive_expect_tx(bars + L::kQFull, L::kQ);
+              const int q_row = (int)(x.group * p.q_rows_per_group + x.q_tok);
 #pragma unroll
-                for (int dh = 0; dh < L::DH; ++dh) {
-                  tma_load_2d(dst + k_slot_off<D>(dh, 0), &tm_k, bars + L::kKFull + ks, dh * 64,
-                              (int)(kv_row0 + r0), pol_kv);
-                  tma_load_2d(dst + k_slot_off<D>(dh, 1), &tm_k, bars + L::kKFull + ks, dh * 64,
-                              (int)(kv_row0 + r1), pol_kv);
-                }
-              }
-            } else {
-              const int vs = (int)(gp % L::NV);
-              const long long u = gp / L::NV;
-              if (u >= 1) ok = mbar_wait(bars + L::kVEmpty + vs, (uint32_t)((u - 1) & 1), abort_flag, p.status);
-              if (ok) {
-                uint8_t* dst = smem + L::kVOff + vs * L::kV2;
-                mbar_arrive_expect_tx(bars + L::kVFull + vs, L::kV2);
-#pragma unroll
-                for (int dh = 0; dh < L::DH; ++dh) {
-                  tma_load_2d(dst + v_slot_off<D>(0, dh), &tm_v, bars + L::kVFull + vs, dh * 64,
-                              (int)(kv_row0 + r0), pol_kv);
-                  tma_load_2d(dst + v_slot_off<D>(1, dh), &tm_v, bars + L::kVFull + vs, dh * 64,
-                              (int)(kv_row0 + r1), pol_kv);
-                }
-              }
+              for (int dh = 0; dh < L::DH; ++dh)
+                tma_load_2d(smem + L::kQOff + dh * 8192, &tm_q, bars + L::kQFull, dh * 64, q_row,
+                            pol_q);
             }
           }
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-          if (!ok) break;
-          ++gp;
+        }
+        const int32_t* idx_row = p.q2k_idx + (x.group * p.nq + x.a) * (long long)p.idx_stride;
+        const int np = (x.num + 1) / 2;
+        const long long kv_row0 = x.group * p.kv_rows_per_group;
+        for (int j0 = 0; ok && j0 < x.num; j0 += 32) {
+          int row, len;
+          resolve_entry(p, x, idx_row, j0 + lane, row, len);
+          const int i_end = min(np, (j0 + 32) / 2);
+          for (int i = j0 / 2; i < i_end; ++i) {
+            const int r0 = __shfl_sync(0xffffffffu, row, 2 * i - j0);
+            const int l0 = __shfl_sync(0xffffffffu, len, 2 * i - j0);
+            int r1 = __shfl_sync(0xffffffffu, row, 2 * i + 1 - j0);
+            int l1 = __shfl_sync(0xffffffffu, len, 2 * i + 1 - j0);
+            if (2 * i + 1 >= x.num) { r1 = r0; l1 = 0; }
+            if (lane == 0) {
+              const int N = is_k ? L::NK : L::NV;
+              const int st = (int)(gp % N);
+              const long long u = gp / N;
+              // One TMA engine serves both producers in request order: K of
+              // pair g waits until V of pair g - kKLead has been requested, so
+              // K requests for far-ahead pairs never queue in front of V
+              // requests that are needed sooner.
+              if (is_k && gp >= kKLead)
+                ok = spin_until_at_least(reinterpret_cast<volatile int*>(smem + L::kVIssuedOff),
+                                         (int)(gp - kKLead + 1), abort_flag, p.status);
+              if (ok && u >= 1)
+                ok = mbar_wait(bars + (is_k ? L::kKEmpty : L::kVEmpty) + st, (uint32_t)((u - 1) & 1),
+                               abort_flag, p.status);
+              if (ok) {
+                uint64_t* full = bars + (is_k ? L::kKFull : L::kVFull) + st;
+                if (is_k) {
+                  kmeta[st] = make_int2(l0, l1);
+                  uint8_t* dst = smem + L::kKOff + st * L::kK2;
+                  mbar_arrive_expect_tx(full, L::kK2);
+#pragma unroll
+                  for (int dh = 0; dh < L::DH; ++dh) {
+                    tma_load_2d(dst + k_slot_off<D>(dh, 0), &tm_k, full, dh * 64, (int)(kv_row0 + r0), pol_kv);
+                    tma_load_2d(dst + k_slot_off<D>(dh, 1), &tm_k, full, dh * 64, (int)(kv_row0 + r1), pol_kv);
+                  }
+                } else {
+                  uint8_t* dst = smem + L::kVOff + st * L::kV2;
+                  mbar_arrive_expect_tx(full, L::kV2);
+#pragma unroll
+                  for (int dh = 0; dh < L::DH; ++dh) {
+                    tma_load_2d(dst + v_slot_off<D>(0, dh), &tm_v, full, dh * 64, (int)(kv_row0 + r0), pol_kv);
+                    tma_load_2d(dst + v_slot_off<D>(1, dh), &tm_v, full, dh * 64, (int)(kv_row0 + r1), pol_kv);
+                  }
+                  *reinterpret_cast<volatile int*>(smem + L::kVIssuedOff) = (int)(gp + 1);
+                }
+              }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            ++gp;
+          }
         }
       }
-    }
-  } else if (warp == 1) {
-    // ===================== MMA issuer =====================
-    if (lane == 0) {
-      // total pairs and items of this CTA: commits that nobody would wait for
-      // are not issued, so no asynchronous arrival outlives the CTA
-      long long total = 0, n_mine = 0;
-      for (long long it = it0; it < n_items; it += it_step, ++n_mine) {
-        const Item x = load_item(p, it);
-        total += (x.num + 1) / 2;
+      // drain: every stage's release (a tcgen05 commit) lands before exit
+      if (ok && lane == 0) {
+        const int N = is_k ? L::NK : L::NV;
+        for (long long g = (gp > N ? gp - N : 0); g < gp; ++g) {
+          if (!mbar_wait(bars + (is_k ? L::kKEmpty : L::kVEmpty) + (int)(g % N),
+                         (uint32_t)((g / N) & 1), abort_flag, p.status))
+            break;
+        }
       }
+      __syncwarp();
+    } else if (warp == 1) {
+      // ===================== score products S^T = K2 . Q^T =====================
+      const uint64_t desc_k = make_sdesc_sw128(sbase + L::kKOff, 16u, 1024u);
+      const uint64_t desc_q = make_sdesc_sw128(sbase + L::kQOff, 16u, 1024u);
+      long long gp = 0, n = 0, n_mine = 0;
+      for (long long it = it0; it < n_items; it += it_step) ++n_mine;
+      bool ok = true;
+      for (long long it = it0; ok && it < n_items; it += it_step, ++n) {
+        const Item x = load_item(p, it);
+        const int np = (x.num + 1) / 2;
+        if (!warp_wait(bars + L::kQFull, (uint32_t)(n & 1), abort_flag, p.status)) { ok = false; break; }
+        for (int i = 0; i < np; ++i, ++gp) {
+          const int sb = (int)(gp % kNS);
+          const int ks = (int)(gp % L::NK);
+          if (!warp_wait(bars + L::kKFull + ks, (uint32_t)((gp / L::NK) & 1), abort_flag, p.status)) { ok = false; break; }
+          if (gp >= kNS && !warp_wait(bars + L::kSEmpty + sb, (uint32_t)((gp / kNS - 1) & 1), abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after_sync();
+          if (elect_one()) {
+            issue_score_desc<D>(tmem_base + 64u * sb, desc_k + (uint64_t)((ks * L::kK2) >> 4), desc_q);
+            umma_commit(bars + L::kSFull + sb);
+            umma_commit(bars + L::kKEmpty + ks);
+            if (i == np - 1 && n + 1 < n_mine) umma_commit(bars + L::kQEmpty);
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (np == 0 && n + 1 < n_mine) {
+          // no products for this item: release its Q tile at once
+          if (elect_one()) umma_commit(bars + L::kQEmpty);
+          __syncwarp();
+        }
+      }
+    } else {
+      // ===================== PV products O^T += V2^T . P^T =====================
+      const uint64_t desc_v = make_sdesc_sw128(sbase + L::kVOff, 8192u, 1024u);
+      const uint64_t desc_p = make_sdesc_sw128(sbase + L::kPOff, 8192u, 1024u);
       long long gp = 0, n = 0;
       bool ok = true;
-      // the PV product runs one step behind the score product
-      long long pv_g = -1, pv_n = 0;
-      int pv_o = 0;
-      bool pv_first = false, pv_last = false;
-      auto issue_pv = [&]() -> bool {
-        const int vs = (int)(pv_g % L::NV);
-        if (!mbar_wait(bars + L::kVFull + vs, (uint32_t)((pv_g / L::NV) & 1), abort_flag, p.status)) return false;
-        if (!mbar_wait(bars + L::kPFull, (uint32_t)(pv_g & 1), abort_flag, p.status)) return false;
-        if (pv_first && pv_n >= 2 &&
-            !mbar_wait(bars + L::kOEmpty + pv_o, (uint32_t)(((pv_n - 2) >> 1) & 1), abort_flag, p.status))
-          return false;
-        tc_fence_after_sync();
-        issue_pv_mma<D>(tmem_base + kTmemO + 64u * pv_o, sbase + L::kVOff + vs * L::kV2,
-                        sbase + L::kPOff, !pv_first);
-        if (pv_g + 1 < total) umma_commit(bars + L::kPEmpty);
-        if (pv_g + L::NV < total) umma_commit(bars + L::kVEmpty + vs);
-        if (pv_last) umma_commit(bars + L::kOFull + pv_o);
-        pv_g = -1;
-        return true;
-      };
       for (long long it = it0; ok && it < n_items; it += it_step, ++n) {
         const Item x = load_item(p, it);
         const int o = (int)(n & 1);
         const int np = (x.num + 1) / 2;
-        if (!mbar_wait(bars + L::kQFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
+        // the epilogue of item n - 2 must have read this output buffer
+        if (n >= 2 && !warp_wait(bars + L::kOEmpty + o, (uint32_t)(((n - 2) >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
         for (int i = 0; i < np; ++i, ++gp) {
-          const int sb = (int)(gp & 1);
-          const int ks = (int)(gp % L::NK);
-          if (!mbar_wait(bars + L::kKFull + ks, (uint32_t)((gp / L::NK) & 1), abort_flag, p.status)) { ok = false; break; }
-          if (gp >= 2 && !mbar_wait(bars + L::kSEmpty + sb, (uint32_t)(((gp - 2) >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
+          const int vs = (int)(gp % L::NV);
+          const int pb = (int)(gp % kNP);
+          if (!warp_wait(bars + L::kVFull + vs, (uint32_t)((gp / L::NV) & 1), abort_flag, p.status)) { ok = false; break; }
+          if (!warp_wait(bars + L::kPFull + pb, (uint32_t)((gp / kNP) & 1), abort_flag, p.status)) { ok = false; break; }
           tc_fence_after_sync();
-          issue_score_mma<D>(tmem_base + 64u * sb, sbase + L::kKOff + ks * L::kK2,
-                             sbase + L::kQOff + o * L::kQ);
-          umma_commit(bars + L::kSFull + sb);
-          if (gp + L::NK < total) umma_commit(bars + L::kKEmpty + ks);
-          if (i == np - 1 && n + 2 < n_mine) umma_commit(bars + L::kQEmpty + o);
-          if (pv_g >= 0 && !issue_pv()) { ok = false; break; }
-          pv_g = gp; pv_n = n; pv_o = o; pv_first = (i == 0); pv_last = (i == np - 1);
+          if (elect_one()) {
+            issue_pv_desc<D>(tmem_base + kTmemO + 64u * o, desc_v + (uint64_t)((vs * L::kV2) >> 4),
+                             desc_p + (uint64_t)((pb * L::kP) >> 4), i > 0);
+            umma_commit(bars + L::kPEmpty + pb);
+            umma_commit(bars + L::kVEmpty + vs);
+            if (i == np - 1) umma_commit(bars + L::kOFull + o);
+          }
+          __syncwarp();
         }
         if (!ok) break;
         if (np == 0) {
-          // empty selection: no products; still hand the O buffer to the
-          // epilogue in order (it writes out_c * gate for this block)
-          if (pv_g >= 0 && !issue_pv()) { ok = false; break; }
-          if (n >= 2 && !mbar_wait(bars + L::kOEmpty + o, (uint32_t)(((n - 2) >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
-          umma_commit(bars + L::kOFull + o);
-          if (n + 2 < n_mine) umma_commit(bars + L::kQEmpty + o);
+          // empty selection: hand the output buffer over in order anyway
+          if (elect_one()) umma_commit(bars + L::kOFull + o);
+          __syncwarp();
         }
       }
-      if (ok && pv_g >= 0) issue_pv();
     }
-  } else if (warp >= 4 && warp < 12) {
+  } else if (warp < 12) {
+    regs_inc<kRegsSoftmax>();
     // ===================== softmax (two groups of 4 warps) =====================
     const int grp = (warp - 4) / 4;              // query columns 32*grp .. 32*grp+31
     const int wq = warp & 3;                     // TMEM lane quarter
@@ -441,15 +511,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = Lr >> 6, r = Lr & 63;
     const uint32_t col0 = 32u * grp;
     const uint32_t t_lane = tmem_base + (uint32_t(wq * 32) << 16);
-    const uint32_t bar_flag = 1 + 2 * grp, bar_red = 2 + 2 * grp;
+    const uint32_t bar_vote = 1 + 2 * grp, bar_red = 2 + 2 * grp;
     float* red = red_all + grp * 128;
     float* fin = fin_all + col0;
-    volatile int* gflags = flags + grp * 8;
-    float* m_g = m_s + col0;
-    float* a_g = alpha_s + col0;
+    float* asc = reinterpret_cast<float*>(smem + L::kAlphaOff) + col0;
     const float c = p.scale_log2;
     long long gp = 0, n = 0;
     bool ok = true;
+    float m[32];                                 // running max per query column (log2 units)
+#pragma unroll
+    for (int q = 0; q < 32; ++q) m[q] = 0.f;
     for (long long it = it0; ok && it < n_items; it += it_step, ++n) {
       const Item x = load_item(p, it);
       const int o = (int)(n & 1);
@@ -457,167 +528,212 @@ __global__ void __launch_bounds__(kThreads, 1)
       float lp[32];
 #pragma unroll
       for (int q = 0; q < 32; ++q) lp[q] = 0.f;
-      for (int i = 0; i < np; ++i, ++gp) {
-        const int sb = (int)(gp & 1);
-        const int ks = (int)(gp % L::NK);
-        if (!mbar_wait(bars + L::kSFull + sb, (uint32_t)((gp >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
+      // Two pairs per iteration (the second may be absent at the end of an
+      // item), so the fixed cost of the handshakes below is paid once per
+      // 4 KV tiles.
+      for (int i = 0; i < np; i += 2) {
+        const bool two = (i + 1 < np);
+        const long long g0 = gp, g1 = gp + 1;
+        bool valid0, valid1 = false;
+        if (!warp_wait(bars + L::kSFull + (int)(g0 % kNS), (uint32_t)((g0 / kNS) & 1), abort_flag, p.status)) { ok = false; break; }
+        if (two && !warp_wait(bars + L::kSFull + (int)(g1 % kNS), (uint32_t)((g1 / kNS) & 1), abort_flag, p.status)) { ok = false; break; }
         // the K stage's barrier also publishes the pair's key counts; the
         // stage cannot be refilled before this group's arrival below
-        if (!mbar_wait(bars + L::kKFull + ks, (uint32_t)((gp / L::NK) & 1), abort_flag, p.status)) { ok = false; break; }
-        const int2 lens = kmeta[ks];
-        const bool valid = r < (half ? lens.y : lens.x);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bars + L::kKEmpty + ks);
-        tc_fence_after_sync();
-        uint32_t sr[32];
-        tmem_ld32(t_lane + 64u * sb + col0, sr);
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bars + L::kSEmpty + sb);
-        bool rescale = (i == 0);
-        if (i > 0) {
-          float worst = -INFINITY;
-          if (valid) {
-#pragma unroll
-            for (int q = 0; q < 32; q += 4) {
-              const float4 mm = *reinterpret_cast<const float4*>(m_g + q);
-              worst = fmaxf(worst, fmaf(__uint_as_float(sr[q]), c, -mm.x));
-              worst = fmaxf(worst, fmaf(__uint_as_float(sr[q + 1]), c, -mm.y));
-              worst = fmaxf(worst, fmaf(__uint_as_float(sr[q + 2]), c, -mm.z));
-              worst = fmaxf(worst, fmaf(__uint_as_float(sr[q + 3]), c, -mm.w));
-            }
+        {
+          const int k0 = (int)(g0 % L::NK);
+          if (!warp_wait(bars + L::kKFull + k0, (uint32_t)((g0 / L::NK) & 1), abort_flag, p.status)) { ok = false; break; }
+          const int2 l0 = kmeta[k0];
+          valid0 = r < (half ? l0.y : l0.x);
+          if (lane == 0) mbar_arrive(bars + L::kKEmpty + k0);
+          if (two) {
+            const int k1 = (int)(g1 % L::NK);
+            if (!warp_wait(bars + L::kKFull + k1, (uint32_t)((g1 / L::NK) & 1), abort_flag, p.status)) { ok = false; break; }
+            const int2 l1 = kmeta[k1];
+            valid1 = r < (half ? l1.y : l1.x);
+            if (lane == 0) mbar_arrive(bars + L::kKEmpty + k1);
           }
-          const int need = __any_sync(0xffffffffu, worst > 8.f) ? 1 : 0;
-          if (lane == 0) gflags[(gp & 1) * 4 + wq] = need;
-          named_barrier_sync(bar_flag, 128);
-          rescale = (gflags[(gp & 1) * 4 + 0] | gflags[(gp & 1) * 4 + 1] |
-                     gflags[(gp & 1) * 4 + 2] | gflags[(gp & 1) * 4 + 3]) != 0;
+        }
+        const uint32_t s0_col = 64u * (uint32_t)(g0 % kNS) + col0;
+        const uint32_t s1_col = 64u * (uint32_t)(g1 % kNS) + col0;
+        tc_fence_after_sync();
+        uint32_t x0[32], x1[32];                 // logits, then log2-domain offsets
+        VSA_TMEM_LD16(t_lane + s0_col, x0, 0);
+        VSA_TMEM_LD16(t_lane + s0_col + 16u, x0, 16);
+        if (two) {
+          VSA_TMEM_LD16(t_lane + s1_col, x1, 0);
+          VSA_TMEM_LD16(t_lane + s1_col + 16u, x1, 16);
+        }
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        bool rescale = (i == 0);
+        {
+          float worst = -INFINITY;
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const float a0 = fmaf(__uint_as_float(x0[q]), c, -m[q]);
+            const float a1 = two ? fmaf(__uint_as_float(x1[q]), c, -m[q]) : -INFINITY;
+            x0[q] = __float_as_uint(a0);
+            x1[q] = __float_as_uint(a1);
+            worst = fmaxf(worst, fmaxf(valid0 ? a0 : -INFINITY, valid1 ? a1 : -INFINITY));
+          }
+          // does any logit exceed the running max by more than 2^8?
+          if (i > 0) rescale = bar_red_or(bar_vote, 128, worst > 8.f);
         }
         if (rescale) {
+          // rare: take the exact column max over this step's valid rows from
+          // the raw logits (the S^T buffers are not released yet), update
+          // the running max, rescale the partial sums and O^T
           {
             float masked[32];
+            tmem_ld32(t_lane + s0_col, x0);
 #pragma unroll
-            for (int q = 0; q < 32; ++q) masked[q] = valid ? __uint_as_float(sr[q]) * c : -INFINITY;
+            for (int q = 0; q < 32; ++q) masked[q] = valid0 ? __uint_as_float(x0[q]) * c : -INFINITY;
+            if (two) {
+              tmem_ld32(t_lane + s1_col, x1);
+#pragma unroll
+              for (int q = 0; q < 32; ++q)
+                masked[q] = fmaxf(masked[q], valid1 ? __uint_as_float(x1[q]) * c : -INFINITY);
+            }
             col_reduce32<true>(masked, red, fin, wq, lane, t128, bar_red);
           }
-          if (t128 < 32) {
-            const float f = fin[t128];
-            if (i == 0) {
-              m_g[t128] = (f == -INFINITY) ? 0.f : f;
-            } else {
-              const float old = m_g[t128];
-              const float nm = fmaxf(old, f);
-              a_g[t128] = fast_exp2(old - nm);
-              m_g[t128] = nm;
-            }
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const float f = fin[q];
+            const float nm = (i == 0) ? ((f == -INFINITY) ? 0.f : f) : fmaxf(m[q], f);
+            const float a = (i == 0) ? 1.f : fast_exp2(m[q] - nm);
+            lp[q] *= a;
+            m[q] = nm;
+            if (t128 == q) asc[q] = a;
           }
           named_barrier_sync(bar_red, 128);
-          if (i > 0) {
+          tmem_ld32(t_lane + s0_col, x0);
+          if (two) tmem_ld32(t_lane + s1_col, x1);
 #pragma unroll
-            for (int q = 0; q < 32; ++q) lp[q] *= a_g[q];
-            // O^T holds this item's PV products up to the previous pair:
-            // wait for the last one, then rescale this lane's columns.
-            if (!mbar_wait(bars + L::kPEmpty, (uint32_t)((gp - 1) & 1), abort_flag, p.status)) { ok = false; break; }
+          for (int q = 0; q < 32; ++q) {
+            x0[q] = __float_as_uint(fmaf(__uint_as_float(x0[q]), c, -m[q]));
+            x1[q] = two ? __float_as_uint(fmaf(__uint_as_float(x1[q]), c, -m[q])) : __float_as_uint(-INFINITY);
+          }
+          if (i > 0) {
+            // O^T holds this item's PV products up to pair g0 - 1: wait for
+            // it, then rescale this lane's columns.
+            const long long gq = g0 - 1;
+            if (!warp_wait(bars + L::kPEmpty + (int)(gq % kNP), (uint32_t)((gq / kNP) & 1), abort_flag, p.status)) { ok = false; break; }
             tc_fence_after_sync();
             uint32_t ov[32];
             tmem_ld32(t_lane + kTmemO + 64u * o + col0, ov);
 #pragma unroll
-            for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * a_g[q]);
+            for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * asc[q]);
             tmem_st32(t_lane + kTmemO + 64u * o + col0, ov);
-            tc_fence_before_sync();
           }
         }
-        uint32_t pk[16];
-#pragma unroll
-        for (int q = 0; q < 32; q += 4) {
-          const float4 mm = *reinterpret_cast<const float4*>(m_g + q);
-          float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-          if (valid) {
-            p0 = fast_exp2(fmaf(__uint_as_float(sr[q]), c, -mm.x));
-            p1 = fast_exp2(fmaf(__uint_as_float(sr[q + 1]), c, -mm.y));
-            p2 = fast_exp2(fmaf(__uint_as_float(sr[q + 2]), c, -mm.z));
-            p3 = fast_exp2(fmaf(__uint_as_float(sr[q + 3]), c, -mm.w));
-          }
-          lp[q] += p0;
-          lp[q + 1] += p1;
-          lp[q + 2] += p2;
-          lp[q + 3] += p3;
-          pk[q / 2] = pack_bf16x2(p0, p1);
-          pk[q / 2 + 1] = pack_bf16x2(p2, p3);
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bars + L::kSEmpty + (int)(g0 % kNS));
+          if (two) mbar_arrive(bars + L::kSEmpty + (int)(g1 % kNS));
         }
-        // the single P^T buffer is free once the previous PV product is done
-        if (gp >= 1 && !mbar_wait(bars + L::kPEmpty, (uint32_t)((gp - 1) & 1), abort_flag, p.status)) { ok = false; break; }
-        uint8_t* pbuf = smem + L::kPOff;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          *reinterpret_cast<uint4*>(pbuf + sw128_off(Lr, 4 * grp + ch)) =
-              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        }
+        // the P^T buffers are free once the PV products two pairs back are done
+        if (g0 >= kNP && !warp_wait(bars + L::kPEmpty + (int)(g0 % kNP), (uint32_t)((g0 / kNP - 1) & 1), abort_flag, p.status)) { ok = false; break; }
+        if (two && g1 >= kNP && !warp_wait(bars + L::kPEmpty + (int)(g1 % kNP), (uint32_t)((g1 / kNP - 1) & 1), abort_flag, p.status)) { ok = false; break; }
+        write_probs(x0, valid0, lp, smem + L::kPOff + (int)(g0 % kNP) * L::kP, Lr, grp);
+        if (two) write_probs(x1, valid1, lp, smem + L::kPOff + (int)(g1 % kNP) * L::kP, Lr, grp);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bars + L::kPFull);
+        if (lane == 0) {
+          mbar_arrive(bars + L::kPFull + (int)(g0 % kNP));
+          if (two) mbar_arrive(bars + L::kPFull + (int)(g1 % kNP));
+        }
+        gp += two ? 2 : 1;
       }
       if (!ok) break;
       // end of item: 1 / row sums for the epilogue
-      if (n >= 2 && !mbar_wait(bars + L::kOEmpty + o, (uint32_t)(((n - 2) >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
+      if (n >= 2 && !warp_wait(bars + L::kOEmpty + o, (uint32_t)(((n - 2) >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
       col_reduce32<false>(lp, red, fin, wq, lane, t128, bar_red);
       if (t128 < 32) inv_l[o * 64 + col0 + t128] = fin[t128] > 0.f ? 1.f / fin[t128] : 0.f;
       named_barrier_sync(bar_red, 128);
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + L::kLFull + o);
     }
-  } else if (warp >= 12) {
+    // drain: the last PV products' releases of the P^T buffers land before exit
+    if (ok) {
+      for (long long g = (gp > kNP ? gp - kNP : 0); g < gp; ++g) {
+        if (!warp_wait(bars + L::kPEmpty + (int)(g % kNP), (uint32_t)((g / kNP) & 1), abort_flag, p.status)) break;
+      }
+    }
+  } else {
+    regs_dec<kRegsEpilogue>();
     // ===================== epilogue =====================
+    // O^T / l leaves TMEM (lane = head dim) in 16-row slices through a small
+    // fp32 tile, so the combine and the global traffic run in row order with
+    // 8-byte loads and stores.
     const int wq = warp & 3;
     const int d = wq * 32 + lane;                // TMEM lane = head dim of O^T
+    const int t128 = (warp - 12) * 32 + lane;
     const uint32_t t_lane = tmem_base + (uint32_t(wq * 32) << 16);
+    const bool active = wq * 32 < D;
+    float* stage = reinterpret_cast<float*>(smem + L::kStageOff);   // [16][D]
+    constexpr int kChunks = 16 * D / 4;                             // 4-float chunks per slice
+    constexpr int kPerThread = kChunks / 128;
+    const int d0 = (t128 % (D / 4)) * 4;                            // fixed per thread
     long long n = 0;
     for (long long it = it0; it < n_items; it += it_step, ++n) {
       const Item x = load_item(p, it);
       const int o = (int)(n & 1);
-      if (!mbar_wait(bars + L::kOFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status)) break;
-      if (!mbar_wait(bars + L::kLFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status)) break;
-      float ov[64];
-      if (wq * 32 < D && x.num > 0) {
-        tc_fence_after_sync();
-        uint32_t raw[32];
-        tmem_ld32(t_lane + kTmemO + 64u * o, raw);
-#pragma unroll
-        for (int q = 0; q < 32; ++q) ov[q] = __uint_as_float(raw[q]) * inv_l[o * 64 + q];
-        tmem_ld32(t_lane + kTmemO + 64u * o + 32u, raw);
-#pragma unroll
-        for (int q = 0; q < 32; ++q) ov[32 + q] = __uint_as_float(raw[q]) * inv_l[o * 64 + 32 + q];
-      } else {
-#pragma unroll
-        for (int q = 0; q < 64; ++q) ov[q] = 0.f;
-      }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bars + L::kOEmpty + o);
-      if (wq * 32 >= D) continue;
-      float oc = 0.f;
-      if (COMBINE) oc = p.out_c[(x.group * p.nq + x.a) * (long long)D + d];
+      if (!warp_wait(bars + L::kOFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status)) break;
+      if (!warp_wait(bars + L::kLFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status)) break;
+      float4 oc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (COMBINE) oc = *reinterpret_cast<const float4*>(p.out_c + (x.group * p.nq + x.a) * (long long)D + d0);
       const long long orow0 = x.group * p.q_rows_per_group + x.q_tok;
       const long long grow0 = ((long long)x.b * p.gate_seq + x.q_tok) * p.H + x.h;
+      for (int rnd = 0; rnd < 4; ++rnd) {
+        if (active) {
+          uint32_t ov[16];
+          if (x.num > 0) {
+            tc_fence_after_sync();
+            VSA_TMEM_LD16(t_lane + kTmemO + 64u * o + 16u * rnd, ov, 0);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+          } else {
 #pragma unroll
-      for (int q = 0; q < 64; ++q) {
-        __nv_bfloat16 val;
-        if (q < x.q_len) {
-          float v = ov[q];
-          if (COMBINE) {
-            if (GATED) {
-              const float g = __bfloat162float(p.gate[(grow0 + (long long)q * p.H) * D + d]);
-              v = fmaf(oc, g, v);
-            } else {
-              v += oc;
-            }
+            for (int q = 0; q < 16; ++q) ov[q] = 0u;
           }
-          val = __float2bfloat16_rn(v);
-        } else {
-          if (p.varlen) continue;
-          val = __float2bfloat16_rn(0.f);
+#pragma unroll
+          for (int q = 0; q < 16; ++q)
+            stage[q * D + d] = __uint_as_float(ov[q]) * inv_l[o * 64 + 16 * rnd + q];
         }
-        p.out[(orow0 + q) * D + d] = val;
+        if (rnd == 3) {
+          // output buffer and 1/l of this item fully read: hand them back
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bars + L::kOEmpty + o);
+        }
+        named_barrier_sync(5, 128);
+#pragma unroll
+        for (int k = 0; k < kPerThread; ++k) {
+          const int c = t128 + 128 * k;
+          const int row = c / (D / 4);
+          const int q = 16 * rnd + row;
+          if (q < x.q_len) {
+            const float4 v4 = *reinterpret_cast<const float4*>(stage + row * D + d0);
+            float v0 = v4.x, v1 = v4.y, v2 = v4.z, v3 = v4.w;
+            if (COMBINE) {
+              if (GATED) {
+                const uint2 graw = *reinterpret_cast<const uint2*>(p.gate + (grow0 + (long long)q * p.H) * D + d0);
+                const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&graw.x));
+                const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&graw.y));
+                v0 = fmaf(oc.x, g01.x, v0);
+                v1 = fmaf(oc.y, g01.y, v1);
+                v2 = fmaf(oc.z, g23.x, v2);
+                v3 = fmaf(oc.w, g23.y, v3);
+              } else {
+                v0 += oc.x; v1 += oc.y; v2 += oc.z; v3 += oc.w;
+              }
+            }
+            *reinterpret_cast<uint2*>(p.out + (orow0 + q) * D + d0) =
+                make_uint2(pack_bf16x2(v0, v1), pack_bf16x2(v2, v3));
+          } else if (!p.varlen) {
+            *reinterpret_cast<uint2*>(p.out + (orow0 + q) * D + d0) = make_uint2(0u, 0u);
+          }
+        }
+        named_barrier_sync(5, 128);
       }
     }
   }
@@ -761,6 +877,14 @@ static int launch_sparse_t(const SparseParams& p, const CUtensorMap& mq, const C
                            const CUtensorMap& mv, cudaStream_t stream) {
   using L = Layout<D>;
   auto kern = sparse_fwd_kernel<D, COMBINE, GATED>;
+  // The warpgroup register split assumes 128 registers per thread at launch;
+  // with fewer, a warpgroup's register increase could never be granted.
+  static int regs_ok = -1;
+  if (regs_ok < 0) {
+    cudaFuncAttributes attr;
+    regs_ok = (cudaFuncGetAttributes(&attr, kern) == cudaSuccess && attr.numRegs == 128) ? 1 : 0;
+  }
+  if (!regs_ok) return VSA_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc) !=
       cudaSuccess)
     return VSA_ERR_CUDA;

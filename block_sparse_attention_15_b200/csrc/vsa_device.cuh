@@ -74,7 +74,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int* status) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_timer_ns();
+  unsigned long long t0 = 0;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0u) {
@@ -85,7 +85,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         *abort_flag = 1;
         return false;
       }
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      // the global timer is read only once a wait has lasted a while
+      if (t0 == 0) t0 = global_timer_ns();
+      else if (global_timer_ns() - t0 > kWaitTimeoutNs) {
         set_status(status, VSA_ERR_DEVICE_TIMEOUT);
         *abort_flag = 1;
         return false;
@@ -254,6 +256,68 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
   VSA_TMEM_ST16(taddr + 0, r, 0);
   VSA_TMEM_ST16(taddr + 16, r, 16);
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Spin (bounded, like mbar_wait) until a shared counter reaches `target`.
+__device__ __forceinline__ bool spin_until_at_least(volatile int* counter, int target,
+                                                    volatile int* abort_flag, int* status) {
+  if (*counter >= target) return true;
+  unsigned long long t0 = 0;
+  for (uint32_t it = 1;; ++it) {
+    if (*counter >= target) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort_flag) return false;
+      if (t0 == 0) t0 = global_timer_ns();
+      else if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+        set_status(status, VSA_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// One lane of the warp waits (bounded) for the phase, then the warp
+// re-converges; the result is the same in every lane.  Only one lane polls
+// the barrier, so a waiting warp costs one shared-memory access per poll.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int* status) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  return ok != 0;
+}
+
+// One lane of the warp (the same every time it is asked under full
+// convergence).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\telect.sync _|P1, 0xffffffff;\n\tselp.b32 %0, 1, 0, P1;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// Named barrier over `n` threads that also ORs a predicate across them.
+__device__ __forceinline__ bool bar_red_or(uint32_t id, uint32_t n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.b32 pi, %1, 0;\n\t"
+      "barrier.cta.red.or.pred po, %2, %3, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+// Move registers between warpgroups (all warps of a warpgroup execute it).
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // 2^x on the special-function unit (PTX ex2.approx, flush-to-zero).
