@@ -83,9 +83,11 @@ struct Layout {
   static constexpr uint32_t kRedOff = kStageOff + 16u * D * 4u; // [2 groups][4 warps][32] f32
   static constexpr uint32_t kFinOff = kRedOff + 2u * 4u * 32u * 4u;  // [64] f32
   static constexpr uint32_t kAlphaOff = kFinOff + 64u * 4u;     // [64] rescale factors
-  static constexpr uint32_t kInvLOff = kAlphaOff + 64u * 4u;    // [2][64] 1 / row sum per O buffer
+  static constexpr uint32_t kMnOff = kAlphaOff + 64u * 4u;      // [64] minus the running max per column
+  static constexpr uint32_t kInvLOff = kMnOff + 64u * 4u;       // [2][64] 1 / row sum per O buffer
   static constexpr uint32_t kKMetaOff = kInvLOff + 2u * 64u * 4u;  // [NK] int2: key counts
-  static constexpr uint32_t kVIssuedOff = kKMetaOff + 32u;        // V pairs requested so far
+  static constexpr uint32_t kSMetaOff = kKMetaOff + 32u;
+  static constexpr uint32_t kVIssuedOff = kSMetaOff + 32u;        // V pairs requested so far
   static constexpr uint32_t kBarOff = kVIssuedOff + 16u;
   // barriers
   static constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + NK,
@@ -212,23 +214,74 @@ __device__ __forceinline__ void col_reduce32(const float (&v)[32], float* red, f
 
 // Probabilities of one key row for 32 query columns: p = 2^x (0 for a
 // masked row), added to the row-sum partials and written as bf16 into this
-// row's half of the swizzled P^T tile.
+// row's half of the swizzled P^T tile.  Three column pairs in eight take the
+// FMA-pipe exponential, the rest the MUFU one, which balances the two units.
 __device__ __forceinline__ void write_probs(const uint32_t (&x)[32], bool valid, float (&lp)[32],
                                             uint8_t* pbuf, int row, int grp) {
   uint32_t pk[16];
+  if (valid) {
 #pragma unroll
-  for (int q = 0; q < 32; q += 2) {
-    const float p0 = valid ? fast_exp2(__uint_as_float(x[q])) : 0.f;
-    const float p1 = valid ? fast_exp2(__uint_as_float(x[q + 1])) : 0.f;
-    lp[q] += p0;
-    lp[q + 1] += p1;
-    pk[q / 2] = pack_bf16x2(p0, p1);
+    for (int j = 0; j < 16; ++j) {
+      const float x0 = __uint_as_float(x[2 * j]), x1 = __uint_as_float(x[2 * j + 1]);
+      const uint64_t pp = ((j & 7) < 3) ? exp2_fma2(x0, x1) : pk2(fast_exp2(x0), fast_exp2(x1));
+      upk2(fadd2(pk2(lp[2 * j], lp[2 * j + 1]), pp), lp[2 * j], lp[2 * j + 1]);
+      float p0, p1;
+      upk2(pp, p0, p1);
+      pk[j] = pack_bf16x2(p0, p1);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) pk[j] = 0u;
   }
 #pragma unroll
   for (int ch = 0; ch < 4; ++ch) {
     *reinterpret_cast<uint4*>(pbuf + sw128_off(row, 4 * grp + ch)) =
         make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
   }
+}
+
+// The rare step of the online softmax (an item's first pair, or a logit more
+// than 2^8 above the running maximum of its column): the exact column maxima
+// over this step's valid key rows, the new running maxima (published in mns),
+// the factors 2^(old - new) (in asc) and, after the first pair, O^T rescaled
+// by them once the PV products so far are done.  Out of line so that its
+// registers do not weigh on the common path.  False if a wait gave up.
+__device__ __noinline__ bool rescale_step(uint32_t t_s0, uint32_t t_s1, bool two, bool valid0,
+                                          bool valid1, float c, bool first, float* red, float* fin,
+                                          float* mns, float* asc, int wq, int lane, int t128,
+                                          uint32_t bar_red, uint64_t* pempty, uint32_t pparity,
+                                          uint32_t t_o, volatile int* abort_flag, int* status) {
+  {
+    uint32_t x[32];
+    float masked[32];
+    tmem_ld32(t_s0, x);
+#pragma unroll
+    for (int q = 0; q < 32; ++q) masked[q] = valid0 ? __uint_as_float(x[q]) * c : -INFINITY;
+    if (two) {
+      tmem_ld32(t_s1, x);
+#pragma unroll
+      for (int q = 0; q < 32; ++q) masked[q] = fmaxf(masked[q], valid1 ? __uint_as_float(x[q]) * c : -INFINITY);
+    }
+    col_reduce32<true>(masked, red, fin, wq, lane, t128, bar_red);
+  }
+  if (t128 < 32) {
+    const float f = fin[t128];
+    const float old = -mns[t128];
+    const float nm = first ? ((f == -INFINITY) ? 0.f : f) : fmaxf(old, f);
+    asc[t128] = first ? 1.f : fast_exp2(old - nm);
+    mns[t128] = -nm;
+  }
+  named_barrier_sync(bar_red, 128);
+  if (!first) {
+    if (!warp_wait(pempty, pparity, abort_flag, status)) return false;
+    tc_fence_after_sync();
+    uint32_t ov[32];
+    tmem_ld32(t_o, ov);
+#pragma unroll
+    for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * asc[q]);
+    tmem_st32(t_o, ov);
+  }
+  return true;
 }
 
 // One work item: query block a of head h of batch b.
@@ -303,6 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* fin_all = reinterpret_cast<float*>(smem + L::kFinOff);
   float* inv_l = reinterpret_cast<float*>(smem + L::kInvLOff);
   int2* kmeta = reinterpret_cast<int2*>(smem + L::kKMetaOff);
+  int2* smeta = reinterpret_cast<int2*>(smem + L::kSMetaOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -318,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if ((i >= L::kSEmpty && i < L::kSEmpty + kNS) || (i >= L::kPFull && i < L::kPFull + kNP) ||
           i == L::kLFull || i == L::kLFull + 1)
         count = 8;  // one arrival per softmax warp
-      if (i >= L::kKEmpty && i < L::kKEmpty + L::NK) count = 9;  // score commit + 8 softmax warps
+      if (i >= L::kSFull && i < L::kSFull + kNS) count = 2;
       if (i == L::kOEmpty || i == L::kOEmpty + 1) count = 4;   // epilogue warps
       mbar_init(bars + i, count);
     }
@@ -450,6 +504,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int ks = (int)(gp % L::NK);
           if (!warp_wait(bars + L::kKFull + ks, (uint32_t)((gp / L::NK) & 1), abort_flag, p.status)) { ok = false; break; }
           if (gp >= kNS && !warp_wait(bars + L::kSEmpty + sb, (uint32_t)((gp / kNS - 1) & 1), abort_flag, p.status)) { ok = false; break; }
+          if (lane == 0) smeta[sb] = kmeta[ks];
+          __syncwarp();
           tc_fence_after_sync();
           if (elect_one()) {
             issue_score_desc<D>(tmem_base + 64u * sb, desc_k + (uint64_t)((ks * L::kK2) >> 4), desc_q);
@@ -458,6 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (i == np - 1 && n + 1 < n_mine) umma_commit(bars + L::kQEmpty);
           }
           __syncwarp();
+          if (lane == 0) mbar_arrive(bars + L::kSFull + sb);
         }
         if (!ok) break;
         if (np == 0 && n + 1 < n_mine) {
@@ -518,9 +575,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.scale_log2;
     long long gp = 0, n = 0;
     bool ok = true;
-    float m[32];                                 // running max per query column (log2 units)
-#pragma unroll
-    for (int q = 0; q < 32; ++q) m[q] = 0.f;
+    // minus the running max per query column (log2 units): the same for all
+    // threads of the group, so it lives in shared memory and is read as
+    // broadcast 16-byte loads (it changes only at a rescale)
+    float* mns = reinterpret_cast<float*>(smem + L::kMnOff) + col0;
+    if (t128 < 32) mns[t128] = 0.f;
+    named_barrier_sync(bar_red, 128);
+    const uint64_t cc = pk2(c, c);
     for (long long it = it0; ok && it < n_items; it += it_step, ++n) {
       const Item x = load_item(p, it);
       const int o = (int)(n & 1);
@@ -535,22 +596,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool two = (i + 1 < np);
         const long long g0 = gp, g1 = gp + 1;
         bool valid0, valid1 = false;
-        if (!warp_wait(bars + L::kSFull + (int)(g0 % kNS), (uint32_t)((g0 / kNS) & 1), abort_flag, p.status)) { ok = false; break; }
-        if (two && !warp_wait(bars + L::kSFull + (int)(g1 % kNS), (uint32_t)((g1 / kNS) & 1), abort_flag, p.status)) { ok = false; break; }
-        // the K stage's barrier also publishes the pair's key counts; the
-        // stage cannot be refilled before this group's arrival below
+        // S^T of pair g1 is committed after that of g0 by the same thread, so
+        // its barrier covers both products (and both key-count records)
         {
-          const int k0 = (int)(g0 % L::NK);
-          if (!warp_wait(bars + L::kKFull + k0, (uint32_t)((g0 / L::NK) & 1), abort_flag, p.status)) { ok = false; break; }
-          const int2 l0 = kmeta[k0];
+          const long long gl = two ? g1 : g0;
+          if (!warp_wait(bars + L::kSFull + (int)(gl % kNS), (uint32_t)((gl / kNS) & 1), abort_flag, p.status)) { ok = false; break; }
+        }
+        {
+          const int2 l0 = smeta[g0 % kNS];
           valid0 = r < (half ? l0.y : l0.x);
-          if (lane == 0) mbar_arrive(bars + L::kKEmpty + k0);
           if (two) {
-            const int k1 = (int)(g1 % L::NK);
-            if (!warp_wait(bars + L::kKFull + k1, (uint32_t)((g1 / L::NK) & 1), abort_flag, p.status)) { ok = false; break; }
-            const int2 l1 = kmeta[k1];
+            const int2 l1 = smeta[g1 % kNS];
             valid1 = r < (half ? l1.y : l1.x);
-            if (lane == 0) mbar_arrive(bars + L::kKEmpty + k1);
           }
         }
         const uint32_t s0_col = 64u * (uint32_t)(g0 % kNS) + col0;
@@ -566,63 +623,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
         bool rescale = (i == 0);
         {
-          float worst = -INFINITY;
+          // offsets s * c - m, two columns per instruction
+          float w0 = -INFINITY, w1 = -INFINITY;
+          const ulonglong2* mn2 = reinterpret_cast<const ulonglong2*>(mns);
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const float a0 = fmaf(__uint_as_float(x0[q]), c, -m[q]);
-            const float a1 = two ? fmaf(__uint_as_float(x1[q]), c, -m[q]) : -INFINITY;
-            x0[q] = __float_as_uint(a0);
-            x1[q] = __float_as_uint(a1);
-            worst = fmaxf(worst, fmaxf(valid0 ? a0 : -INFINITY, valid1 ? a1 : -INFINITY));
+          for (int j = 0; j < 16; ++j) {
+            const ulonglong2 mm = mn2[j / 2];
+            const uint64_t nm = (j & 1) ? mm.y : mm.x;
+            float a, b;
+            upk2(ffma2(pk2(__uint_as_float(x0[2 * j]), __uint_as_float(x0[2 * j + 1])), cc, nm), a, b);
+            x0[2 * j] = __float_as_uint(a);
+            x0[2 * j + 1] = __float_as_uint(b);
+            w0 = fmax3(w0, a, b);
+            if (two) {
+              upk2(ffma2(pk2(__uint_as_float(x1[2 * j]), __uint_as_float(x1[2 * j + 1])), cc, nm), a, b);
+              x1[2 * j] = __float_as_uint(a);
+              x1[2 * j + 1] = __float_as_uint(b);
+              w1 = fmax3(w1, a, b);
+            }
           }
+          const float worst = fmaxf(valid0 ? w0 : -INFINITY, valid1 ? w1 : -INFINITY);
           // does any logit exceed the running max by more than 2^8?
           if (i > 0) rescale = bar_red_or(bar_vote, 128, worst > 8.f);
         }
         if (rescale) {
-          // rare: take the exact column max over this step's valid rows from
-          // the raw logits (the S^T buffers are not released yet), update
-          // the running max, rescale the partial sums and O^T
-          {
-            float masked[32];
-            tmem_ld32(t_lane + s0_col, x0);
+          // rare step, out of line: new running maxima (shared memory), the
+          // factors 2^(old - new) (asc) and O^T rescaled; the partial sums
+          // and the offsets are brought up to date here
+          const long long gq = (i > 0) ? g0 - 1 : 0;
+          if (!rescale_step(t_lane + s0_col, t_lane + s1_col, two, valid0, valid1, c, i == 0, red, fin, mns,
+                            asc, wq, lane, t128, bar_red, bars + L::kPEmpty + (int)(gq % kNP),
+                            (uint32_t)((gq / kNP) & 1), t_lane + kTmemO + 64u * o + col0, abort_flag,
+                            p.status)) { ok = false; break; }
 #pragma unroll
-            for (int q = 0; q < 32; ++q) masked[q] = valid0 ? __uint_as_float(x0[q]) * c : -INFINITY;
-            if (two) {
-              tmem_ld32(t_lane + s1_col, x1);
-#pragma unroll
-              for (int q = 0; q < 32; ++q)
-                masked[q] = fmaxf(masked[q], valid1 ? __uint_as_float(x1[q]) * c : -INFINITY);
-            }
-            col_reduce32<true>(masked, red, fin, wq, lane, t128, bar_red);
-          }
-#pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const float f = fin[q];
-            const float nm = (i == 0) ? ((f == -INFINITY) ? 0.f : f) : fmaxf(m[q], f);
-            const float a = (i == 0) ? 1.f : fast_exp2(m[q] - nm);
-            lp[q] *= a;
-            m[q] = nm;
-            if (t128 == q) asc[q] = a;
-          }
-          named_barrier_sync(bar_red, 128);
+          for (int q = 0; q < 32; ++q) lp[q] *= asc[q];
           tmem_ld32(t_lane + s0_col, x0);
           if (two) tmem_ld32(t_lane + s1_col, x1);
 #pragma unroll
           for (int q = 0; q < 32; ++q) {
-            x0[q] = __float_as_uint(fmaf(__uint_as_float(x0[q]), c, -m[q]));
-            x1[q] = two ? __float_as_uint(fmaf(__uint_as_float(x1[q]), c, -m[q])) : __float_as_uint(-INFINITY);
-          }
-          if (i > 0) {
-            // O^T holds this item's PV products up to pair g0 - 1: wait for
-            // it, then rescale this lane's columns.
-            const long long gq = g0 - 1;
-            if (!warp_wait(bars + L::kPEmpty + (int)(gq % kNP), (uint32_t)((gq / kNP) & 1), abort_flag, p.status)) { ok = false; break; }
-            tc_fence_after_sync();
-            uint32_t ov[32];
-            tmem_ld32(t_lane + kTmemO + 64u * o + col0, ov);
-#pragma unroll
-            for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * asc[q]);
-            tmem_st32(t_lane + kTmemO + 64u * o + col0, ov);
+            const float mq = mns[q];
+            x0[q] = __float_as_uint(fmaf(__uint_as_float(x0[q]), c, mq));
+            x1[q] = two ? __float_as_uint(fmaf(__uint_as_float(x1[q]), c, mq)) : __float_as_uint(-INFINITY);
           }
         }
         tc_fence_before_sync();
@@ -631,9 +672,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(bars + L::kSEmpty + (int)(g0 % kNS));
           if (two) mbar_arrive(bars + L::kSEmpty + (int)(g1 % kNS));
         }
-        // the P^T buffers are free once the PV products two pairs back are done
-        if (g0 >= kNP && !warp_wait(bars + L::kPEmpty + (int)(g0 % kNP), (uint32_t)((g0 / kNP - 1) & 1), abort_flag, p.status)) { ok = false; break; }
-        if (two && g1 >= kNP && !warp_wait(bars + L::kPEmpty + (int)(g1 % kNP), (uint32_t)((g1 / kNP - 1) & 1), abort_flag, p.status)) { ok = false; break; }
+        // the P^T buffers are free once the PV products of pairs g0 - 2 and
+        // g0 - 1 are done; both are committed by one thread in order, so the
+        // barrier of g0 - 1 covers both
+        if (g0 >= 1) {
+          const long long gq = g0 - 1;
+          if (!warp_wait(bars + L::kPEmpty + (int)(gq % kNP), (uint32_t)((gq / kNP) & 1), abort_flag, p.status)) { ok = false; break; }
+        }
         write_probs(x0, valid0, lp, smem + L::kPOff + (int)(g0 % kNP) * L::kP, Lr, grp);
         if (two) write_probs(x1, valid1, lp, smem + L::kPOff + (int)(g1 % kNP) * L::kP, Lr, grp);
         fence_proxy_async_smem();

@@ -327,6 +327,56 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction, two lanes).
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of floats on the FMA pipe, so that part of the
+// exponentials leaves the MUFU unit (which does 16 per cycle per SM) alone.
+// Range reduction x = j + f with j = round(x) (added to the exponent field)
+// and f in [-1/2, 1/2]; 2^f by a cubic fitted by weighted least squares to
+// the relative error on that interval (max relative error 7.5e-5, far below
+// the bf16 rounding of the probabilities).  x is clamped to >= -120, where
+// the result (< 2^-120) is negligible next to the row maximum's 1.
+__device__ __forceinline__ uint64_t exp2_fma2(float x0, float x1) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23: adding it rounds to an integer
+  const uint64_t xx = pk2(fmaxf(x0, -120.f), fmaxf(x1, -120.f));
+  const uint64_t t = fadd2(xx, pk2(kRound, kRound));
+  const uint64_t j = fadd2(t, pk2(-kRound, -kRound));
+  const uint64_t f = ffma2(j, pk2(-1.f, -1.f), xx);
+  uint64_t q = ffma2(f, pk2(0x1.c3f75ep-5f, 0x1.c3f75ep-5f), pk2(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
+  q = ffma2(q, f, pk2(0x1.62f31ap-1f, 0x1.62f31ap-1f));
+  q = ffma2(q, f, pk2(0x1.fff692p-1f, 0x1.fff692p-1f));
+  float q0, q1, t0, t1;
+  upk2(q, q0, q1);
+  upk2(t, t0, t1);
+  // the low bits of t hold j; shifted into the exponent field they scale q by 2^j
+  const float r0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  const float r1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+  return pk2(r0, r1);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
