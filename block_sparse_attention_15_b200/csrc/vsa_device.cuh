@@ -277,11 +277,13 @@ __device__ __forceinline__ bool spin_until_at_least(volatile int* counter, int t
   }
 }
 
-// One lane of the warp waits (bounded) for the phase, then the warp
-// re-converges; the result is the same in every lane.  Only one lane polls
-// the barrier, so a waiting warp costs one shared-memory access per poll.
+// The whole warp waits (bounded) for the phase; the result is the same in
+// every lane.  Fast path: all lanes test the phase in one instruction and
+// agree through a vote, with no divergence (a completed phase costs a few
+// cycles).  Otherwise one lane polls and the warp re-converges after it.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int* status) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
   ok = __shfl_sync(0xffffffffu, ok, 0);
