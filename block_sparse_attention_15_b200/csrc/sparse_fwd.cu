@@ -52,7 +52,7 @@ constexpr uint32_t kRegsProducer = 64, kRegsSoftmax = 192, kRegsEpilogue = 64;
 static_assert(128u * (kRegsProducer + 2u * kRegsSoftmax + kRegsEpilogue) <= 512u * 128u,
               "register split exceeds the launch's 128 registers per thread");
 #ifndef VSA_KLEAD
-#define VSA_KLEAD 4
+#define VSA_KLEAD 6
 #endif
 constexpr int kKLead = VSA_KLEAD;      // K requests run at most this many pairs ahead of V
 constexpr int kNS = 4;                 // S^T buffers in TMEM
@@ -240,14 +240,14 @@ __device__ __forceinline__ void write_probs(const uint32_t (&x)[32], bool valid,
   }
 }
 
-// The rare step of the online softmax (an item's first pair, or a logit more
-// than 2^8 above the running maximum of its column): the exact column maxima
-// over this step's valid key rows, the new running maxima (published in mns),
-// the factors 2^(old - new) (in asc) and, after the first pair, O^T rescaled
-// by them once the PV products so far are done.  Out of line so that its
+// The rare step of the online softmax (a logit more than 2^8 above the
+// running maximum of its column, after an item's first step): the exact
+// column maxima over this step's valid key rows, the new running maxima
+// (published in mns), the factors 2^(old - new) (in asc) and O^T rescaled by
+// them once the PV products so far are done.  Out of line so that its
 // registers do not weigh on the common path.  False if a wait gave up.
 __device__ __noinline__ bool rescale_step(uint32_t t_s0, uint32_t t_s1, bool two, bool valid0,
-                                          bool valid1, float c, bool first, float* red, float* fin,
+                                          bool valid1, float c, float* red, float* fin,
                                           float* mns, float* asc, int wq, int lane, int t128,
                                           uint32_t bar_red, uint64_t* pempty, uint32_t pparity,
                                           uint32_t t_o, volatile int* abort_flag, int* status) {
@@ -265,22 +265,19 @@ __device__ __noinline__ bool rescale_step(uint32_t t_s0, uint32_t t_s1, bool two
     col_reduce32<true>(masked, red, fin, wq, lane, t128, bar_red);
   }
   if (t128 < 32) {
-    const float f = fin[t128];
     const float old = -mns[t128];
-    const float nm = first ? ((f == -INFINITY) ? 0.f : f) : fmaxf(old, f);
-    asc[t128] = first ? 1.f : fast_exp2(old - nm);
+    const float nm = fmaxf(old, fin[t128]);
+    asc[t128] = fast_exp2(old - nm);
     mns[t128] = -nm;
   }
   named_barrier_sync(bar_red, 128);
-  if (!first) {
-    if (!warp_wait(pempty, pparity, abort_flag, status)) return false;
-    tc_fence_after_sync();
-    uint32_t ov[32];
-    tmem_ld32(t_o, ov);
+  if (!warp_wait(pempty, pparity, abort_flag, status)) return false;
+  tc_fence_after_sync();
+  uint32_t ov[32];
+  tmem_ld32(t_o, ov);
 #pragma unroll
-    for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * asc[q]);
-    tmem_st32(t_o, ov);
-  }
+  for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * asc[q]);
+  tmem_st32(t_o, ov);
   return true;
 }
 
@@ -621,7 +618,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           VSA_TMEM_LD16(t_lane + s1_col + 16u, x1, 16);
         }
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        bool rescale = (i == 0);
+        if (i == 0) {
+          // an item's first step: the running max starts as the exact column
+          // max over this step's valid key rows (x0 is loaded again after)
+          float fm[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const float a = valid0 ? __uint_as_float(x0[q]) * c : -INFINITY;
+            const float b = valid1 ? __uint_as_float(x1[q]) * c : -INFINITY;
+            fm[q] = fmaxf(a, b);
+          }
+          col_reduce32<true>(fm, red, fin, wq, lane, t128, bar_red);
+          if (t128 < 32) mns[t128] = (fin[t128] == -INFINITY) ? 0.f : -fin[t128];
+          named_barrier_sync(bar_red, 128);
+          VSA_TMEM_LD16(t_lane + s0_col, x0, 0);
+          VSA_TMEM_LD16(t_lane + s0_col + 16u, x0, 16);
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        }
+        bool rescale = false;
         {
           // offsets s * c - m, two columns per instruction
           float w0 = -INFINITY, w1 = -INFINITY;
@@ -650,8 +664,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // rare step, out of line: new running maxima (shared memory), the
           // factors 2^(old - new) (asc) and O^T rescaled; the partial sums
           // and the offsets are brought up to date here
-          const long long gq = (i > 0) ? g0 - 1 : 0;
-          if (!rescale_step(t_lane + s0_col, t_lane + s1_col, two, valid0, valid1, c, i == 0, red, fin, mns,
+          const long long gq = g0 - 1;
+          if (!rescale_step(t_lane + s0_col, t_lane + s1_col, two, valid0, valid1, c, red, fin, mns,
                             asc, wq, lane, t128, bar_red, bars + L::kPEmpty + (int)(gq % kNP),
                             (uint32_t)((gq / kNP) & 1), t_lane + kTmemO + 64u * o + col0, abort_flag,
                             p.status)) { ok = false; break; }
