@@ -152,6 +152,7 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
   cp.q2k_idx = q2k_idx;
   cp.q2k_num = q2k_num;
   cp.out_c = oc;
+  cp.status = status;
   rc = launch_coarse_topk(cp, D, st);
   if (rc != VSA_OK) return rc;
   prof_record(2, st);

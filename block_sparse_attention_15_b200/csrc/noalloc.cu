@@ -128,6 +128,7 @@ extern "C" int vsa_forward_noalloc(const void* q, const void* k, const void* v, 
   cp.q2k_idx = q2k_idx;
   cp.q2k_num = q2k_num;
   cp.out_c = oc;
+  cp.status = status;
   rc = launch_coarse_topk(cp, D, st);
   if (rc != VSA_OK) return rc;
 

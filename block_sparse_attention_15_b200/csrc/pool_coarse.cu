@@ -91,8 +91,8 @@ __global__ void __launch_bounds__(256) pool_kernel(PoolParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// a2 + a3: coarse attention and top-k.  One CTA of 256 threads per
-// (batch*head, tile of QT query blocks).
+// a2 + a3: coarse attention and top-k.  One CTA of 256 threads (8 warps) per
+// (batch*head, tile of kQT query blocks); two CTAs per SM.
 // ---------------------------------------------------------------------------
 // Order-preserving map from fp32 to uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t float_to_key(float f) {
@@ -104,78 +104,165 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
   return __uint_as_float(u);
 }
 
-template <int D, int QT>
-__global__ void __launch_bounds__(256) coarse_topk_kernel(CoarseParams p) {
-  constexpr int LD = D + 4;           // padded row pitch (floats), keeps float4 alignment
-  constexpr int RT = QT / 16;         // query rows per thread in the score product
-  extern __shared__ __align__(16) float smem[];
-  float* qs = smem;                   // [QT][LD]
-  float* cs = qs + QT * LD;           // [64][LD]   kc or vc chunk
-  float* rowsum = cs + 64 * LD;       // [QT]
-  float* sc = rowsum + QT;            // [QT][nkv_pad]
-  const int nkv_pad = (p.nkv + 63) & ~63;
+constexpr int kQT = 16;        // query blocks per CTA
+constexpr int kCH = 64;        // pooled key / value rows per staged chunk
+
+// Shared memory of one CTA (byte offsets; the score rows have a runtime pitch).
+template <int D>
+struct CoarseSmem {
+  static constexpr int LD = D + 4;  // row pitch in floats: 16-byte column reads hit distinct banks
+  static constexpr uint32_t kQs = 0;                                  // [kQT][LD]
+  static constexpr uint32_t kCs = kQs + kQT * LD * 4;                 // [2][kCH][LD]
+  static constexpr uint32_t kHist = kCs + 2 * kCH * LD * 4;           // [8 warps][256] u32
+  static constexpr uint32_t kRowSum = kHist + 8 * 256 * 4;            // [kQT]
+  static constexpr uint32_t kBars = kRowSum + kQT * 4;                // [3] u64: two chunk buffers, query tile
+  static constexpr uint32_t kSc = kBars + 32;                         // [kQT][sp] f32
+  static_assert(kCs % 128 == 0 && (kCH * LD * 4) % 128 == 0, "TMA destinations");
+  static uint32_t bytes(int sp) { return kSc + (uint32_t)kQT * sp * 4u; }
+};
+
+// k-th largest key of one row by four 8-bit radix passes (most significant
+// digit first) over a per-warp histogram; returns the key T and, in
+// ties_needed, how many keys equal to T belong to the top k.
+__device__ __forceinline__ uint32_t radix_select(const uint32_t* keys, int n, uint32_t k,
+                                                 uint32_t* hist, int lane, uint32_t& ties_needed) {
+  uint32_t prefix = 0u, need = k;
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
+    reinterpret_cast<uint4*>(hist)[2 * lane] = make_uint4(0u, 0u, 0u, 0u);
+    reinterpret_cast<uint4*>(hist)[2 * lane + 1] = make_uint4(0u, 0u, 0u, 0u);
+    __syncwarp();
+    for (int j = lane; j < n; j += 32) {
+      const uint32_t key = keys[j];
+      if ((key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    // lane l owns digits 255-8l down to 248-8l; counts accumulate from the top
+    uint32_t cnt[8], local = 0u;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      cnt[t] = hist[255 - 8 * lane - t];
+      local += cnt[t];
+    }
+    uint32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const uint32_t ball = __ballot_sync(0xffffffffu, incl >= need);
+    const int src = __ffs(ball) - 1;
+    uint32_t digit = 0u, above = 0u;
+    if (lane == src) {
+      uint32_t cum = incl - local;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (cum + cnt[t] >= need) {
+          digit = 255u - 8u * lane - t;
+          above = cum;
+          break;
+        }
+        cum += cnt[t];
+      }
+    }
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    need -= above;
+    prefix |= digit << shift;
+    __syncwarp();
+  }
+  ties_needed = need;
+  return prefix;
+}
+
+// The pooled tensors are read through 3D tensor maps (D, blocks, groups) whose
+// boxes are D + 4 columns wide: the 4 columns past D are out of range and
+// arrive as zeros, which gives the padded row pitch in one TMA request per
+// chunk; rows past a group's last block arrive as zeros too.
+template <int D>
+__global__ void __launch_bounds__(256, 2)
+    coarse_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, CoarseParams p) {
+  using S = CoarseSmem<D>;
+  constexpr int LD = S::LD;
+  constexpr int DV = D / 32;  // head dims per thread in the output product
+  extern __shared__ __align__(128) uint8_t csm[];
+  float* qs = reinterpret_cast<float*>(csm + S::kQs);
+  float* cs = reinterpret_cast<float*>(csm + S::kCs);
+  float* rowsum = reinterpret_cast<float*>(csm + S::kRowSum);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(csm + S::kBars);
+  float* sc = reinterpret_cast<float*>(csm + S::kSc);
+  const int nkv_pad = (p.nkv + kCH - 1) / kCH * kCH;
+  const int sp = nkv_pad + 4;  // score row pitch: rows start on different banks
+  const int nch = nkv_pad / kCH;
 
   const int group = blockIdx.y;
-  const int a0 = blockIdx.x * QT;
-  const int tid = threadIdx.x;
-  const int ty = tid / 16, tx = tid % 16;
-  const float* qc = p.qc + (long long)group * p.nq * D;
-  const float* kc = p.kc + (long long)group * p.nkv * D;
-  const float* vc = p.vc + (long long)group * p.nkv * D;
+  const int a0 = blockIdx.x * kQT;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int ty = lane / 8, tx = lane % 8;
+  volatile int abort_flag_s = 0;
+  volatile int* abort_flag = &abort_flag_s;
 
-  // pooled query tile
-  for (int i = tid; i < QT * (D / 4); i += 256) {
-    const int r = i / (D / 4), c4 = i % (D / 4);
-    float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (a0 + r < p.nq) val = reinterpret_cast<const float4*>(qc + (long long)(a0 + r) * D)[c4];
-    *reinterpret_cast<float4*>(qs + r * LD + 4 * c4) = val;
-  }
-
-  // scores = scale * qc . kc, one 64-block chunk of kc at a time
-  for (int c0 = 0; c0 < nkv_pad; c0 += 64) {
-    __syncthreads();
-    for (int i = tid; i < 64 * (D / 4); i += 256) {
-      const int r = i / (D / 4), c4 = i % (D / 4);
-      float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + r < p.nkv) val = reinterpret_cast<const float4*>(kc + (long long)(c0 + r) * D)[c4];
-      *reinterpret_cast<float4*>(cs + r * LD + 4 * c4) = val;
-    }
-    __syncthreads();
-    float acc[RT][4];
-#pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[r][i] = 0.f;
-#pragma unroll 4
-    for (int d = 0; d < D; d += 4) {
-      float4 qv[RT], kv[4];
-#pragma unroll
-      for (int r = 0; r < RT; ++r) qv[r] = *reinterpret_cast<const float4*>(qs + (ty * RT + r) * LD + d);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) kv[i] = *reinterpret_cast<const float4*>(cs + (tx + 16 * i) * LD + d);
-#pragma unroll
-      for (int r = 0; r < RT; ++r)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[r][i] = fmaf(qv[r].x, kv[i].x, acc[r][i]);
-          acc[r][i] = fmaf(qv[r].y, kv[i].y, acc[r][i]);
-          acc[r][i] = fmaf(qv[r].z, kv[i].z, acc[r][i]);
-          acc[r][i] = fmaf(qv[r].w, kv[i].w, acc[r][i]);
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) sc[(ty * RT + r) * nkv_pad + c0 + tx + 16 * i] = acc[r][i] * p.scale;
+  if (tid == 0) {
+    mbar_init(bars, 1);
+    mbar_init(bars + 1, 1);
+    mbar_init(bars + 2, 1);
+    mbar_fence_init();
   }
   __syncthreads();
+  // chunk stream: kc chunks 0..nch-1, then vc chunks; chunk t lands in buffer t & 1
+  auto issue_chunk = [&](int t) {
+    mbar_arrive_expect_tx(bars + (t & 1), (uint32_t)(kCH * LD * 4));
+    tma_load_3d(cs + (t & 1) * kCH * LD, t < nch ? &tm_k : &tm_v, bars + (t & 1), 0, (t % nch) * kCH, group);
+  };
+  if (tid == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    // pooled query tile (rows past nq arrive as zeros)
+    mbar_arrive_expect_tx(bars + 2, (uint32_t)(kQT * LD * 4));
+    tma_load_3d(qs, &tm_q, bars + 2, 0, a0, group);
+    issue_chunk(0);
+    issue_chunk(1);
+  }
+  warp_wait(bars + 2, 0u, abort_flag, p.status);
+
+  // scores = scale * qc . kc: warp w owns row 8w + tx of each chunk, a
+  // thread query rows ty + 4r
+  for (int t = 0; t < nch; ++t) {
+    // (a wait that gives up has recorded the timeout; later waits give up at once)
+    warp_wait(bars + (t & 1), (uint32_t)((t >> 1) & 1), abort_flag, p.status);
+    const float* cb = cs + (t & 1) * kCH * LD;
+    float acc[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) acc[r] = 0.f;
+#pragma unroll 8
+    for (int d = 0; d < D; d += 4) {
+      float4 qv[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) qv[r] = *reinterpret_cast<const float4*>(qs + (ty + 4 * r) * LD + d);
+      const float4 kv = *reinterpret_cast<const float4*>(cb + (8 * warp + tx) * LD + d);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        acc[r] = fmaf(qv[r].x, kv.x, acc[r]);
+        acc[r] = fmaf(qv[r].y, kv.y, acc[r]);
+        acc[r] = fmaf(qv[r].z, kv.z, acc[r]);
+        acc[r] = fmaf(qv[r].w, kv.w, acc[r]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) sc[(ty + 4 * r) * sp + t * kCH + 8 * warp + tx] = acc[r] * p.scale;
+    __syncthreads();  // buffer t & 1 is free again
+    if (tid == 0 && t + 2 < 2 * nch) issue_chunk(t + 2);
+  }
 
   // per row: top-k on the scaled logits, then the softmax numerators
-  const int warp = tid / 32, lane = tid % 32;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(csm + S::kHist) + warp * 256;
   const int k = p.topk;  // already clamped to [1, nkv]
-  for (int r = warp; r < QT; r += 8) {
+  for (int r = warp; r < kQT; r += 8) {
     const int a = a0 + r;
-    float* row = sc + r * nkv_pad;
+    float* row = sc + r * sp;
     if (a >= p.nq) {
       for (int j = lane; j < nkv_pad; j += 32) row[j] = 0.f;
       if (lane == 0) rowsum[r] = 1.f;
@@ -189,19 +276,9 @@ __global__ void __launch_bounds__(256) coarse_topk_kernel(CoarseParams p) {
       kmax = max(kmax, kk);
     }
     kmax = __reduce_max_sync(0xffffffffu, kmax);
-    // largest T with #{key >= T} >= k: the k-th largest key
-    uint32_t T = 0u;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = T | (1u << bit);
-      uint32_t cnt = 0u;
-      for (int j = lane; j < p.nkv; j += 32) cnt += (keys[j] >= cand) ? 1u : 0u;
-      cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if (cnt >= (uint32_t)k) T = cand;
-    }
-    uint32_t gt = 0u;
-    for (int j = lane; j < p.nkv; j += 32) gt += (keys[j] > T) ? 1u : 0u;
-    gt = __reduce_add_sync(0xffffffffu, gt);
-    const uint32_t ties_needed = (uint32_t)k - gt;
+    __syncwarp();
+    uint32_t ties_needed;
+    const uint32_t T = radix_select(keys, p.nkv, (uint32_t)k, hist, lane, ties_needed);
     // ascending compaction: keys above T, then the lowest-index ties
     int32_t* out_idx = p.q2k_idx + ((long long)group * p.nq + a) * p.idx_stride;
     uint32_t written = 0u, ties_seen = 0u;
@@ -235,52 +312,56 @@ __global__ void __launch_bounds__(256) coarse_topk_kernel(CoarseParams p) {
   }
   __syncthreads();
 
-  // out_c = (e . vc) / rowsum; thread columns tx*4 + 64*j, rows ty*RT + r
-  constexpr int CJ = D / 64;
-  float acc[RT][CJ][4];
+  // out_c = (e . vc) / rowsum: warp w owns a quarter of the head dims (DV
+  // consecutive ones per thread) for query rows 8 (w / 4) + ty + 4r, r < 2
+  const int d0 = (warp % 4) * (D / 4) + tx * DV;
+  const int qr0 = 8 * (warp / 4) + ty;
+  float acc[2][DV];
 #pragma unroll
-  for (int r = 0; r < RT; ++r)
+  for (int r = 0; r < 2; ++r)
 #pragma unroll
-    for (int j = 0; j < CJ; ++j)
+    for (int e = 0; e < DV; ++e) acc[r][e] = 0.f;
+  for (int t = nch; t < 2 * nch; ++t) {
+    // (a wait that gives up has recorded the timeout; later waits give up at once)
+    warp_wait(bars + (t & 1), (uint32_t)((t >> 1) & 1), abort_flag, p.status);
+    const float* cb = cs + (t & 1) * kCH * LD;
+    const int c0 = (t - nch) * kCH;
+#pragma unroll 2
+    for (int c = 0; c < kCH; c += 4) {
+      float4 ev[2];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[r][j][e] = 0.f;
-  for (int c0 = 0; c0 < nkv_pad; c0 += 64) {
-    for (int i = tid; i < 64 * (D / 4); i += 256) {
-      const int r = i / (D / 4), c4 = i % (D / 4);
-      float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + r < p.nkv) val = reinterpret_cast<const float4*>(vc + (long long)(c0 + r) * D)[c4];
-      *reinterpret_cast<float4*>(cs + r * LD + 4 * c4) = val;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int c = 0; c < 64; ++c) {
-      float pr[RT];
+      for (int r = 0; r < 2; ++r) ev[r] = *reinterpret_cast<const float4*>(sc + (qr0 + 4 * r) * sp + c0 + c);
 #pragma unroll
-      for (int r = 0; r < RT; ++r) pr[r] = sc[(ty * RT + r) * nkv_pad + c0 + c];
+      for (int u = 0; u < 4; ++u) {
+        float vv[DV];
+        if constexpr (DV == 4) {
+          const float4 v4 = *reinterpret_cast<const float4*>(cb + (c + u) * LD + d0);
+          vv[0] = v4.x; vv[1] = v4.y; vv[2] = v4.z; vv[3] = v4.w;
+        } else {
+          const float2 v2 = *reinterpret_cast<const float2*>(cb + (c + u) * LD + d0);
+          vv[0] = v2.x; vv[1] = v2.y;
+        }
 #pragma unroll
-      for (int j = 0; j < CJ; ++j) {
-        const float4 vv = *reinterpret_cast<const float4*>(cs + c * LD + 64 * j + 4 * tx);
+        for (int r = 0; r < 2; ++r) {
+          const float pr = u == 0 ? ev[r].x : u == 1 ? ev[r].y : u == 2 ? ev[r].z : ev[r].w;
 #pragma unroll
-        for (int r = 0; r < RT; ++r) {
-          acc[r][j][0] = fmaf(pr[r], vv.x, acc[r][j][0]);
-          acc[r][j][1] = fmaf(pr[r], vv.y, acc[r][j][1]);
-          acc[r][j][2] = fmaf(pr[r], vv.z, acc[r][j][2]);
-          acc[r][j][3] = fmaf(pr[r], vv.w, acc[r][j][3]);
+          for (int e = 0; e < DV; ++e) acc[r][e] = fmaf(pr, vv[e], acc[r][e]);
         }
       }
     }
     __syncthreads();
+    if (tid == 0 && t + 2 < 2 * nch) issue_chunk(t + 2);
   }
 #pragma unroll
-  for (int r = 0; r < RT; ++r) {
-    const int a = a0 + ty * RT + r;
+  for (int r = 0; r < 2; ++r) {
+    const int a = a0 + qr0 + 4 * r;
     if (a >= p.nq) continue;
-    const float inv = 1.f / rowsum[ty * RT + r];
-#pragma unroll
-    for (int j = 0; j < CJ; ++j) {
-      float4 o = make_float4(acc[r][j][0] * inv, acc[r][j][1] * inv, acc[r][j][2] * inv,
-                             acc[r][j][3] * inv);
-      *reinterpret_cast<float4*>(p.out_c + ((long long)group * p.nq + a) * D + 64 * j + 4 * tx) = o;
+    const float inv = 1.f / rowsum[qr0 + 4 * r];
+    float* dst = p.out_c + ((long long)group * p.nq + a) * D + d0;
+    if constexpr (DV == 4) {
+      *reinterpret_cast<float4*>(dst) = make_float4(acc[r][0] * inv, acc[r][1] * inv, acc[r][2] * inv, acc[r][3] * inv);
+    } else {
+      *reinterpret_cast<float2*>(dst) = make_float2(acc[r][0] * inv, acc[r][1] * inv);
     }
   }
 }
@@ -297,25 +378,40 @@ int launch_pool(const PoolParams& p, int D, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
-template <int D, int QT>
+// 3D fp32 map (D, n, groups) over a [groups][n][D] array, boxes of
+// (D + 4) x rows x 1 (the 4 extra columns are out of range: zeros).
+static bool make_pooled_map(CUtensorMap* map, const float* base, int D, int n, int groups, int rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)n, (cuuint64_t)groups};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)n * D * 4};
+  cuuint32_t box[3] = {(cuuint32_t)(D + 4), (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
 static int launch_coarse_t(const CoarseParams& p, cudaStream_t stream) {
-  const int nkv_pad = (p.nkv + 63) & ~63;
-  const size_t smem = sizeof(float) * ((size_t)(QT + 64) * (D + 4) + QT + (size_t)QT * nkv_pad);
+  const int nkv_pad = (p.nkv + kCH - 1) / kCH * kCH;
+  const size_t smem = CoarseSmem<D>::bytes(nkv_pad + 4);
   if (smem > 227 * 1024) return VSA_ERR_UNSUPPORTED;
-  auto kern = coarse_topk_kernel<D, QT>;
+  CUtensorMap mq, mk, mv;
+  if (!make_pooled_map(&mq, p.qc, D, p.nq, p.groups, kQT) || !make_pooled_map(&mk, p.kc, D, p.nkv, p.groups, kCH) ||
+      !make_pooled_map(&mv, p.vc, D, p.nkv, p.groups, kCH))
+    return VSA_ERR_CUDA;
+  auto kern = coarse_topk_kernel<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return VSA_ERR_CUDA;
-  dim3 grid((p.nq + QT - 1) / QT, p.groups);
-  kern<<<grid, 256, smem, stream>>>(p);
+  dim3 grid((p.nq + kQT - 1) / kQT, p.groups);
+  kern<<<grid, 256, smem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
 int launch_coarse_topk(const CoarseParams& p, int D, cudaStream_t stream) {
-  if (p.nkv <= 1280) {
-    return D == 128 ? launch_coarse_t<128, 32>(p, stream) : launch_coarse_t<64, 32>(p, stream);
-  }
-  return D == 128 ? launch_coarse_t<128, 16>(p, stream) : launch_coarse_t<64, 16>(p, stream);
+  return D == 128 ? launch_coarse_t<128>(p, stream) : launch_coarse_t<64>(p, stream);
 }
 
 }  // namespace vsa

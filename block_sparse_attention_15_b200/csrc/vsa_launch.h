@@ -34,6 +34,7 @@ struct CoarseParams {
   int32_t* q2k_idx;
   int32_t* q2k_num;
   float* out_c;    // [groups, nq, D]
+  int* status;     // device status word (wait timeouts)
 };
 
 // One launch of the block-sparse kernel.  Work item = (query block a, head h,
@@ -81,6 +82,14 @@ int launch_rebase(const int32_t* q2k_idx, const int32_t* q2k_num, const int32_t*
 int launch_gather_tokens(const void* src, void* dst, const int64_t* slot_token, int64_t n_tokens,
                          int64_t n_slots, int64_t groups, int D, bool scatter,
                          cudaStream_t stream);
+
+// cuTensorMapEncodeTiled from the driver (through the runtime's entry-point
+// query, so no link against libcuda); null if unavailable.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_fn();
 
 // Device status word of the current device (address via cudaGetSymbolAddress).
 int* device_status_ptr();
