@@ -226,6 +226,22 @@ def config_of(wl: I.Workload, flushed: bool) -> dict:
 # ---------------------------------------------------------------------------
 # the two arms
 # ---------------------------------------------------------------------------
+def max_over_ranks(values, world: int, device):
+    """Element-wise maximum of per-rank timings (every rank gets the result;
+    the slowest rank sets the job's time)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def weak_scaling_value(world: int, flops_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank runs its own copy of the workload
+    (weak scaling), timed as the maximum over ranks."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -320,13 +336,10 @@ def run_ours(args, wl):
     k_pool = sum(e[0].elapsed_time(e[1]) for e in ev_k) / K
     k_coarse = sum(e[1].elapsed_time(e[2]) for e in ev_k) / K
     k_sparse = sum(e[2].elapsed_time(e[3]) for e in ev_k) / K
-    t = torch.tensor([total_ms, k_sparse], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, k_sparse_max = float(t[0]), float(t[1])
+    total_ms, k_sparse_max = max_over_ranks([total_ms, k_sparse], world, dev)
     ms_per_step = total_ms / K
     flops_gpu = wl.flops
-    value = world * flops_gpu / (ms_per_step * 1e-3) / 1e12
+    value = weak_scaling_value(world, flops_gpu, ms_per_step)
 
     # end to end through the public API with host buffers (pinned)
     E = max(1, min(K, args.e2e_steps))
@@ -354,10 +367,7 @@ def run_ours(args, wl):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    te = torch.tensor([e0.elapsed_time(e1) / E], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te[0])
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / E], world, dev)[0]
     h2d = sum(x.numel() * x.element_size() for x in pin)
     d2h = out_h.numel() * out_h.element_size()
     vsa.check_device_status()
@@ -380,7 +390,7 @@ def run_ours(args, wl):
             "kernels_ms": {"pool": k_pool, "coarse_topk": k_coarse, "sparse_combine": k_sparse,
                            "sparse_combine_max_over_ranks": k_sparse_max},
             "forward_frac_of_peak": (flops_gpu / (ms_per_step * 1e-3) / 1e12) / peak,
-            "e2e": {"value": world * flops_gpu / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": weak_scaling_value(world, flops_gpu, e2e_ms), "unit": "TFLOP/s",
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": 3 * K,
             "clocks": clocks,
