@@ -64,7 +64,7 @@ template <int D>
 struct Layout {
   static constexpr int DH = D / 64;                        // 64-element head-dim halves
 #ifndef VSA_NK
-#define VSA_NK 3
+#define VSA_NK 2
 #endif
 #ifndef VSA_NV
 #define VSA_NV 2
