@@ -86,8 +86,8 @@ struct Layout {
   static constexpr uint32_t kMnOff = kAlphaOff + 64u * 4u;      // [64] minus the running max per column
   static constexpr uint32_t kInvLOff = kMnOff + 64u * 4u;       // [2][64] 1 / row sum per O buffer
   static constexpr uint32_t kKMetaOff = kInvLOff + 2u * 64u * 4u;  // [NK] int2: key counts
-  static constexpr uint32_t kSMetaOff = kKMetaOff + 32u;
-  static constexpr uint32_t kVIssuedOff = kSMetaOff + 32u;        // V pairs requested so far
+  static constexpr uint32_t kSMetaOff = kKMetaOff + 8u * NK;       // [kNS] int2: key counts per S^T buffer
+  static constexpr uint32_t kVIssuedOff = kSMetaOff + 8u * kNS;   // V pairs requested so far
   static constexpr uint32_t kBarOff = kVIssuedOff + 16u;
   // barriers
   static constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + NK,
