@@ -27,6 +27,7 @@ import re
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 import numpy as np
@@ -98,6 +99,10 @@ def profiled_traffic():
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """nvidia-smi samples every 50 ms, started ahead of the timed region (its
+    first sample comes ~0.1-0.3 s after launch); only samples that fall inside
+    [start(), stop()] are kept, plus, for a region shorter than one period, the
+    first sample after it."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
@@ -105,6 +110,8 @@ class ClockSampler:
 
     def __init__(self, device_index: int):
         self.proc = None
+        self.lines = []          # (monotonic time, line)
+        self.t0 = self.t1 = None
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
             ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
@@ -114,19 +121,37 @@ class ClockSampler:
                 text=True)
         except Exception:  # noqa: BLE001 - clocks are best effort
             self.proc = None
+            return
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        deadline = time.monotonic() + 5.0
+        while not self.lines and time.monotonic() < deadline and self.proc.poll() is None:
+            time.sleep(0.01)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.monotonic(), line))
+
+    def start(self):
+        self.t0 = time.monotonic()
 
     def stop(self) -> dict:
+        self.t1 = time.monotonic()
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.06)
+        time.sleep(0.12)
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-            out, _ = self.proc.communicate()
+        self.reader.join(timeout=5)
+        t0 = self.t0 if self.t0 is not None else self.t1
+        inside = [ln for t, ln in self.lines if t0 <= t <= self.t1]
+        if not inside:
+            inside = [ln for t, ln in self.lines if t > self.t1][:1]
         sm, smax, reasons, power = [], [], set(), []
-        for line in out.splitlines():
+        for line in inside:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 7:
                 continue
@@ -306,6 +331,7 @@ def run_ours(args, wl):
             flush.fill_(1)
         vsa.vsa_forward(q, k, v, gate, qbs, kbs, topk=wl.topk, out=out, workspace=ws)
 
+    sampler = ClockSampler(local)  # nvidia-smi starts up during the warm-up
     for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
         step()
     torch.cuda.synchronize(dev)
@@ -318,7 +344,7 @@ def run_ours(args, wl):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    sampler = ClockSampler(local)
+    sampler.start()
     ev_step[0].record(stream)
     for i in range(K):
         vsa.set_profile_events(ev_k[i])

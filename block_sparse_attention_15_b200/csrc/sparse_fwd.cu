@@ -56,7 +56,14 @@ static_assert(128u * (kRegsProducer + 2u * kRegsSoftmax + kRegsEpilogue) <= 512u
 #endif
 constexpr int kKLead = VSA_KLEAD;      // K requests run at most this many pairs ahead of V
 constexpr int kNS = 4;                 // S^T buffers in TMEM
-constexpr int kNP = 2;                 // P^T buffers in shared memory
+#ifndef VSA_NP
+#define VSA_NP 2
+#endif
+#ifndef VSA_POLY8
+#define VSA_POLY8 3   // column pairs in eight whose exponential runs on the FMA pipe
+#endif
+constexpr int kNP = VSA_NP;            // P^T buffers in shared memory (even)
+static_assert(kNP >= 2 && kNP % 2 == 0, "two pairs per softmax step");
 constexpr uint32_t kTmemCols = 512;    // S^T buffers at 64*i (i < 4), O^T buffers at 256, 320
 constexpr uint32_t kTmemO = 256;
 
@@ -213,17 +220,16 @@ __device__ __forceinline__ void col_reduce32(const float (&v)[32], float* red, f
 }
 
 // Probabilities of one key row for 32 query columns: p = 2^x (0 for a
-// masked row), added to the row-sum partials and written as bf16 into this
-// row's half of the swizzled P^T tile.  Three column pairs in eight take the
-// FMA-pipe exponential, the rest the MUFU one, which balances the two units.
-__device__ __forceinline__ void write_probs(const uint32_t (&x)[32], bool valid, float (&lp)[32],
-                                            uint8_t* pbuf, int row, int grp) {
-  uint32_t pk[16];
+// masked row), added to the row-sum partials and packed as bf16 pairs.  Three
+// column pairs in eight take the FMA-pipe exponential, the rest the MUFU one,
+// which balances the two units.
+__device__ __forceinline__ void compute_probs(const uint32_t (&x)[32], bool valid, float (&lp)[32],
+                                              uint32_t (&pk)[16]) {
   if (valid) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const float x0 = __uint_as_float(x[2 * j]), x1 = __uint_as_float(x[2 * j + 1]);
-      const uint64_t pp = ((j & 7) < 3) ? exp2_fma2(x0, x1) : pk2(fast_exp2(x0), fast_exp2(x1));
+      const uint64_t pp = ((j & 7) < VSA_POLY8) ? exp2_fma2(x0, x1) : pk2(fast_exp2(x0), fast_exp2(x1));
       upk2(fadd2(pk2(lp[2 * j], lp[2 * j + 1]), pp), lp[2 * j], lp[2 * j + 1]);
       float p0, p1;
       upk2(pp, p0, p1);
@@ -233,6 +239,10 @@ __device__ __forceinline__ void write_probs(const uint32_t (&x)[32], bool valid,
 #pragma unroll
     for (int j = 0; j < 16; ++j) pk[j] = 0u;
   }
+}
+
+// This key row's half of the swizzled P^T tile.
+__device__ __forceinline__ void store_probs(const uint32_t (&pk)[16], uint8_t* pbuf, int row, int grp) {
 #pragma unroll
   for (int ch = 0; ch < 4; ++ch) {
     *reinterpret_cast<uint4*>(pbuf + sw128_off(row, 4 * grp + ch)) =
@@ -686,15 +696,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(bars + L::kSEmpty + (int)(g0 % kNS));
           if (two) mbar_arrive(bars + L::kSEmpty + (int)(g1 % kNS));
         }
-        // the P^T buffers are free once the PV products of pairs g0 - 2 and
-        // g0 - 1 are done; both are committed by one thread in order, so the
-        // barrier of g0 - 1 covers both
-        if (g0 >= 1) {
-          const long long gq = g0 - 1;
+        // the exponentials first, so that they overlap the PV products still
+        // reading the P^T buffers
+        uint32_t pk0[16], pk1[16];
+        compute_probs(x0, valid0, lp, pk0);
+        if (two) compute_probs(x1, valid1, lp, pk1);
+        // the P^T buffers are free once the PV products of pairs g0 - kNP and
+        // g0 + 1 - kNP are done; both are committed by one thread in order, so
+        // the barrier of the later one covers both
+        if (g0 + 1 >= kNP) {
+          const long long gq = g0 + 1 - kNP;
           if (!warp_wait(bars + L::kPEmpty + (int)(gq % kNP), (uint32_t)((gq / kNP) & 1), abort_flag, p.status)) { ok = false; break; }
         }
-        write_probs(x0, valid0, lp, smem + L::kPOff + (int)(g0 % kNP) * L::kP, Lr, grp);
-        if (two) write_probs(x1, valid1, lp, smem + L::kPOff + (int)(g1 % kNP) * L::kP, Lr, grp);
+        store_probs(pk0, smem + L::kPOff + (int)(g0 % kNP) * L::kP, Lr, grp);
+        if (two) store_probs(pk1, smem + L::kPOff + (int)(g1 % kNP) * L::kP, Lr, grp);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {

@@ -147,12 +147,14 @@ def test_sparse_edge_cases():
 
 
 def test_sparse_peaked_softmax_rescale():
-    """Queries scaled x8 make logits far larger than the first pair's max, so
-    the running-max refresh and O rescale path must run."""
+    """Queries scaled x8 and the keys of blocks 4-11 a further x4 put later
+    logits far (tens to hundreds of log2 units) above the first step's max,
+    so the running-max refresh and O rescale path must run."""
     B, H, D = 1, 2, 128
     qs, ks = [64] * 3, [64] * 12
     q = _bhsd(B, H, qs, D, 13, 0, scale=8.0)
     k = _bhsd(B, H, ks, D, 13, 1)
+    k[:, :, 256:] *= 4
     v = _bhsd(B, H, ks, D, 13, 2)
     idx = np.broadcast_to(np.arange(12, dtype=np.int32), (B, H, 3, 12)).copy()
     num = np.full((B, H, 3), 12, dtype=np.int32)
@@ -231,6 +233,50 @@ def test_vsa_forward(case):
     P.assert_outputs_close(got[:, :, rr], want[:, :, rr])
     pad = np.setdiff1d(np.arange(got.shape[2]), rr)
     assert np.all(got[:, :, pad] == 0.0)
+
+
+def _forward_vs_oracle(q, k, v, gate, qs, ks, topk):
+    out, idx, num, out_c = vsa.vsa_forward(
+        q.to(DEV), k.to(DEV), v.to(DEV), None if gate is None else gate.to(DEV), qs, ks, topk=topk,
+        return_out_c=True)
+    vsa.check_device_status()
+    qn, kn, vn = P.to_np(q), P.to_np(k), P.to_np(v)
+    scale = O.default_scale(q.shape[-1])
+    qc, kc, vc = (O.block_pool(x, s) for x, s in ((qn, qs), (kn, ks), (vn, ks)))
+    scores, oc_want = O.coarse_attention(qc, kc, vc, scale)
+    P.check_topk(P.to_np(idx), P.to_np(num), scores, topk)
+    o_s = O.block_sparse_attention(qn, kn, vn, P.to_np(idx), P.to_np(num), qs, ks, scale)
+    want = O.combine(oc_want, o_s, None if gate is None else P.to_np(gate), qs)
+    got = P.to_np(out)
+    rr = P.real_rows(qs)
+    P.assert_outputs_close(got[:, :, rr], want[:, :, rr], rel_rms=2e-2)
+    pad = np.setdiff1d(np.arange(got.shape[2]), rr)
+    assert np.all(got[:, :, pad] == 0.0)
+
+
+def test_forward_large_late_keys_rescale():
+    """Keys of the later blocks x16: logits far above the first step's max, so
+    the forward's running-max refresh and rescale must run."""
+    B, H, D = 1, 2, 128
+    qs, ks = [64] * 4, [64] * 10
+    q = _bhsd(B, H, qs, D, 2400, 0, scale=2.0)
+    k = _bhsd(B, H, ks, D, 2400, 1)
+    k[:, :, 256:] *= 16
+    v = _bhsd(B, H, ks, D, 2400, 2)
+    gate = I.gate_bf16((B, 64 * len(qs), H, D), 2400)
+    _forward_vs_oracle(q, k, v, gate, qs, ks, topk=10)
+
+
+def test_forward_large_padding_rows():
+    """Padding rows of a partial query block hold large values: their logits
+    are computed in the block's tile but must not reach any real row, and the
+    padding rows of the output stay zero."""
+    B, H, D = 1, 2, 128
+    qs, ks = [64, 17, 64], [64] * 6
+    q = _bhsd(B, H, qs, D, 2500, 0, pad_value=30.0)
+    k = _bhsd(B, H, ks, D, 2500, 1)
+    v = _bhsd(B, H, ks, D, 2500, 2)
+    _forward_vs_oracle(q, k, v, None, qs, ks, topk=4)
 
 
 def test_forward_ungated_equals_broadcast_plus_sparse():
