@@ -16,10 +16,11 @@ from .binding import (  # noqa: F401
     lib,
     scatter_tokens,
     vsa_forward,
+    vsa_forward_host,
 )
 
 __all__ = [
     "VSAError", "block_sparse_attn_from_indices", "block_sparse_attn_varlen", "build_vsa_metadata",
     "check_device_status", "gather_tokens", "get_device_status", "lib", "scatter_tokens",
-    "vsa_forward",
+    "vsa_forward", "vsa_forward_host",
 ]

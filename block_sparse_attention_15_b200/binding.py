@@ -46,6 +46,10 @@ SIGNATURES = {
     "vsa_forward_noalloc": (_c_int, [_c_void_p] * 4 + [_c_void_p, _c_void_p] + [_c_int] * 6 +
                             [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p,
                              _c_void_p]),
+    "vsa_forward_host_workspace_size": (_c_size_t, [_c_int] * 8),
+    "vsa_forward_host": (_c_int, [_c_void_p] * 4 + [_c_void_p, _c_void_p] + [_c_int] * 6 +
+                         [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_int,
+                          _c_void_p, _c_size_t, _c_void_p]),
     "block_sparse_attn_from_indices": (_c_int, [_c_void_p] * 7 + [_c_int] * 6 +
                                        [_c_float, _c_void_p, _c_void_p]),
     "block_sparse_attn_varlen_workspace_size": (_c_size_t, [_c_int] * 3),
@@ -178,6 +182,66 @@ def vsa_forward(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=None, *, 
     if return_pooled:
         res.append(pooled_views(workspace, B, H, nq, nkv, D))
     return tuple(res)
+
+
+def vsa_forward_host(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=None, *, topk: int,
+                     scale: float | None = None, idx_stride: int | None = None, out=None,
+                     return_indices: bool = False, return_out_c: bool = False,
+                     heads_per_chunk: int = 0, workspace=None, device=None, stream=None):
+    """Full VSA forward on HOST tensors through ``vsa_forward_host`` (see
+    include/vsa.h): the library stages chunks of heads onto the GPU, runs the
+    forward and copies the results back, overlapping the three.
+
+    q, k, v, gate: CPU bf16 tensors, shapes as in :func:`vsa_forward` (page-locked
+    for the copies to overlap).  Returns ``out`` (a page-locked CPU tensor unless
+    ``out`` is given) and, when asked, the host ``q2k_idx``, ``q2k_num`` and
+    ``out_c``.  The call is asynchronous on ``stream``; synchronise it before
+    reading the results.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, torch.bfloat16, n, device=False)
+        if t.is_cuda:
+            raise ValueError(f"{n} must be a CPU tensor")
+    B, H, Sq, D = q.shape
+    Skv = k.shape[2]
+    if k.shape != (B, H, Skv, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H, Skv_pad, D] matching q")
+    if gate is not None:
+        _require(gate, torch.bfloat16, "gate", device=False)
+        if gate.is_cuda or gate.shape != (B, Sq, H, D):
+            raise ValueError(f"gate must be a CPU [B, Sq_pad, H, D] = {(B, Sq, H, D)} tensor")
+    nq, nkv = Sq // 64, Skv // 64
+    k_eff = min(int(topk), nkv)
+    stride = k_eff if idx_stride is None else int(idx_stride)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    qbs = None if q_block_sizes is None else torch.tensor(list(q_block_sizes), dtype=torch.int32)
+    kbs = None if kv_block_sizes is None else torch.tensor(list(kv_block_sizes), dtype=torch.int32)
+    for bs, n, name in ((qbs, nq, "q_block_sizes"), (kbs, nkv, "kv_block_sizes")):
+        if bs is not None and bs.numel() != n:
+            raise ValueError(f"expected {n} {name}, got {bs.numel()}")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
+    elif out.is_cuda or out.dtype != torch.bfloat16 or out.shape != q.shape or not out.is_contiguous():
+        raise ValueError("out must be a contiguous CPU bf16 tensor shaped like q")
+    q2k_idx = torch.empty((B, H, nq, stride), dtype=torch.int32, pin_memory=True) if return_indices else None
+    q2k_num = torch.empty((B, H, nq), dtype=torch.int32, pin_memory=True) if return_indices else None
+    out_c = torch.empty((B, H, nq, D), dtype=torch.float32, pin_memory=True) if return_out_c else None
+    L = lib()
+    ws_bytes = L.vsa_forward_host_workspace_size(B, H, nq, nkv, D, stride, 1 if gate is not None else 0,
+                                                 int(heads_per_chunk))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check("vsa_forward_host", L.vsa_forward_host(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(qbs), _ptr(kbs), B, H, Sq, Skv, D, int(topk),
+            float(scale) if scale is not None else 0.0, _ptr(out), _ptr(q2k_idx), _ptr(q2k_num), stride,
+            _ptr(out_c), int(heads_per_chunk), _ptr(workspace), workspace.numel(), _stream(stream)))
+    res = [out]
+    if return_indices:
+        res += [q2k_idx, q2k_num]
+    if return_out_c:
+        res.append(out_c)
+    return res[0] if len(res) == 1 else tuple(res)
 
 
 def pooled_views(workspace, B, H, nq, nkv, D):

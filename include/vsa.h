@@ -164,6 +164,41 @@ int vsa_forward_noalloc(const void* q, const void* k, const void* v, const void*
                         int32_t* q2k_idx, int32_t* q2k_num, int idx_stride, float* out_c,
                         void* stream);
 
+/*
+ * vsa_forward_host -- vsa_forward on tensors in HOST memory.  The library
+ * copies the inputs into `workspace` and the results back, in chunks of
+ * heads, so that the copies in, the kernels and the copies out of
+ * consecutive chunks overlap.  Each chunk is one vsa_forward call (batch of
+ * one, the chunk's heads) on the caller's stream, so results equal a single
+ * vsa_forward on the same data bit for bit.  The pages define the forward
+ * only (see vsa_forward); this entry point is the host-data path around it.
+ *
+ * q, k, v, gate, out: host, same shapes and types as in vsa_forward.  The
+ *          copies overlap the kernels only when these are page-locked
+ *          (cudaHostAlloc / cudaHostRegister); pageable memory works but
+ *          serialises the copies.  All must stay valid and unchanged until
+ *          `stream` has completed the call.
+ * q_block_sizes, kv_block_sizes  host int32 or NULL, as in vsa_forward
+ * q2k_idx, q2k_num, out_c  host outputs as in vsa_forward, or NULL to skip
+ *          copying them back
+ * heads_per_chunk  heads per chunk, 0 = about eight chunks in all
+ * workspace  device, >= vsa_forward_host_workspace_size(...) bytes,
+ *          256-aligned; two chunks' inputs, outputs and forward scratch
+ * stream   the caller's stream: the kernels run on it and it waits for the
+ *          last copy out, so synchronising it completes the call.  The
+ *          copies run on two streams the library keeps per device.
+ *
+ * Errors are returned before anything is enqueued, except VSA_ERR_CUDA from
+ * a failed enqueue, after which part of the work may be queued.
+ */
+size_t vsa_forward_host_workspace_size(int B, int H, int n_q_blocks, int n_kv_blocks, int D,
+                                       int idx_stride, int gated, int heads_per_chunk);
+int vsa_forward_host(const void* q, const void* k, const void* v, const void* gate,
+                     const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B, int H,
+                     int Sq_pad, int Skv_pad, int D, int topk, float scale, void* out,
+                     int32_t* q2k_idx, int32_t* q2k_num, int idx_stride, float* out_c,
+                     int heads_per_chunk, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ======================================================================== *
  * a4: block-sparse attention from indices
  * ======================================================================== */

@@ -93,6 +93,51 @@ def test_forward_host_argument_checks():
     assert _fwd(lib, **base, ws=fake + 64, wsb=1 << 30) == 7            # misaligned workspace
 
 
+def _fwd_host(lib, **kw):
+    args = dict(q=1, k=1, v=1, gate=None, qbs=None, kbs=None, B=1, H=1, Sq=64, Skv=64, D=128,
+                topk=1, scale=0.0, out=1, idx=None, num=None, stride=1, out_c=None, hpc=0, ws=None,
+                wsb=0)
+    args.update(kw)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.vsa_forward_host(v(args["q"]), v(args["k"]), v(args["v"]), v(args["gate"]),
+                                v(args["qbs"]), v(args["kbs"]), args["B"], args["H"], args["Sq"],
+                                args["Skv"], args["D"], args["topk"], args["scale"], v(args["out"]),
+                                v(args["idx"]), v(args["num"]), args["stride"], v(args["out_c"]),
+                                args["hpc"], v(args["ws"]), args["wsb"], None)
+
+
+def test_forward_host_entry_argument_checks():
+    """The host-buffer forward rejects bad arguments before it enqueues anything."""
+    lib = _lib()
+    fake = 1 << 20
+    base = dict(q=fake, k=fake, v=fake, out=fake)
+    assert _fwd_host(lib, **{**base, "out": None}) == 1                 # null output
+    assert _fwd_host(lib, **base, D=96) == 3                            # unsupported head dim
+    assert _fwd_host(lib, **base, Skv=100) == 2                         # not 64 * n
+    assert _fwd_host(lib, **base, hpc=-1) == 1                          # negative chunk
+    assert _fwd_host(lib, **base, Sq=64 * 4, Skv=64 * 4, topk=3, stride=2) == 2
+    assert _fwd_host(lib, **base) == 7                                  # no workspace
+    need = lib.vsa_forward_host_workspace_size(1, 1, 1, 1, 128, 1, 0, 0)
+    assert _fwd_host(lib, **base, ws=fake, wsb=need - 1) == 7           # too small
+    assert _fwd_host(lib, **base, ws=fake + 64, wsb=need) == 7          # misaligned
+
+
+def test_forward_host_workspace_size():
+    """Two slots of one chunk each: inputs, outputs and a forward workspace."""
+    lib = _lib()
+    a = lambda x: (x + 255) // 256 * 256
+    B, H, nq, nkv, D, stride = 1, 56, 242, 242, 128, 48
+    hc = 7  # about eight chunks of 56 heads
+    fwd = lib.vsa_forward_workspace_size(1, hc, nq, nkv, D)
+    slot = (a(hc * 64 * nq * D * 2) + 2 * a(hc * 64 * nkv * D * 2) + a(64 * nq * hc * D * 2) +
+            a(hc * 64 * nq * D * 2) + a(hc * nq * stride * 4) + a(hc * nq * 4) + a(hc * nq * D * 4) + a(fwd))
+    assert lib.vsa_forward_host_workspace_size(B, H, nq, nkv, D, stride, 1, 0) == a(4 * (nq + nkv)) + 2 * slot
+    # an explicit chunk of all heads needs more; ungated needs less; bad sizes give 0
+    assert lib.vsa_forward_host_workspace_size(B, H, nq, nkv, D, stride, 1, H) > 2 * slot
+    assert lib.vsa_forward_host_workspace_size(B, H, nq, nkv, D, stride, 0, 0) < a(4 * (nq + nkv)) + 2 * slot
+    assert lib.vsa_forward_host_workspace_size(B, H, 0, nkv, D, stride, 1, 0) == 0
+
+
 def test_varlen_host_argument_checks():
     lib = _lib()
     from block_sparse_attention_15_b200.binding import _P32

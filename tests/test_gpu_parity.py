@@ -431,3 +431,36 @@ def test_tile_gather_scatter(shape):
     assert np.array_equal(P.to_np(xp).reshape(want.shape), want)
     back = vsa.scatter_tokens(xp, slot, N)
     assert torch.equal(back.cpu().reshape(x.shape), x)
+
+
+# ---------------------------------------------------------------------------
+# the host-buffer forward: chunked copies around the same forward
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("pinned", [True, False])
+@pytest.mark.parametrize("case", [
+    # B, H, D, q sizes, kv sizes, topk, gated, heads per chunk
+    (2, 5, 128, [64, 64, 64, 20, 64, 64], [64] * 5 + [3] + [64] * 2, 3, True, 2),
+    (1, 9, 64, [64] * 7, [64] * 9, 4, False, 0),
+], ids=["B2-H5-gated-chunk2", "B1-H9-default-chunks"])
+def test_forward_host_equals_device_forward(case, pinned):
+    """vsa_forward_host on host tensors returns exactly what vsa_forward
+    returns on the same data on the device (every chunk is one vsa_forward)."""
+    B, H, D, qs, ks, topk, gated, hpc = case
+    q = _bhsd(B, H, qs, D, 2700, 0)
+    k = _bhsd(B, H, ks, D, 2700, 1)
+    v = _bhsd(B, H, ks, D, 2700, 2)
+    gate = I.gate_bf16((B, 64 * len(qs), H, D), 2700) if gated else None
+    host = [t.pin_memory() if pinned else t for t in (q, k, v)]
+    gh = None if gate is None else (gate.pin_memory() if pinned else gate)
+    out_h, idx_h, num_h, oc_h = vsa.vsa_forward_host(
+        host[0], host[1], host[2], gh, qs, ks, topk=topk, return_indices=True, return_out_c=True,
+        heads_per_chunk=hpc)
+    torch.cuda.current_stream().synchronize()
+    vsa.check_device_status()
+    out, idx, num, oc = vsa.vsa_forward(q.to(DEV), k.to(DEV), v.to(DEV), None if gate is None else gate.to(DEV),
+                                        qs, ks, topk=topk, return_out_c=True)
+    vsa.check_device_status()
+    assert torch.equal(out_h, out.cpu())
+    assert torch.equal(idx_h, idx.cpu())
+    assert torch.equal(num_h, num.cpu())
+    assert torch.equal(oc_h, oc.cpu())
