@@ -433,6 +433,108 @@ def run_ours(args, wl):
     return 0
 
 
+def run_varlen(args):
+    """Varlen entry (a6 + a4): four sequences packed virtually, one call per
+    step; the whole call is timed (a small host-to-device copy of the block
+    tables, then one sparse-kernel launch)."""
+    import torch.distributed as dist
+    from block_sparse_attention_15_b200 import binding as vsa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    H, D, frac, seed = 24, 128, 0.15, 1004
+    q_lens, kv_lens = I.VARLEN_Q_LENS, I.VARLEN_KV_LENS
+    cu_q, cu_kv = I.cu_seqlens(q_lens), I.cu_seqlens(kv_lens)
+    q_h = I.normal_bf16((H, cu_q[-1], D), seed, I.STREAM_Q)
+    k_h = I.normal_bf16((H, cu_kv[-1], D), seed, I.STREAM_K)
+    v_h = I.normal_bf16((H, cu_kv[-1], D), seed, I.STREAM_V)
+    idx_np, num_np, ks = I.varlen_random_selection(q_lens, kv_lens, H, frac, seed)
+    tiles = int(num_np.sum())
+    flops = 4.0 * 64 * 64 * D * tiles
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    idx, num = torch.from_numpy(idx_np).to(dev), torch.from_numpy(num_np).to(dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        vsa.block_sparse_attn_varlen(q, k, v, cu_q, cu_kv, idx, num, out=out)
+
+    sampler = ClockSampler(local)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    vsa.check_device_status()
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    vsa.check_device_status()
+    ms = max_over_ranks([e0.elapsed_time(e1) / K], world, dev)[0]
+    # end to end: page-locked host tensors copied in, the call, the output copied back
+    pin = [x.pin_memory() for x in (q_h, k_h, v_h)]
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        q.copy_(pin[0], non_blocking=True)
+        k.copy_(pin[1], non_blocking=True)
+        v.copy_(pin[2], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+
+    E = max(1, min(K, args.e2e_steps))
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / E], world, dev)[0]
+    if rank == 0:
+        peaks, peak_kind = load_peaks()
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        value = weak_scaling_value(world, flops, ms)
+        line = {
+            "metric": "VSA varlen block-sparse attention ms & effective TFLOPS (selected tiles)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"varlen: 4 sequences, Q {list(q_lens)}, KV {list(kv_lens)}, H{H} D{D}, "
+                                   f"top {frac:.0%} per sequence (k = {ks}), uniformly random selections",
+                       "selected_tiles_per_gpu": tiles, "l2": "inputs larger than L2 (126 MB) every step",
+                       "per_gpu_work": "fixed (weak)"},
+            "roofline": {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peak,
+                         "unit": "TFLOP/s", "frac": flops / (ms * 1e-3) / 1e12 / peak, "traffic": None,
+                         "kernel": "whole varlen call (block-table copy + sparse kernel)",
+                         "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS)"},
+            "e2e": {"value": weak_scaling_value(world, flops, e2e_ms), "unit": "TFLOP/s",
+                    "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in pin),
+                    "d2h_bytes_per_step": out_h.numel() * out_h.element_size()},
+            "gpu_launches": K,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -448,6 +550,12 @@ def main(argv=None):
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (smaller cases for profiler captures)")
     args = ap.parse_args(argv)
+    if args.workload == "varlen":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the "
+                              "default workload; the varlen line has no oracle timing"}), flush=True)
+            return 0
+        return run_varlen(args)
     wl = make_workload(args.workload)
     if args.heads > 0:
         wl.H = args.heads

@@ -1,10 +1,11 @@
 """Seeded synthetic inputs for the VSA forward path.
 
 This module holds random-number generation and tensor layout only: it draws
-N(0,1) activations, sigmoid gates and sequence-length mixes, and places tokens
-into the padded 64-slot block layout that every entry point consumes.  It does
-none of the method's arithmetic (no pooling, no attention, no selection), so
-the CPU oracle and the CUDA library can both be fed from it.
+N(0,1) activations, sigmoid gates, sequence-length mixes and uniformly random
+block selections (inputs of the entry points that take indices), and places
+tokens into the padded 64-slot block layout that every entry point consumes.
+It does none of the method's arithmetic (no pooling, no attention, no top-k),
+so the CPU oracle and the CUDA library can both be fed from it.
 
 Recipe (used by the tests and by ``bench.py``):
 
@@ -25,6 +26,7 @@ from __future__ import annotations
 import math
 from dataclasses import dataclass, field
 
+import numpy as np
 import torch
 
 BLOCK = 64  # tokens per block slot group (the 64-token VSA tile)
@@ -153,3 +155,25 @@ def cu_seqlens(lengths) -> list[int]:
     for n in lengths:
         out.append(out[-1] + int(n))
     return out
+
+
+def varlen_random_selection(q_lens, kv_lens, H: int, frac: float, seed: int):
+    """Seeded per-sequence block selections for the varlen entry: for every
+    sequence i, query block and head (in that order), topk_count(frac, n_kv_i)
+    distinct KV blocks of sequence i drawn uniformly, ascending, with -1 after
+    them.  Returns (q2k_idx int32 [H, total_q_blocks, max_k], q2k_num int32
+    [H, total_q_blocks], per-sequence k)."""
+    nq = [-(-int(n) // BLOCK) for n in q_lens]
+    nkv = [-(-int(n) // BLOCK) for n in kv_lens]
+    ks = [topk_count(frac, n) for n in nkv]
+    rng = np.random.default_rng(seed)
+    idx = np.full((H, sum(nq), max(ks)), -1, dtype=np.int32)
+    num = np.zeros((H, sum(nq)), dtype=np.int32)
+    row = 0
+    for i in range(len(nq)):
+        for _ in range(nq[i]):
+            for h in range(H):
+                idx[h, row, :ks[i]] = np.sort(rng.choice(nkv[i], size=ks[i], replace=False))
+                num[h, row] = ks[i]
+            row += 1
+    return idx, num, ks

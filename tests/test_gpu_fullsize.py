@@ -136,20 +136,9 @@ def test_varlen_full():
     k = I.normal_bf16((H, cu_kv[-1], D), seed, 1)
     v = I.normal_bf16((H, cu_kv[-1], D), seed, 2)
     nq = [-(-n // 64) for n in q_lens]
-    nkv = [-(-n // 64) for n in kv_lens]
-    ks = [I.topk_count(0.15, n) for n in nkv]
+    idx, num, ks = I.varlen_random_selection(q_lens, kv_lens, H, 0.15, seed)
     assert ks == [7, 16, 21, 30]
-    rng = np.random.default_rng(seed)
-    width = max(ks)
-    idx = np.full((H, sum(nq), width), -1, dtype=np.int32)
-    num = np.zeros((H, sum(nq)), dtype=np.int32)
-    row = 0
-    for i in range(4):
-        for _ in range(nq[i]):
-            for h in range(H):
-                idx[h, row, :ks[i]] = np.sort(rng.choice(nkv[i], size=ks[i], replace=False))
-                num[h, row] = ks[i]
-            row += 1
+    rng = np.random.default_rng(seed + 1)
     out, pq, pkv, reb = vsa.block_sparse_attn_varlen(
         q.to(DEV), k.to(DEV), v.to(DEV), cu_q, cu_kv, torch.from_numpy(idx).to(DEV),
         torch.from_numpy(num).to(DEV), return_aux=True)
