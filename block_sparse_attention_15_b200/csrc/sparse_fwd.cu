@@ -47,6 +47,11 @@
 
 namespace vsa {
 
+template <bool B>
+struct BoolTag {
+  static constexpr bool value = B;
+};
+
 constexpr int kThreads = 512;
 constexpr uint32_t kRegsProducer = 64, kRegsSoftmax = 192, kRegsEpilogue = 64;
 static_assert(128u * (kRegsProducer + 2u * kRegsSoftmax + kRegsEpilogue) <= 512u * 128u,
@@ -596,18 +601,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       float lp[32];
 #pragma unroll
       for (int q = 0; q < 32; ++q) lp[q] = 0.f;
-      // Two pairs per iteration (the second may be absent at the end of an
-      // item), so the fixed cost of the handshakes below is paid once per
-      // 4 KV tiles.
-      for (int i = 0; i < np; i += 2) {
-        const bool two = (i + 1 < np);
+      // One step: two pairs (the second may be absent at the end of an
+      // item), so the fixed cost of the handshakes is paid once per 4 KV
+      // tiles.  The step is compiled once for two pairs and once for one, so
+      // that the common two-pair step carries no run-time tests of the pair
+      // count.  (A third copy for two pairs of full blocks, free of the masked
+      // key-row tests, ran slower: instruction-cache pressure.)
+      auto step = [&](int i, auto two_tag) -> bool {
+        constexpr bool two = decltype(two_tag)::value;
         const long long g0 = gp, g1 = gp + 1;
         bool valid0, valid1 = false;
         // S^T of pair g1 is committed after that of g0 by the same thread, so
         // its barrier covers both products (and both key-count records)
         {
           const long long gl = two ? g1 : g0;
-          if (!warp_wait(bars + L::kSFull + (int)(gl % kNS), (uint32_t)((gl / kNS) & 1), abort_flag, p.status)) { ok = false; break; }
+          if (!warp_wait(bars + L::kSFull + (int)(gl % kNS), (uint32_t)((gl / kNS) & 1), abort_flag, p.status)) return false;
         }
         {
           const int2 l0 = smeta[g0 % kNS];
@@ -678,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!rescale_step(t_lane + s0_col, t_lane + s1_col, two, valid0, valid1, c, red, fin, mns,
                             asc, wq, lane, t128, bar_red, bars + L::kPEmpty + (int)(gq % kNP),
                             (uint32_t)((gq / kNP) & 1), t_lane + kTmemO + 64u * o + col0, abort_flag,
-                            p.status)) { ok = false; break; }
+                            p.status)) return false;
 #pragma unroll
           for (int q = 0; q < 32; ++q) lp[q] *= asc[q];
           tmem_ld32(t_lane + s0_col, x0);
@@ -706,7 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the barrier of the later one covers both
         if (g0 + 1 >= kNP) {
           const long long gq = g0 + 1 - kNP;
-          if (!warp_wait(bars + L::kPEmpty + (int)(gq % kNP), (uint32_t)((gq / kNP) & 1), abort_flag, p.status)) { ok = false; break; }
+          if (!warp_wait(bars + L::kPEmpty + (int)(gq % kNP), (uint32_t)((gq / kNP) & 1), abort_flag, p.status)) return false;
         }
         store_probs(pk0, smem + L::kPOff + (int)(g0 % kNP) * L::kP, Lr, grp);
         if (two) store_probs(pk1, smem + L::kPOff + (int)(g1 % kNP) * L::kP, Lr, grp);
@@ -717,6 +725,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (two) mbar_arrive(bars + L::kPFull + (int)(g1 % kNP));
         }
         gp += two ? 2 : 1;
+        return true;
+      };
+      for (int i = 0; i < np; i += 2) {
+        const bool more = (i + 1 < np) ? step(i, BoolTag<true>{}) : step(i, BoolTag<false>{});
+        if (!more) { ok = false; break; }
       }
       if (!ok) break;
       // end of item: 1 / row sums for the epilogue
