@@ -83,7 +83,8 @@ int vsa_get_device_status(void* stream) {
 size_t vsa_forward_workspace_size(int B, int H, int n_q_blocks, int n_kv_blocks, int D) {
   if (B <= 0 || H <= 0 || n_q_blocks <= 0 || n_kv_blocks <= 0 || D <= 0) return 0;
   const size_t g = (size_t)B * H * D * sizeof(float);
-  return align256(g * n_q_blocks) * 2 + align256(g * n_kv_blocks) * 2;
+  const size_t norms = (size_t)B * H * (2 * (size_t)n_q_blocks + n_kv_blocks) * sizeof(float);
+  return align256(g * n_q_blocks) * 2 + align256(g * n_kv_blocks) * 2 + align256(norms);
 }
 
 int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
@@ -119,6 +120,12 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
   float* vc = reinterpret_cast<float*>(ws);
   ws += align256(g * nkv);
   float* oc = out_c ? out_c : reinterpret_cast<float*>(ws);
+  ws += align256(g * nq);
+  // block row norms and the per-query-block logit bound
+  const size_t G = (size_t)B * H;
+  float* qn = reinterpret_cast<float*>(ws);
+  float* kn = qn + G * nq;
+  float* qk_bound = kn + G * nkv;
 
   PoolParams pp;
   pp.q = static_cast<const __nv_bfloat16*>(q);
@@ -132,6 +139,8 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
   pp.qc = qc;
   pp.kc = kc;
   pp.vc = vc;
+  pp.qn = qn;
+  pp.kn = kn;
   pp.status = status;
   prof_record(0, st);
   int rc = launch_pool(pp, D, st);
@@ -152,6 +161,10 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
   cp.q2k_idx = q2k_idx;
   cp.q2k_num = q2k_num;
   cp.out_c = oc;
+  cp.qn = qn;
+  cp.kn = kn;
+  cp.qk_bound = qk_bound;
+  cp.bound_scale = sc * 1.4426950408889634f * (1.f + 0x1p-8f);
   cp.status = status;
   rc = launch_coarse_topk(cp, D, st);
   if (rc != VSA_OK) return rc;
@@ -175,6 +188,7 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
   sp.kv_rows_per_group = Skv_pad;
   sp.gate_seq = Sq_pad;
   sp.scale_log2 = sc * 1.4426950408889634f;
+  sp.qk_bound = qk_bound;
   sp.varlen = 0;
   sp.status = status;
   rc = launch_sparse(sp, q, k, v, (long long)B * H * Sq_pad, (long long)B * H * Skv_pad, D,

@@ -74,9 +74,12 @@ extern "C" int vsa_forward_noalloc(const void* q, const void* k, const void* v, 
   if (mis & 15u) return VSA_ERR_INVALID_ARG;
 
   // Scratch plan, same order as vsa_forward's workspace: pooled q, pooled k,
-  // pooled v, then the coarse output unless the caller receives it in out_c.
+  // pooled v, the coarse output unless the caller receives it in out_c, then
+  // the block row norms and the per-query-block logit bound.
   const size_t g = (size_t)B * H * D * sizeof(float);
-  const size_t need = noalloc_align256(g * nq) * 2 + noalloc_align256(g * nkv) * 2;
+  const size_t G = (size_t)B * H;
+  const size_t need = noalloc_align256(g * nq) * 2 + noalloc_align256(g * nkv) * 2 +
+                      noalloc_align256(G * (2 * (size_t)nq + nkv) * sizeof(float));
   if (need > (size_t)VSA_NOALLOC_SCRATCH_BYTES) return VSA_ERR_WORKSPACE;  // too big for the array
 
   void* base = nullptr;
@@ -97,6 +100,10 @@ extern "C" int vsa_forward_noalloc(const void* q, const void* k, const void* v, 
   float* vc = reinterpret_cast<float*>(ws);
   ws += noalloc_align256(g * nkv);
   float* oc = out_c ? out_c : reinterpret_cast<float*>(ws);
+  ws += noalloc_align256(g * nq);
+  float* qn = reinterpret_cast<float*>(ws);
+  float* kn = qn + G * nq;
+  float* qk_bound = kn + G * nkv;
 
   PoolParams pp;
   pp.q = static_cast<const __nv_bfloat16*>(q);
@@ -110,6 +117,8 @@ extern "C" int vsa_forward_noalloc(const void* q, const void* k, const void* v, 
   pp.qc = qc;
   pp.kc = kc;
   pp.vc = vc;
+  pp.qn = qn;
+  pp.kn = kn;
   pp.status = status;
   rc = launch_pool(pp, D, st);
   if (rc != VSA_OK) return rc;
@@ -128,6 +137,10 @@ extern "C" int vsa_forward_noalloc(const void* q, const void* k, const void* v, 
   cp.q2k_idx = q2k_idx;
   cp.q2k_num = q2k_num;
   cp.out_c = oc;
+  cp.qn = qn;
+  cp.kn = kn;
+  cp.qk_bound = qk_bound;
+  cp.bound_scale = sc * 1.4426950408889634f * (1.f + 0x1p-8f);
   cp.status = status;
   rc = launch_coarse_topk(cp, D, st);
   if (rc != VSA_OK) return rc;
@@ -150,6 +163,7 @@ extern "C" int vsa_forward_noalloc(const void* q, const void* k, const void* v, 
   sp.kv_rows_per_group = Skv_pad;
   sp.gate_seq = Sq_pad;
   sp.scale_log2 = sc * 1.4426950408889634f;
+  sp.qk_bound = qk_bound;
   sp.varlen = 0;
   sp.status = status;
   return launch_sparse(sp, q, k, v, (long long)B * H * Sq_pad, (long long)B * H * Skv_pad, D,

@@ -24,11 +24,12 @@ namespace vsa {
 // a1: pooling.  One CTA of 256 threads per (tensor, batch*head, block).
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256) pool_kernel(PoolParams p) {
+__global__ void __launch_bounds__(256, 8) pool_kernel(PoolParams p) {
   constexpr int CPR = D / 8;          // 16-byte chunks per row
   constexpr int RPP = 256 / CPR;      // rows per pass
   constexpr int PASSES = 64 / RPP;
   __shared__ float red[RPP][D + 1];
+  __shared__ float wmax[8];
 
   long long item = blockIdx.x;
   const long long nq_items = (long long)p.groups * p.nq;
@@ -36,15 +37,17 @@ __global__ void __launch_bounds__(256) pool_kernel(PoolParams p) {
   const __nv_bfloat16* src;
   const int32_t* bs;
   float* dst;
+  float* nrm;        // largest row norm of the block, or null
+  bool all_rows;     // the norm covers the padding rows too (query side)
   int nblocks;
   if (item < nq_items) {
-    src = p.q; bs = p.q_bs; dst = p.qc; nblocks = p.nq;
+    src = p.q; bs = p.q_bs; dst = p.qc; nblocks = p.nq; nrm = p.qn; all_rows = true;
   } else if (item < nq_items + nkv_items) {
     item -= nq_items;
-    src = p.k; bs = p.kv_bs; dst = p.kc; nblocks = p.nkv;
+    src = p.k; bs = p.kv_bs; dst = p.kc; nblocks = p.nkv; nrm = p.kn; all_rows = false;
   } else {
     item -= nq_items + nkv_items;
-    src = p.v; bs = p.kv_bs; dst = p.vc; nblocks = p.nkv;
+    src = p.v; bs = p.kv_bs; dst = p.vc; nblocks = p.nkv; nrm = nullptr; all_rows = false;
   }
   const int blk = (int)(item % nblocks);
   int m = bs ? bs[blk] : 64;
@@ -52,6 +55,7 @@ __global__ void __launch_bounds__(256) pool_kernel(PoolParams p) {
     if (threadIdx.x == 0) set_status(p.status, VSA_ERR_BLOCK_SIZE);
     m = m < 1 ? 1 : 64;
   }
+  const int lim = (nrm && all_rows) ? 64 : m;  // rows read
   const __nv_bfloat16* base = src + item * 64 * D;  // item = group*nblocks + blk
   const int chunk = threadIdx.x % CPR;
   const int r0 = threadIdx.x / CPR;
@@ -60,24 +64,46 @@ __global__ void __launch_bounds__(256) pool_kernel(PoolParams p) {
 #pragma unroll
   for (int ps = 0; ps < PASSES; ++ps) {
     const int row = r0 + ps * RPP;
-    if (row < m) {
+    if (row < lim) {
       buf[ps] = __ldcs(reinterpret_cast<const uint4*>(base + (long long)row * D) + chunk);
     } else {
       buf[ps] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
-  float acc[8];
+  // block sums over the real rows and, per pass, this chunk's part of the
+  // row's squared norm (over every row read)
+  float acc[8], sq[PASSES];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
   for (int ps = 0; ps < PASSES; ++ps) {
     const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&buf[ps]);
+    const bool real = r0 + ps * RPP < m;
+    sq[ps] = 0.f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      float2 f = __bfloat1622float2(h2[e]);
-      acc[2 * e] += f.x;
-      acc[2 * e + 1] += f.y;
+      const float2 f = __bfloat1622float2(h2[e]);
+      sq[ps] = fmaf(f.x, f.x, sq[ps]);
+      sq[ps] = fmaf(f.y, f.y, sq[ps]);
+      if (real) {
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
     }
+  }
+  if (nrm) {
+    // a row's CPR chunks sit in CPR consecutive lanes
+    float mx = 0.f;
+#pragma unroll
+    for (int ps = 0; ps < PASSES; ++ps) {
+      float t = sq[ps];
+#pragma unroll
+      for (int o = CPR / 2; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      mx = fmaxf(mx, t);
+    }
+#pragma unroll
+    for (int o = CPR; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = mx;
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) red[r0][chunk * 8 + e] = acc[e];
@@ -87,6 +113,12 @@ __global__ void __launch_bounds__(256) pool_kernel(PoolParams p) {
 #pragma unroll
     for (int r = 0; r < RPP; ++r) s += red[r][threadIdx.x];
     dst[item * D + threadIdx.x] = __fdiv_rn(s, (float)m);
+  }
+  if (nrm && threadIdx.x == 0) {
+    float mx = wmax[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) mx = fmaxf(mx, wmax[w]);
+    nrm[item] = __fsqrt_rn(mx);
   }
 }
 
@@ -115,7 +147,8 @@ struct CoarseSmem {
   static constexpr uint32_t kCs = kQs + kQT * LD * 4;                 // [2][kCH][LD]
   static constexpr uint32_t kHist = kCs + 2 * kCH * LD * 4;           // [8 warps][256] u32
   static constexpr uint32_t kRowSum = kHist + 8 * 256 * 4;            // [kQT]
-  static constexpr uint32_t kBars = kRowSum + kQT * 4;                // [3] u64: two chunk buffers, query tile
+  static constexpr uint32_t kKnMax = kRowSum + kQT * 4;               // [8] per-warp largest key norm
+  static constexpr uint32_t kBars = kKnMax + 8 * 4;                   // [3] u64: two chunk buffers, query tile
   static constexpr uint32_t kSc = kBars + 32;                         // [kQT][sp] f32
   static_assert(kCs % 128 == 0 && (kCH * LD * 4) % 128 == 0, "TMA destinations");
   static uint32_t bytes(int sp) { return kSc + (uint32_t)kQT * sp * 4u; }
@@ -226,6 +259,14 @@ __global__ void __launch_bounds__(256, 2)
     issue_chunk(0);
     issue_chunk(1);
   }
+  if (p.qk_bound) {
+    // largest key row norm of the group (every CTA of the group takes it)
+    float km = 0.f;
+    for (int j = tid; j < p.nkv; j += 256) km = fmaxf(km, p.kn[(long long)group * p.nkv + j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, o));
+    if (lane == 0) reinterpret_cast<float*>(csm + S::kKnMax)[warp] = km;
+  }
   warp_wait(bars + 2, 0u, abort_flag, p.status);
 
   // scores = scale * qc . kc: warp w owns row 8w + tx of each chunk, a
@@ -255,6 +296,17 @@ __global__ void __launch_bounds__(256, 2)
     for (int r = 0; r < 4; ++r) sc[(ty + 4 * r) * sp + t * kCH + 8 * warp + tx] = acc[r] * p.scale;
     __syncthreads();  // buffer t & 1 is free again
     if (tid == 0 && t + 2 < 2 * nch) issue_chunk(t + 2);
+  }
+
+  // logit bound per query block of the tile (the per-warp key norms were
+  // published before the score loop's barriers)
+  if (p.qk_bound && tid < kQT && a0 + tid < p.nq) {
+    const float* kw = reinterpret_cast<const float*>(csm + S::kKnMax);
+    float km = kw[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) km = fmaxf(km, kw[w]);
+    const long long qi = (long long)group * p.nq + a0 + tid;
+    p.qk_bound[qi] = p.bound_scale * p.qn[qi] * km;
   }
 
   // per row: top-k on the scaled logits, then the softmax numerators

@@ -32,10 +32,14 @@
 //   warps 12-15  epilogue: O^T / l, the gated combine, bf16 stores
 // P^T is double-buffered in shared memory, so the softmax of pair g only
 // waits for the PV product of pair g - 2.  The running max per query column
-// is exact after an item's first pair (column reduction across lanes) and
-// refreshed only when a logit exceeds it by more than 2^8 (barrier vote),
-// then O^T and the partial sums are rescaled.  Row sums are accumulated per
-// lane and reduced across lanes once per item.
+// is exact after an item's first step (column reduction across lanes) and
+// refreshed only when a logit exceeds it by more than 2^kOffsetLimit
+// (barrier vote), then O^T and the partial sums are rescaled.  Where a
+// Cauchy-Schwarz bound on an item's logits (largest query row norm of the
+// block x largest key row norm of the head x scale) already keeps every later
+// offset within the limit, the item's later steps run a copy of the step
+// without the vote.  Row sums are accumulated per lane and reduced across
+// lanes once per item.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -71,6 +75,10 @@ constexpr int kNP = VSA_NP;            // P^T buffers in shared memory (even)
 static_assert(kNP >= 2 && kNP % 2 == 0, "two pairs per softmax step");
 constexpr uint32_t kTmemCols = 512;    // S^T buffers at 64*i (i < 4), O^T buffers at 256, 320
 constexpr uint32_t kTmemO = 256;
+// Largest offset (log2 units) of a logit above its column's running max that
+// is exponentiated without a refresh: probabilities stay below 2^32, far from
+// fp32 / bf16 overflow in P^T, O^T and the row sums.
+constexpr float kOffsetLimit = 32.f;
 
 template <int D>
 struct Layout {
@@ -255,8 +263,8 @@ __device__ __forceinline__ void store_probs(const uint32_t (&pk)[16], uint8_t* p
   }
 }
 
-// The rare step of the online softmax (a logit more than 2^8 above the
-// running maximum of its column, after an item's first step): the exact
+// The rare step of the online softmax (a logit more than kOffsetLimit above
+// the running maximum of its column, log2 units, after an item's first step): the exact
 // column maxima over this step's valid key rows, the new running maxima
 // (published in mns), the factors 2^(old - new) (in asc) and O^T rescaled by
 // them once the PV products so far are done.  Out of line so that its
@@ -598,17 +606,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item x = load_item(p, it);
       const int o = (int)(n & 1);
       const int np = (x.num + 1) / 2;
+      // bound on every logit of the item (log2 units); infinite without one
+      const float qk_bound = p.qk_bound ? p.qk_bound[x.group * p.nq + x.a] : INFINITY;
+      bool novote = false;  // set by the item's first step
       float lp[32];
 #pragma unroll
       for (int q = 0; q < 32; ++q) lp[q] = 0.f;
       // One step: two pairs (the second may be absent at the end of an
       // item), so the fixed cost of the handshakes is paid once per 4 KV
-      // tiles.  The step is compiled once for two pairs and once for one, so
-      // that the common two-pair step carries no run-time tests of the pair
-      // count.  (A third copy for two pairs of full blocks, free of the masked
-      // key-row tests, ran slower: instruction-cache pressure.)
-      auto step = [&](int i, auto two_tag) -> bool {
+      // tiles.  The step is compiled for two pairs with the overflow vote, for
+      // one pair with it, and for two pairs without it (later steps of an item
+      // whose bound rules a refresh out), so that the common step carries no
+      // run-time tests of the pair count.  (A further copy for two pairs of
+      // full blocks, free of the masked key-row tests, ran slower:
+      // instruction-cache pressure.)
+      auto step = [&](int i, auto two_tag, auto vote_tag) -> bool {
         constexpr bool two = decltype(two_tag)::value;
+        constexpr bool vote = decltype(vote_tag)::value;
         const long long g0 = gp, g1 = gp + 1;
         bool valid0, valid1 = false;
         // S^T of pair g1 is committed after that of g0 by the same thread, so
@@ -636,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           VSA_TMEM_LD16(t_lane + s1_col + 16u, x1, 16);
         }
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        if (i == 0) {
+        if (vote && i == 0) {
           // an item's first step: the running max starts as the exact column
           // max over this step's valid key rows (x0 is loaded again after)
           float fm[32];
@@ -647,8 +661,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             fm[q] = fmaxf(a, b);
           }
           col_reduce32<true>(fm, red, fin, wq, lane, t128, bar_red);
-          if (t128 < 32) mns[t128] = (fin[t128] == -INFINITY) ? 0.f : -fin[t128];
-          named_barrier_sync(bar_red, 128);
+          // later offsets are at most bound - max: if that is within the
+          // limit for every column of the group, later steps need no vote
+          bool fits = true;
+          if (t128 < 32) {
+            const float mn = (fin[t128] == -INFINITY) ? 0.f : -fin[t128];
+            mns[t128] = mn;
+            fits = qk_bound + mn <= kOffsetLimit;
+          }
+          novote = bar_red_and(bar_red, 128, fits);
           VSA_TMEM_LD16(t_lane + s0_col, x0, 0);
           VSA_TMEM_LD16(t_lane + s0_col + 16u, x0, 16);
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -666,19 +687,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             upk2(ffma2(pk2(__uint_as_float(x0[2 * j]), __uint_as_float(x0[2 * j + 1])), cc, nm), a, b);
             x0[2 * j] = __float_as_uint(a);
             x0[2 * j + 1] = __float_as_uint(b);
-            w0 = fmax3(w0, a, b);
+            if (vote) w0 = fmax3(w0, a, b);
             if (two) {
               upk2(ffma2(pk2(__uint_as_float(x1[2 * j]), __uint_as_float(x1[2 * j + 1])), cc, nm), a, b);
               x1[2 * j] = __float_as_uint(a);
               x1[2 * j + 1] = __float_as_uint(b);
-              w1 = fmax3(w1, a, b);
+              if (vote) w1 = fmax3(w1, a, b);
             }
           }
           const float worst = fmaxf(valid0 ? w0 : -INFINITY, valid1 ? w1 : -INFINITY);
-          // does any logit exceed the running max by more than 2^8?
-          if (i > 0) rescale = bar_red_or(bar_vote, 128, worst > 8.f);
+          // does any logit exceed the running max by more than the limit?
+          if (vote && i > 0) rescale = bar_red_or(bar_vote, 128, worst > kOffsetLimit);
         }
-        if (rescale) {
+        if (vote && rescale) {
           // rare step, out of line: new running maxima (shared memory), the
           // factors 2^(old - new) (asc) and O^T rescaled; the partial sums
           // and the offsets are brought up to date here
@@ -728,7 +749,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       for (int i = 0; i < np; i += 2) {
-        const bool more = (i + 1 < np) ? step(i, BoolTag<true>{}) : step(i, BoolTag<false>{});
+        bool more;
+        if (i + 1 >= np) more = step(i, BoolTag<false>{}, BoolTag<true>{});
+        else if (novote) more = step(i, BoolTag<true>{}, BoolTag<false>{});
+        else more = step(i, BoolTag<true>{}, BoolTag<true>{});
         if (!more) { ok = false; break; }
       }
       if (!ok) break;

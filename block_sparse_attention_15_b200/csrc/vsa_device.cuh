@@ -317,7 +317,18 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
-// Named barrier over `n` threads that also ORs a predicate across them.
+// Named barriers over `n` threads that also AND / OR a predicate across them.
+__device__ __forceinline__ bool bar_red_and(uint32_t id, uint32_t n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.b32 pi, %1, 0;\n\t"
+      "barrier.cta.red.and.pred po, %2, %3, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ bool bar_red_or(uint32_t id, uint32_t n, bool pred) {
   uint32_t r;
   asm volatile(

@@ -20,6 +20,8 @@ struct PoolParams {
   float* qc;             // [groups, nq, D]
   float* kc;             // [groups, nkv, D]
   float* vc;
+  float* qn;             // [groups, nq] largest row L2 norm of the block's 64 rows, or null
+  float* kn;             // [groups, nkv] largest row L2 norm of the block's real rows, or null
   int* status;
 };
 
@@ -34,6 +36,13 @@ struct CoarseParams {
   int32_t* q2k_idx;
   int32_t* q2k_num;
   float* out_c;    // [groups, nq, D]
+  // Optional logit bound (qk_bound null: none): per query block
+  // bound_scale * qn[a] * (largest kn of the group), an upper bound on
+  // scale_log2 * q.k over the block's query rows and the group's key rows.
+  const float* qn;
+  const float* kn;
+  float* qk_bound;  // [groups, nq]
+  float bound_scale;
   int* status;     // device status word (wait timeouts)
 };
 
@@ -60,6 +69,7 @@ struct SparseParams {
   long long kv_rows_per_group;
   int gate_seq;
   float scale_log2;           // softmax scale * log2(e)
+  const float* qk_bound;      // [groups, nq] bound on scale_log2 * q.k (CoarseParams), or null
   int varlen;                 // write only real rows
   int* status;
 };

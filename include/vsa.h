@@ -88,8 +88,12 @@ int vsa_get_device_status(void* stream);
  * ======================================================================== */
 
 /*
- * Workspace bytes vsa_forward needs for these sizes (pooled q/k/v and the
- * coarse output when `out_c` is not supplied, fp32).
+ * Workspace bytes vsa_forward needs for these sizes, in this order, each
+ * region starting on a 256-byte boundary: pooled q [B, H, n_q_blocks, D],
+ * pooled k and pooled v [B, H, n_kv_blocks, D], the coarse output when
+ * `out_c` is not supplied [B, H, n_q_blocks, D] (all fp32), then fp32 block
+ * row norms and a per-query-block bound on the logits, with which the sparse
+ * kernel skips its running-max check where the bound proves it unneeded.
  */
 size_t vsa_forward_workspace_size(int B, int H, int n_q_blocks, int n_kv_blocks, int D);
 
@@ -138,16 +142,16 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
  * counterpart to this entry point; it exists for such callers only.
  *
  * Same arguments, results and launches as vsa_forward, minus the workspace:
- * the scratch (pooled q/k/v and, when out_c is NULL, the coarse output, all
- * fp32) lives in one fixed array of VSA_NOALLOC_SCRATCH_BYTES that the
+ * the scratch (vsa_forward's workspace regions, in the same order) lives in
+ * one fixed array of VSA_NOALLOC_SCRATCH_BYTES that the
  * library's device image defines.  Every GPU that uses the library holds that
  * array until the process exits.  The call allocates and frees nothing.
  *
  * - Sizes whose scratch exceeds the array, i.e. when
- *     4*B*H*D*(n_q_blocks + n_kv_blocks) * 2 (each term rounded up to 256 B)
- *   is above VSA_NOALLOC_SCRATCH_BYTES, return VSA_ERR_WORKSPACE before
- *   anything is launched.  (The H3-like shape B=1, H=56, D=128, 242 + 242
- *   blocks needs 27.8 MB and fits.)
+ *   vsa_forward_workspace_size(B, H, n_q_blocks, n_kv_blocks, D) is above
+ *   VSA_NOALLOC_SCRATCH_BYTES, return VSA_ERR_WORKSPACE before anything is
+ *   launched.  (The H3-like shape B=1, H=56, D=128, 242 + 242 blocks needs
+ *   27.9 MB and fits.)
  * - The first call on each device looks the array's device address up and
  *   may load the library's device image there; make that first call before
  *   any stream capture.

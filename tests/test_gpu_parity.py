@@ -279,6 +279,45 @@ def test_forward_large_padding_rows():
     _forward_vs_oracle(q, k, v, None, qs, ks, topk=4)
 
 
+def test_forward_logit_bound_holds():
+    """The workspace's per-query-block bound is at least scale*log2(e)*q.k for
+    every query row of the block (padding rows included) and every key row of
+    the head, within 1% of the norm product, and the stored block norms equal
+    the largest row norms (padding rows count for queries, not for keys)."""
+    B, H, D = 1, 3, 128
+    qs, ks = [64, 64, 40], [64, 64, 64, 23]
+    q = _bhsd(B, H, qs, D, 2600, 0, pad_value=3.0)
+    k = _bhsd(B, H, ks, D, 2600, 1)
+    k[:, 1] *= 3
+    v = _bhsd(B, H, ks, D, 2600, 2)
+    nq, nkv = len(qs), len(ks)
+    ws = torch.zeros(vsa.lib().vsa_forward_workspace_size(B, H, nq, nkv, D), dtype=torch.uint8, device=DEV)
+    vsa.vsa_forward(q.to(DEV), k.to(DEV), v.to(DEV), None, qs, ks, topk=2, workspace=ws)
+    vsa.check_device_status()
+    a256 = lambda x: (x + 255) // 256 * 256
+    g = B * H * D * 4
+    off = a256(g * nq) * 2 + a256(g * nkv) * 2
+    G = B * H
+    norms = ws[off:off + 4 * G * (2 * nq + nkv)].view(torch.float32).cpu().numpy().astype(np.float64)
+    qn_got = norms[:G * nq].reshape(B, H, nq)
+    kn_got = norms[G * nq:G * (nq + nkv)].reshape(B, H, nkv)
+    bound = norms[G * (nq + nkv):].reshape(B, H, nq)
+    qq, kk = P.to_np(q), P.to_np(k)
+    row_q = np.linalg.norm(qq, axis=-1).reshape(B, H, nq, 64)
+    row_k = np.linalg.norm(kk, axis=-1).reshape(B, H, nkv, 64)
+    np.testing.assert_allclose(qn_got, row_q.max(-1), rtol=1e-6)
+    kmask = np.arange(64)[None, :] < np.array(ks)[:, None]
+    np.testing.assert_allclose(kn_got, np.where(kmask, row_k, 0.0).max(-1), rtol=1e-6)
+    c = O.default_scale(D) / np.log(2.0)
+    kreal = np.concatenate([np.arange(64 * j, 64 * j + n) for j, n in enumerate(ks)])
+    for b in range(B):
+        for h in range(H):
+            logits = c * qq[b, h] @ kk[b, h, kreal].T            # [Sq_pad, real keys]
+            worst = logits.reshape(nq, 64, -1).max(axis=(1, 2))
+            assert np.all(bound[b, h] >= worst), (bound[b, h], worst)
+            assert np.all(bound[b, h] <= 1.01 * c * qn_got[b, h] * kn_got[b, h].max())
+
+
 def test_forward_ungated_equals_broadcast_plus_sparse():
     """The ungated combine is out_c broadcast per block plus the sparse branch
     computed on the same selection (the combine page's ungated check)."""
