@@ -17,6 +17,9 @@ namespace vsa {
 // timer).  A healthy launch waits microseconds; this only ends a launch whose
 // producer has stopped, so the GPU stays usable and the host sees a status.
 constexpr unsigned long long kWaitTimeoutNs = 1000000000ull;  // 1 s
+// Longest sleep of one poll of an mbarrier wait (the thread wakes earlier
+// when the phase completes).
+constexpr uint32_t kPollSleepNs = 2000;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -68,6 +71,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test, but a thread whose phase is not complete yet may sleep up
+// to `hint_ns` (or until the phase completes) before it gets its answer, so
+// that a long wait polls rarely and leaves the issue slots to other warps.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false when
 // the CTA-wide abort flag is raised or the wait exceeds kWaitTimeoutNs (then
 // the status word records VSA_ERR_DEVICE_TIMEOUT and the abort flag is set).
@@ -76,7 +94,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = 0;
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, kPollSleepNs)) return true;
     if ((it & 63u) == 0u) {
       if (*abort_flag) return false;
       // another CTA already timed out: stop waiting here too, so a broken
@@ -281,6 +299,7 @@ __device__ __forceinline__ bool spin_until_at_least(volatile int* counter, int t
   if (*counter >= target) return true;
   unsigned long long t0 = 0;
   for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
     if (*counter >= target) return true;
     if ((it & 63u) == 0u) {
       if (*abort_flag) return false;
