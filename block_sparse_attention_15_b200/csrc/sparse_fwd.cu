@@ -421,9 +421,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool is_k = (warp == 0);
       const uint64_t pol_q = l2_policy_evict_first();
       const uint64_t pol_kv = l2_policy_evict_last();
-      long long gp = 0;  // pair counter over this CTA's items
+      uint32_t gp = 0;  // pair counter over this CTA's items (32 bits: power-of-two ring math)
       bool ok = true;
-      long long n = 0;
+      uint32_t n = 0;
       for (long long it = it0; ok && it < n_items; it += it_step, ++n) {
         const Item x = load_item(p, it);
         if (is_k) {
@@ -457,8 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (2 * i + 1 >= x.num) { r1 = r0; l1 = 0; }
             if (lane == 0) {
               const int N = is_k ? L::NK : L::NV;
-              const int st = (int)(gp % N);
-              const long long u = gp / N;
+              const int st = (int)(gp % (uint32_t)N);
+              const uint32_t u = gp / (uint32_t)N;
               // One TMA engine serves both producers in request order: K of
               // pair g waits until V of pair g - kKLead has been requested, so
               // K requests for far-ahead pairs never queue in front of V
@@ -501,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // drain: every stage's release (a tcgen05 commit) lands before exit
       if (ok && lane == 0) {
         const int N = is_k ? L::NK : L::NV;
-        for (long long g = (gp > N ? gp - N : 0); g < gp; ++g) {
+        for (uint32_t g = (gp > (uint32_t)N ? gp - N : 0u); g < gp; ++g) {
           if (!mbar_wait(bars + (is_k ? L::kKEmpty : L::kVEmpty) + (int)(g % N),
                          (uint32_t)((g / N) & 1), abort_flag, p.status))
             break;
@@ -512,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ===================== score products S^T = K2 . Q^T =====================
       const uint64_t desc_k = make_sdesc_sw128(sbase + L::kKOff, 16u, 1024u);
       const uint64_t desc_q = make_sdesc_sw128(sbase + L::kQOff, 16u, 1024u);
-      long long gp = 0, n = 0, n_mine = 0;
+      uint32_t gp = 0, n = 0, n_mine = 0;
       for (long long it = it0; it < n_items; it += it_step) ++n_mine;
       bool ok = true;
       for (long long it = it0; ok && it < n_items; it += it_step, ++n) {
@@ -547,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ===================== PV products O^T += V2^T . P^T =====================
       const uint64_t desc_v = make_sdesc_sw128(sbase + L::kVOff, 8192u, 1024u);
       const uint64_t desc_p = make_sdesc_sw128(sbase + L::kPOff, 8192u, 1024u);
-      long long gp = 0, n = 0;
+      uint32_t gp = 0, n = 0;
       bool ok = true;
       for (long long it = it0; ok && it < n_items; it += it_step, ++n) {
         const Item x = load_item(p, it);
@@ -593,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* fin = fin_all + col0;
     float* asc = reinterpret_cast<float*>(smem + L::kAlphaOff) + col0;
     const float c = p.scale_log2;
-    long long gp = 0, n = 0;
+    uint32_t gp = 0, n = 0;
     bool ok = true;
     // minus the running max per query column (log2 units): the same for all
     // threads of the group, so it lives in shared memory and is read as
@@ -623,12 +623,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto step = [&](int i, auto two_tag, auto vote_tag) -> bool {
         constexpr bool two = decltype(two_tag)::value;
         constexpr bool vote = decltype(vote_tag)::value;
-        const long long g0 = gp, g1 = gp + 1;
+        const uint32_t g0 = gp, g1 = gp + 1;
         bool valid0, valid1 = false;
         // S^T of pair g1 is committed after that of g0 by the same thread, so
         // its barrier covers both products (and both key-count records)
         {
-          const long long gl = two ? g1 : g0;
+          const uint32_t gl = two ? g1 : g0;
           if (!warp_wait(bars + L::kSFull + (int)(gl % kNS), (uint32_t)((gl / kNS) & 1), abort_flag, p.status)) return false;
         }
         {
@@ -703,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // rare step, out of line: new running maxima (shared memory), the
           // factors 2^(old - new) (asc) and O^T rescaled; the partial sums
           // and the offsets are brought up to date here
-          const long long gq = g0 - 1;
+          const uint32_t gq = g0 - 1;
           if (!rescale_step(t_lane + s0_col, t_lane + s1_col, two, valid0, valid1, c, red, fin, mns,
                             asc, wq, lane, t128, bar_red, bars + L::kPEmpty + (int)(gq % kNP),
                             (uint32_t)((gq / kNP) & 1), t_lane + kTmemO + 64u * o + col0, abort_flag,
@@ -734,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // g0 + 1 - kNP are done; both are committed by one thread in order, so
         // the barrier of the later one covers both
         if (g0 + 1 >= kNP) {
-          const long long gq = g0 + 1 - kNP;
+          const uint32_t gq = g0 + 1 - kNP;
           if (!warp_wait(bars + L::kPEmpty + (int)(gq % kNP), (uint32_t)((gq / kNP) & 1), abort_flag, p.status)) return false;
         }
         store_probs(pk0, smem + L::kPOff + (int)(g0 % kNP) * L::kP, Lr, grp);
@@ -766,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // drain: the last PV products' releases of the P^T buffers land before exit
     if (ok) {
-      for (long long g = (gp > kNP ? gp - kNP : 0); g < gp; ++g) {
+      for (uint32_t g = (gp > (uint32_t)kNP ? gp - kNP : 0u); g < gp; ++g) {
         if (!warp_wait(bars + L::kPEmpty + (int)(g % kNP), (uint32_t)((g / kNP) & 1), abort_flag, p.status)) break;
       }
     }
@@ -785,7 +785,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kChunks = 16 * D / 4;                             // 4-float chunks per slice
     constexpr int kPerThread = kChunks / 128;
     const int d0 = (t128 % (D / 4)) * 4;                            // fixed per thread
-    long long n = 0;
+    uint32_t n = 0;
     for (long long it = it0; it < n_items; it += it_step, ++n) {
       const Item x = load_item(p, it);
       const int o = (int)(n & 1);
