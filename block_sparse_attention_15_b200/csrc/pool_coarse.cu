@@ -8,8 +8,8 @@
 // 0.3.0", index-native q2k_idx / q2k_num) is tiny (a few GFLOP per forward);
 // it keeps a tile of pooled queries and one score row per query block in
 // shared memory, runs fp32 SIMT dot products, picks the top-k by a bitwise
-// radix select on order-preserving integer keys (ties to the lower index)
-// and writes the selection in ascending order.
+// search for the k-th largest order-preserving integer key (ties to the lower
+// index) and writes the selection in ascending order.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -145,8 +145,7 @@ struct CoarseSmem {
   static constexpr int LD = D + 4;  // row pitch in floats: 16-byte column reads hit distinct banks
   static constexpr uint32_t kQs = 0;                                  // [kQT][LD]
   static constexpr uint32_t kCs = kQs + kQT * LD * 4;                 // [2][kCH][LD]
-  static constexpr uint32_t kHist = kCs + 2 * kCH * LD * 4;           // [8 warps][256] u32
-  static constexpr uint32_t kRowSum = kHist + 8 * 256 * 4;            // [kQT]
+  static constexpr uint32_t kRowSum = kCs + 2 * kCH * LD * 4;         // [kQT]
   static constexpr uint32_t kKnMax = kRowSum + kQT * 4;               // [8] per-warp largest key norm
   static constexpr uint32_t kBars = kKnMax + 8 * 4;                   // [3] u64: two chunk buffers, query tile
   static constexpr uint32_t kSc = kBars + 32;                         // [kQT][sp] f32
@@ -154,60 +153,44 @@ struct CoarseSmem {
   static uint32_t bytes(int sp) { return kSc + (uint32_t)kQT * sp * 4u; }
 };
 
-// k-th largest key of one row by four 8-bit radix passes (most significant
-// digit first) over a per-warp histogram; returns the key T and, in
-// ties_needed, how many keys equal to T belong to the top k.
-__device__ __forceinline__ uint32_t radix_select(const uint32_t* keys, int n, uint32_t k,
-                                                 uint32_t* hist, int lane, uint32_t& ties_needed) {
-  uint32_t prefix = 0u, need = k;
-#pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
-    reinterpret_cast<uint4*>(hist)[2 * lane] = make_uint4(0u, 0u, 0u, 0u);
-    reinterpret_cast<uint4*>(hist)[2 * lane + 1] = make_uint4(0u, 0u, 0u, 0u);
-    __syncwarp();
-    for (int j = lane; j < n; j += 32) {
-      const uint32_t key = keys[j];
-      if ((key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-    }
-    __syncwarp();
-    // lane l owns digits 255-8l down to 248-8l; counts accumulate from the top
-    uint32_t cnt[8], local = 0u;
+// k-th largest key of one row (n <= 32 * KPL keys in shared memory, one
+// warp): the largest T with at least k keys >= T, built two bits at a time
+// from the most significant, the three candidates' counts taken by the whole
+// warp in independent reductions over keys held in registers; ties_needed is
+// how many keys equal to T belong to the top k.  No shared-memory atomics:
+// the scores of one row share their leading bits, which would pile a
+// histogram's increments onto a few bins.  Padding keys are 0, below every
+// finite score's key.
+template <int KPL>
+__device__ __forceinline__ uint32_t bitwise_select(const uint32_t* keys, int n, uint32_t k, int lane,
+                                                   uint32_t& ties_needed) {
+  uint32_t kr[KPL];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      cnt[t] = hist[255 - 8 * lane - t];
-      local += cnt[t];
-    }
-    uint32_t incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const uint32_t ball = __ballot_sync(0xffffffffu, incl >= need);
-    const int src = __ffs(ball) - 1;
-    uint32_t digit = 0u, above = 0u;
-    if (lane == src) {
-      uint32_t cum = incl - local;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        if (cum + cnt[t] >= need) {
-          digit = 255u - 8u * lane - t;
-          above = cum;
-          break;
-        }
-        cum += cnt[t];
-      }
-    }
-    digit = __shfl_sync(0xffffffffu, digit, src);
-    above = __shfl_sync(0xffffffffu, above, src);
-    need -= above;
-    prefix |= digit << shift;
-    __syncwarp();
+  for (int i = 0; i < KPL; ++i) {
+    const int j = lane + 32 * i;
+    kr[i] = j < n ? keys[j] : 0u;
   }
-  ties_needed = need;
-  return prefix;
+  uint32_t T = 0u;
+#pragma unroll 1
+  for (int b = 30; b >= 0; b -= 2) {
+    const uint32_t c1 = T | (1u << b), c2 = T | (2u << b), c3 = T | (3u << b);
+    uint32_t n1 = 0u, n2 = 0u, n3 = 0u;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+      n1 += kr[i] >= c1 ? 1u : 0u;
+      n2 += kr[i] >= c2 ? 1u : 0u;
+      n3 += kr[i] >= c3 ? 1u : 0u;
+    }
+    n1 = __reduce_add_sync(0xffffffffu, n1);
+    n2 = __reduce_add_sync(0xffffffffu, n2);
+    n3 = __reduce_add_sync(0xffffffffu, n3);
+    T = n3 >= k ? c3 : n2 >= k ? c2 : n1 >= k ? c1 : T;
+  }
+  uint32_t above = 0u;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) above += kr[i] > T ? 1u : 0u;
+  ties_needed = k - __reduce_add_sync(0xffffffffu, above);
+  return T;
 }
 
 // The pooled tensors are read through 3D tensor maps (D, blocks, groups) whose
@@ -310,7 +293,6 @@ __global__ void __launch_bounds__(256, 2)
   }
 
   // per row: top-k on the scaled logits, then the softmax numerators
-  uint32_t* hist = reinterpret_cast<uint32_t*>(csm + S::kHist) + warp * 256;
   const int k = p.topk;  // already clamped to [1, nkv]
   for (int r = warp; r < kQT; r += 8) {
     const int a = a0 + r;
@@ -330,7 +312,11 @@ __global__ void __launch_bounds__(256, 2)
     kmax = __reduce_max_sync(0xffffffffu, kmax);
     __syncwarp();
     uint32_t ties_needed;
-    const uint32_t T = radix_select(keys, p.nkv, (uint32_t)k, hist, lane, ties_needed);
+    uint32_t T;
+    if (p.nkv <= 256) T = bitwise_select<8>(keys, p.nkv, (uint32_t)k, lane, ties_needed);
+    else if (p.nkv <= 512) T = bitwise_select<16>(keys, p.nkv, (uint32_t)k, lane, ties_needed);
+    else if (p.nkv <= 1024) T = bitwise_select<32>(keys, p.nkv, (uint32_t)k, lane, ties_needed);
+    else T = bitwise_select<64>(keys, p.nkv, (uint32_t)k, lane, ties_needed);
     // ascending compaction: keys above T, then the lowest-index ties
     int32_t* out_idx = p.q2k_idx + ((long long)group * p.nq + a) * p.idx_stride;
     uint32_t written = 0u, ties_seen = 0u;
