@@ -147,27 +147,34 @@ class ClockSampler:
             self.proc.kill()
         self.reader.join(timeout=5)
         t0 = self.t0 if self.t0 is not None else self.t1
-        inside = [ln for t, ln in self.lines if t0 <= t <= self.t1]
-        if not inside:
-            inside = [ln for t, ln in self.lines if t > self.t1][:1]
-        sm, smax, reasons, power = [], [], set(), []
-        for line in inside:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-                power.append(float(parts[2]))
-            except ValueError:
-                continue
-            for name, val in zip(self.NAMES, parts[3:7]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "power_w_max": max(power) if power else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        return summarize_clock_lines(self.lines, t0, self.t1, self.NAMES)
+
+
+def summarize_clock_lines(lines, t0: float, t1: float, names) -> dict:
+    """Median SM clock, max clock and power, and the throttle reasons seen, over
+    the (time, csv line) samples inside [t0, t1]; for a window shorter than one
+    sampling period, the first sample after it."""
+    inside = [ln for t, ln in lines if t0 <= t <= t1]
+    if not inside:
+        inside = [ln for t, ln in lines if t > t1][:1]
+    sm, smax, reasons, power = [], [], set(), []
+    for line in inside:
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 3 + len(names):
+            continue
+        try:
+            sm.append(float(parts[0]))
+            smax.append(float(parts[1]))
+            power.append(float(parts[2]))
+        except ValueError:
+            continue
+        for name, val in zip(names, parts[3:3 + len(names)]):
+            if val.lower().startswith("active"):
+                reasons.add(name)
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(smax) if smax else None,
+            "power_w_max": max(power) if power else None,
+            "samples": len(sm), "reasons": sorted(reasons)}
 
 
 # ---------------------------------------------------------------------------
