@@ -4,7 +4,9 @@
 // combine", Problem / Notes: the compression branch runs on per-block means,
 // taken as an fp32 block sum) is a pure HBM stream: every CTA reads one
 // 64-slot block with 16-byte loads, all issued before any use, and reduces in
-// fp32.  Coarse attention plus top-k ("[chore] release fastvideo-kernel
+// fp32.  For q and k it also keeps the block's largest row norm, from which
+// the coarse kernel forms a bound on every logit of a query block (the
+// sparse kernel's vote-free step relies on it).  Coarse attention plus top-k ("[chore] release fastvideo-kernel
 // 0.3.0", index-native q2k_idx / q2k_num) is tiny (a few GFLOP per forward);
 // it keeps a tile of pooled queries and one score row per query block in
 // shared memory, runs fp32 SIMT dot products, picks the top-k by a bitwise

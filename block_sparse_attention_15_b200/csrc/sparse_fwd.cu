@@ -14,14 +14,14 @@
 //   S^T[128 kv][64 q] = K2[128 kv][D] . Q[64 q][D]^T           (K-major A, B)
 //   O^T[D][64 q]     += V2[128 kv][D]^T . P^T[128 kv][64 q]      (MN-major A, B)
 // TMEM lane = key row of S^T (softmax needs no cross-thread work per
-// element) and lane = head dim of O^T.  S^T is double-buffered in TMEM and
-// O^T too, so the epilogue of one work item overlaps the next item's loop.
+// element) and lane = head dim of O^T.  S^T has four TMEM buffers and O^T
+// two, so the epilogue of one work item overlaps the next item's loop.
 //
 // Persistent grid: one CTA per SM walks the work items (query block, head,
 // batch) b-major, h, a-minor with stride gridDim.x.  512 threads, four
 // warpgroups:
 //   warp 0       K producer: the item's Q tile and K tile pairs into a
-//                3-stage ring with each pair's key counts (TMA, 128-byte
+//                2-stage ring with each pair's key counts (TMA, 128-byte
 //                swizzle, no multicast)
 //   warp 1       TMEM owner; issues the score products S^T into four TMEM
 //                buffers, running ahead of the softmax
@@ -30,11 +30,12 @@
 //   warps 4-7    softmax for query columns 0..31
 //   warps 8-11   softmax for query columns 32..63
 //   warps 12-15  epilogue: O^T / l, the gated combine, bf16 stores
-// P^T is double-buffered in shared memory, so the softmax of pair g only
-// waits for the PV product of pair g - 2.  The running max per query column
-// is exact after an item's first step (column reduction across lanes) and
-// refreshed only when a logit exceeds it by more than 2^kOffsetLimit
-// (barrier vote), then O^T and the partial sums are rescaled.  Where a
+// The softmax takes two pairs per step; P^T is double-buffered in shared
+// memory, so a step waits for the PV products of the previous step.  The
+// running max per query column is exact after an item's first step (column
+// reduction across lanes) and refreshed only when a logit exceeds it by more
+// than kOffsetLimit (log2 units; barrier vote), then O^T and the partial sums
+// are rescaled.  Where a
 // Cauchy-Schwarz bound on an item's logits (largest query row norm of the
 // block x largest key row norm of the head x scale) already keeps every later
 // offset within the limit, the item's later steps run a copy of the step
