@@ -52,7 +52,7 @@ SIGNATURES = {
                           _c_void_p, _c_size_t, _c_void_p]),
     "block_sparse_attn_from_indices": (_c_int, [_c_void_p] * 7 + [_c_int] * 6 +
                                        [_c_float, _c_void_p, _c_void_p]),
-    "block_sparse_attn_varlen_workspace_size": (_c_size_t, [_c_int] * 3),
+    "block_sparse_attn_varlen_workspace_size": (_c_size_t, [_c_int] * 4),
     "block_sparse_attn_varlen": (_c_int, [_c_void_p] * 3 + [_P32, _P32, _P32, _P32, _P32, _P32] +
                                  [_c_int] * 3 + [_c_void_p, _c_void_p, _c_int, _c_float,
                                                  _c_void_p, _c_void_p, _c_void_p, _c_void_p,
@@ -333,7 +333,7 @@ def block_sparse_attn_varlen(q, k, v, cu_seqlens_q, cu_seqlens_kv, q2k_idx, q2k_
     if out is None:
         out = torch.zeros_like(q)
     L = lib()
-    ws_bytes = L.block_sparse_attn_varlen_workspace_size(max(n, 1), max(nqb, 1), max(nkb, 1))
+    ws_bytes = L.block_sparse_attn_varlen_workspace_size(max(n, 1), max(nqb, 1), max(nkb, 1), max(H, 1))
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     aux = None
     if return_aux:

@@ -66,7 +66,7 @@ const char* vsa_status_string(int status) {
   }
 }
 
-int vsa_abi_version(void) { return (1 << 16) | 0; }
+int vsa_abi_version(void) { return (1 << 16) | 1; }
 
 int vsa_get_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return VSA_ERR_CUDA;
@@ -241,9 +241,11 @@ int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
 // block_sparse_attn_varlen
 // ---------------------------------------------------------------------------
 size_t block_sparse_attn_varlen_workspace_size(int n_seqs, int total_q_blocks,
-                                               int total_kv_blocks) {
-  if (n_seqs <= 0 || total_q_blocks <= 0 || total_kv_blocks <= 0) return 0;
-  return align256(sizeof(int32_t) * (4 * (size_t)total_q_blocks + 2 * (size_t)total_kv_blocks));
+                                               int total_kv_blocks, int H) {
+  if (n_seqs <= 0 || total_q_blocks <= 0 || total_kv_blocks <= 0 || H <= 0) return 0;
+  // block tables, then block row norms and the per-query-block logit bound
+  return align256(sizeof(int32_t) * (4 * (size_t)total_q_blocks + 2 * (size_t)total_kv_blocks)) +
+         align256(sizeof(float) * (size_t)H * (2 * (size_t)total_q_blocks + total_kv_blocks));
 }
 
 // Resolve one side's blocks: per block first token row and size.
@@ -317,7 +319,7 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
   }
   memcpy(t_ktok, ktok.data(), sizeof(int32_t) * nkvb);
   memcpy(t_klen, klen.data(), sizeof(int32_t) * nkvb);
-  const size_t need = block_sparse_attn_varlen_workspace_size(n_seqs, nqb, nkvb);
+  const size_t need = block_sparse_attn_varlen_workspace_size(n_seqs, nqb, nkvb, H);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return VSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -345,6 +347,26 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
     return rc;
   const long long total_q = cu_seqlens_q[n_seqs], total_kv = cu_seqlens_kv[n_seqs];
   const float sc = resolve_scale(scale, D);
+  // logit bound (lets the sparse kernel skip its running-max check where it
+  // proves the check unneeded): block row norms, then per query block
+  float* qn = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                       align256(sizeof(int32_t) * table.size()));
+  VarlenBoundParams bp;
+  bp.q_tok = d_qtok;
+  bp.kv_tok = d_ktok;
+  bp.kv_len = d_klen;
+  bp.q_kv_base = d_kvbase;
+  bp.q_kv_count = d_kvcount;
+  bp.H = H;
+  bp.nqb = nqb;
+  bp.nkvb = nkvb;
+  bp.total_q = total_q;
+  bp.total_kv = total_kv;
+  bp.bound_scale = sc * 1.4426950408889634f * (1.f + 0x1p-8f);
+  bp.qn = qn;
+  bp.kn = qn + (size_t)H * nqb;
+  bp.qk_bound = bp.kn + (size_t)H * nkvb;
+  if ((rc = launch_varlen_bound(q, k, bp, D, st)) != VSA_OK) return rc;
   SparseParams sp;
   memset(&sp, 0, sizeof(sp));
   sp.out = static_cast<__nv_bfloat16*>(out);
@@ -364,6 +386,7 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
   sp.q_rows_per_group = total_q;
   sp.kv_rows_per_group = total_kv;
   sp.scale_log2 = sc * 1.4426950408889634f;
+  sp.qk_bound = bp.qk_bound;
   sp.varlen = 1;
   sp.status = status;
   return launch_sparse(sp, q, k, v, (long long)H * total_q, (long long)H * total_kv, D, false,

@@ -84,6 +84,24 @@ int launch_selftest_umma(int mode, int D, const void* a, const void* b, float* c
                          cudaStream_t stream);
 
 // varlen / metadata helpers (vsa_varlen.cu)
+// Logit bound for the varlen entry (same meaning as CoarseParams::qk_bound):
+// block row norms of the packed q and k, then per (head, query block) the
+// bound over its sequence's KV blocks.
+struct VarlenBoundParams {
+  const int32_t* q_tok;       // [nqb] first packed row of each query block
+  const int32_t* kv_tok;      // [nkvb]
+  const int32_t* kv_len;      // [nkvb] real rows
+  const int32_t* q_kv_base;   // [nqb] first KV block of the query block's sequence
+  const int32_t* q_kv_count;  // [nqb]
+  int H, nqb, nkvb;
+  long long total_q, total_kv;  // packed rows per head
+  float bound_scale;
+  float* qn;                  // [H, nqb]
+  float* kn;                  // [H, nkvb]
+  float* qk_bound;            // [H, nqb]
+};
+int launch_varlen_bound(const void* q, const void* k, const VarlenBoundParams& p, int D,
+                        cudaStream_t stream);
 int launch_varlen_aux(const int32_t* blk_tok, const int32_t* blk_len, int n_blocks,
                       int64_t* pack_index, cudaStream_t stream);
 int launch_rebase(const int32_t* q2k_idx, const int32_t* q2k_num, const int32_t* q_kv_base,

@@ -68,6 +68,102 @@ __global__ void gather_tokens_kernel(const uint4* src, uint4* dst, const int64_t
   }
 }
 
+// Largest row L2 norm of one packed block per (head, block): query blocks
+// over the 64 rows from the block's first token (the rows the sparse kernel's
+// query tile holds, clipped at the end of the tensor), key blocks over their
+// real rows.  One CTA of 256 threads per (head, block); the squared norms of
+// a row's D/8 16-byte chunks add up across consecutive lanes.
+template <int D>
+__global__ void __launch_bounds__(256, 8) varlen_norm_kernel(const __nv_bfloat16* q,
+                                                          const __nv_bfloat16* k, VarlenBoundParams p) {
+  constexpr int CPR = D / 8, RPP = 256 / CPR, PASSES = 64 / RPP;
+  __shared__ float wmax[8];
+  const long long item = blockIdx.x;  // h * (nqb + nkvb) + block
+  const int per_head = p.nqb + p.nkvb;
+  const int h = (int)(item / per_head), blk = (int)(item % per_head);
+  const bool is_q = blk < p.nqb;
+  const __nv_bfloat16* src;
+  long long row0, rows_end;
+  int rows;
+  float* dst;
+  if (is_q) {
+    src = q;
+    row0 = (long long)h * p.total_q + p.q_tok[blk];
+    rows_end = (long long)p.H * p.total_q;
+    rows = 64;
+    dst = p.qn + (long long)h * p.nqb + blk;
+  } else {
+    const int c = blk - p.nqb;
+    src = k;
+    row0 = (long long)h * p.total_kv + p.kv_tok[c];
+    rows_end = (long long)p.H * p.total_kv;
+    rows = p.kv_len[c];
+    dst = p.kn + (long long)h * p.nkvb + c;
+  }
+  const int chunk = threadIdx.x % CPR, r0 = threadIdx.x / CPR;
+  uint4 buf[PASSES];  // every load issued before any use
+#pragma unroll
+  for (int ps = 0; ps < PASSES; ++ps) {
+    const int r = r0 + ps * RPP;
+    buf[ps] = (r < rows && row0 + r < rows_end)
+                  ? __ldcs(reinterpret_cast<const uint4*>(src + (row0 + r) * D) + chunk)
+                  : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float mx = 0.f;
+#pragma unroll
+  for (int ps = 0; ps < PASSES; ++ps) {
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&buf[ps]);
+    float sq = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h2[e]);
+      sq = fmaf(f.x, f.x, sq);
+      sq = fmaf(f.y, f.y, sq);
+    }
+#pragma unroll
+    for (int o = CPR / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    mx = fmaxf(mx, sq);
+  }
+#pragma unroll
+  for (int o = CPR; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = wmax[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, wmax[w]);
+    *dst = __fsqrt_rn(m);
+  }
+}
+
+// Per (head, query block): bound_scale * its query norm * the largest key
+// norm among its sequence's KV blocks.
+__global__ void varlen_bound_kernel(VarlenBoundParams p) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)p.H * p.nqb) return;
+  const int h = (int)(i / p.nqb), a = (int)(i % p.nqb);
+  const float* kn = p.kn + (long long)h * p.nkvb + p.q_kv_base[a];
+  float km = 0.f;
+  for (int j = 0; j < p.q_kv_count[a]; ++j) km = fmaxf(km, kn[j]);
+  p.qk_bound[i] = p.bound_scale * p.qn[i] * km;
+}
+
+int launch_varlen_bound(const void* q, const void* k, const VarlenBoundParams& p, int D,
+                        cudaStream_t stream) {
+  const unsigned grid = (unsigned)((long long)p.H * (p.nqb + p.nkvb));
+  if (grid == 0) return VSA_OK;
+  if (D == 128)
+    varlen_norm_kernel<128><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q),
+                                                       static_cast<const __nv_bfloat16*>(k), p);
+  else
+    varlen_norm_kernel<64><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q),
+                                                      static_cast<const __nv_bfloat16*>(k), p);
+  if (cudaGetLastError() != cudaSuccess) return VSA_ERR_CUDA;
+  const long long n = (long long)p.H * p.nqb;
+  varlen_bound_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
 int launch_varlen_aux(const int32_t* blk_tok, const int32_t* blk_len, int n_blocks,
                       int64_t* pack_index, cudaStream_t stream) {
   const long long n = 64LL * n_blocks;

@@ -236,9 +236,12 @@ int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
  * a6: varlen block-sparse attention
  * ======================================================================== */
 
-/* Workspace bytes for block_sparse_attn_varlen (device block tables). */
+/* Workspace bytes for block_sparse_attn_varlen: the device block tables,
+ * then fp32 block row norms of q and k and a per-(head, query block) bound
+ * on the logits, with which the sparse kernel skips its running-max check
+ * where the bound proves it unneeded (H heads).  (ABI 1.1 added H.) */
 size_t block_sparse_attn_varlen_workspace_size(int n_seqs, int total_q_blocks,
-                                               int total_kv_blocks);
+                                               int total_kv_blocks, int H);
 
 /*
  * block_sparse_attn_varlen -- block-sparse attention over several sequences

@@ -138,6 +138,16 @@ def test_forward_host_workspace_size():
     assert lib.vsa_forward_host_workspace_size(B, H, 0, nkv, D, stride, 1, 0) == 0
 
 
+def test_varlen_workspace_size():
+    """Block tables (4 ints per query block, 2 per KV block), then fp32 norms
+    and bounds for H heads, each region 256-aligned."""
+    lib = _lib()
+    a = lambda x: (x + 255) // 256 * 256
+    assert lib.block_sparse_attn_varlen_workspace_size(2, 5, 3, 4) == a(4 * (20 + 6)) + a(4 * 4 * (10 + 3))
+    assert lib.block_sparse_attn_varlen_workspace_size(2, 529, 501, 24) == a(4 * (4 * 529 + 2 * 501)) + a(4 * 24 * (2 * 529 + 501))
+    assert lib.block_sparse_attn_varlen_workspace_size(2, 5, 3, 0) == 0
+
+
 def test_varlen_host_argument_checks():
     lib = _lib()
     from block_sparse_attention_15_b200.binding import _P32

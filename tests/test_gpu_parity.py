@@ -411,6 +411,22 @@ def test_varlen(case):
     P.assert_outputs_close(P.to_np(out), want)
 
 
+def test_varlen_large_logits_one_sequence_peaked():
+    """One sequence's keys scaled x16 and its queries x4: its logit bound is
+    far above the refresh limit, so its items keep the running-max check and
+    rescale, while the other sequence's items may run the vote-free step."""
+    q_lens, kv_lens, H, D = [200, 150], [300, 260], 2, 128
+    cu_q, cu_kv, q, k, v, idx, num = _varlen_inputs(q_lens, kv_lens, H, D, 0.8, 3200)
+    q[:, cu_q[1]:] *= 4
+    k[:, cu_kv[1]:] *= 16
+    out = vsa.block_sparse_attn_varlen(q.to(DEV), k.to(DEV), v.to(DEV), cu_q, cu_kv,
+                                       torch.from_numpy(idx).to(DEV), torch.from_numpy(num).to(DEV))
+    vsa.check_device_status()
+    want = O.block_sparse_attn_varlen(P.to_np(q), P.to_np(k), P.to_np(v), cu_q, cu_kv, idx, num,
+                                      O.default_scale(D))
+    P.assert_outputs_close(P.to_np(out), want, rel_rms=2e-2)
+
+
 def test_varlen_packed_equals_per_sequence_bitwise():
     """One packed launch gives exactly the per-sequence results (the varlen
     page's error = 0.0), because each query block runs the same arithmetic."""
