@@ -274,6 +274,40 @@ def weak_scaling_value(world: int, flops_per_rank: float, ms_per_step: float) ->
     return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
+def a7_timing(wl: I.Workload, dev, vsa, reps: int = 20) -> dict:
+    """a7 device token moves of the tiled workload, timed apart from the
+    forward: q's tokens into the padded tile layout (gather) and back
+    (scatter), L2 flushed before each launch.  Algorithmic bytes: gather
+    reads the tokens and writes every slot, scatter reads and writes the
+    real tokens."""
+    meta = wl.extra["meta"]
+    n_tok = int(sum(wl.q_block_sizes))
+    G = wl.B * wl.H
+    tok = I.normal_bf16((wl.B, wl.H, n_tok, wl.D), wl.seed, I.STREAM_Q).view(G, n_tok, wl.D).to(dev)
+    slot = torch.from_numpy(meta["slot_token"]).to(dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    padded = vsa.gather_tokens(tok, slot)
+    vsa.scatter_tokens(padded, slot, n_tok)
+    torch.cuda.synchronize(dev)
+    res = {}
+    for name, fn, nbytes in (
+            ("gather", lambda: vsa.gather_tokens(tok, slot), 2 * G * wl.D * (n_tok + slot.numel())),
+            ("scatter", lambda: vsa.scatter_tokens(padded, slot, n_tok), 2 * G * wl.D * 2 * n_tok)):
+        total = 0.0
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            total += e0.elapsed_time(e1)
+        ms = total / reps
+        res[name] = {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9, "bytes": nbytes}
+    vsa.check_device_status()
+    return res
+
+
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -405,6 +439,7 @@ def run_ours(args, wl):
     d2h = out_h.numel() * out_h.element_size()
     vsa.check_device_status()
 
+    a7 = a7_timing(wl, dev, vsa) if "meta" in wl.extra else None
     if rank == 0:
         peaks, peak_kind = load_peaks()
         peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -431,6 +466,8 @@ def run_ours(args, wl):
         # pooling streams q, k and v once: algorithmic bytes = their real tokens
         pool_bytes = 2 * wl.B * wl.H * wl.D * (sum(wl.q_block_sizes) + 2 * sum(wl.kv_block_sizes))
         line["pool_gbs"] = pool_bytes / (k_pool * 1e-3) / 1e9
+        if a7 is not None:
+            line["a7_tile_layout"] = a7
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, q_h, k_h, v_h, g_h, args.cpu_seconds)
         print(json.dumps(line), flush=True)

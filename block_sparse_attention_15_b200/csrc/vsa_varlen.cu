@@ -47,24 +47,28 @@ __global__ void rebase_kernel(const int32_t* q2k_idx, const int32_t* q2k_num,
   out[i] = v;
 }
 
-template <bool SCATTER>
-__global__ void gather_tokens_kernel(const uint4* src, uint4* dst, const int64_t* slot_token,
-                                     int64_t n_tokens, int64_t n_slots, int64_t groups,
-                                     int chunks) {
-  const long long total = groups * n_slots * chunks;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int ch = (int)(i % chunks);
-    const long long gs = i / chunks;
-    const long long s = gs % n_slots, g = gs / n_slots;
-    const int64_t tok = slot_token[s];
-    if (!SCATTER) {
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (tok >= 0 && tok < n_tokens) v = __ldcs(src + ((g * n_tokens + tok) * chunks + ch));
-      __stcs(dst + i, v);
-    } else if (tok >= 0 && tok < n_tokens) {
-      __stcs(dst + ((g * n_tokens + tok) * chunks + ch), __ldcs(src + i));
-    }
+// One CTA per (16 slots, group): thread t moves 16-byte chunk t % (D / 8) of
+// slot t / (D / 8); 32-bit index arithmetic only (every tensor here holds
+// fewer than 2^31 16-byte chunks per group).
+template <bool SCATTER, int D>
+__global__ void __launch_bounds__(256) gather_tokens_kernel(const uint4* src, uint4* dst,
+                                                            const int64_t* slot_token,
+                                                            int n_tokens, int n_slots) {
+  constexpr int CH = D / 8;             // 16-byte chunks per row
+  constexpr int SPB = 256 / CH;         // slots per CTA
+  const int s = blockIdx.x * SPB + (int)threadIdx.x / CH;
+  const int ch = (int)threadIdx.x % CH;
+  if (s >= n_slots) return;
+  const long long g = blockIdx.y;
+  const int64_t tok = slot_token[s];
+  const bool real = tok >= 0 && tok < n_tokens;
+  const long long slot_i = (g * n_slots + s) * CH + ch;
+  if (!SCATTER) {
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (real) v = __ldcs(src + ((g * n_tokens + tok) * CH + ch));
+    __stcs(dst + slot_i, v);
+  } else if (real) {
+    __stcs(dst + ((g * n_tokens + tok) * CH + ch), __ldcs(src + slot_i));
   }
 }
 
@@ -183,28 +187,48 @@ int launch_rebase(const int32_t* q2k_idx, const int32_t* q2k_num, const int32_t*
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
+// Any other row width (D a multiple of 8): one CTA per (slot, group), the
+// threads striding over the row's chunks.
+template <bool SCATTER>
+__global__ void __launch_bounds__(256) gather_tokens_any_kernel(const uint4* src, uint4* dst,
+                                                                const int64_t* slot_token,
+                                                                int n_tokens, int n_slots, int CH) {
+  const int s = blockIdx.x;
+  const long long g = blockIdx.y;
+  const int64_t tok = slot_token[s];
+  const bool real = tok >= 0 && tok < n_tokens;
+  for (int ch = threadIdx.x; ch < CH; ch += blockDim.x) {
+    const long long slot_i = (g * n_slots + s) * CH + ch;
+    if (!SCATTER) {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (real) v = __ldcs(src + ((g * n_tokens + tok) * CH + ch));
+      __stcs(dst + slot_i, v);
+    } else if (real) {
+      __stcs(dst + ((g * n_tokens + tok) * CH + ch), __ldcs(src + slot_i));
+    }
+  }
+}
+
 int launch_gather_tokens(const void* src, void* dst, const int64_t* slot_token, int64_t n_tokens,
                          int64_t n_slots, int64_t groups, int D, bool scatter,
                          cudaStream_t stream) {
-  const int chunks = D / 8;
-  const long long total = groups * n_slots * chunks;
-  if (total <= 0) return VSA_OK;
-  int sms = 148;
-  int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess) {
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  }
-  long long blocks = (total + 255) / 256;
-  const long long cap = (long long)sms * 8;  // 8 resident CTAs of 256 threads per SM
-  if (blocks > cap) blocks = cap;
-  if (scatter) {
-    gather_tokens_kernel<true><<<(unsigned)blocks, 256, 0, stream>>>(
-        static_cast<const uint4*>(src), static_cast<uint4*>(dst), slot_token, n_tokens, n_slots,
-        groups, chunks);
+  if (groups <= 0 || n_slots <= 0) return VSA_OK;
+  if (n_tokens > 0x7FFFFFFFLL || n_slots > 0x7FFFFFFFLL || groups > 65535) return VSA_ERR_UNSUPPORTED;
+  const int spb = D <= 2048 ? 256 / (D / 8) : 1;
+  const dim3 grid((unsigned)((n_slots + spb - 1) / spb), (unsigned)groups);
+  const uint4* s4 = static_cast<const uint4*>(src);
+  uint4* d4 = static_cast<uint4*>(dst);
+  const int nt = (int)n_tokens, ns = (int)n_slots;
+  if (D == 128) {
+    if (scatter) gather_tokens_kernel<true, 128><<<grid, 256, 0, stream>>>(s4, d4, slot_token, nt, ns);
+    else gather_tokens_kernel<false, 128><<<grid, 256, 0, stream>>>(s4, d4, slot_token, nt, ns);
+  } else if (D == 64) {
+    if (scatter) gather_tokens_kernel<true, 64><<<grid, 256, 0, stream>>>(s4, d4, slot_token, nt, ns);
+    else gather_tokens_kernel<false, 64><<<grid, 256, 0, stream>>>(s4, d4, slot_token, nt, ns);
   } else {
-    gather_tokens_kernel<false><<<(unsigned)blocks, 256, 0, stream>>>(
-        static_cast<const uint4*>(src), static_cast<uint4*>(dst), slot_token, n_tokens, n_slots,
-        groups, chunks);
+    const dim3 g1((unsigned)n_slots, (unsigned)groups);
+    if (scatter) gather_tokens_any_kernel<true><<<g1, 256, 0, stream>>>(s4, d4, slot_token, nt, ns, D / 8);
+    else gather_tokens_any_kernel<false><<<g1, 256, 0, stream>>>(s4, d4, slot_token, nt, ns, D / 8);
   }
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
