@@ -26,9 +26,10 @@
  * - `scale` <= 0 selects 1/sqrt(D).
  * - Pointers documented "device" must point to memory of the current CUDA
  *   device; "host" pointers to ordinary host memory.  The caller owns every
- *   buffer; the library allocates and frees nothing.  Scratch comes from the
- *   caller's `workspace` (size from the matching *_workspace_size call,
- *   256-byte aligned).
+ *   buffer; the library allocates and frees no memory.  Scratch comes from
+ *   the caller's `workspace` (size from the matching *_workspace_size call,
+ *   256-byte aligned).  (vsa_forward_host creates two copy streams per
+ *   device on first use, kept for the process, and a few events per call.)
  * - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *   asynchronous on that stream and never synchronise it, except
  *   vsa_get_device_status.
