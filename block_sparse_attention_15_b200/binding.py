@@ -213,12 +213,12 @@ def vsa_forward_host(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=None
     nq, nkv = Sq // 64, Skv // 64
     k_eff = min(int(topk), nkv)
     stride = k_eff if idx_stride is None else int(idx_stride)
-    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     qbs = None if q_block_sizes is None else torch.tensor(list(q_block_sizes), dtype=torch.int32)
     kbs = None if kv_block_sizes is None else torch.tensor(list(kv_block_sizes), dtype=torch.int32)
     for bs, n, name in ((qbs, nq, "q_block_sizes"), (kbs, nkv, "kv_block_sizes")):
         if bs is not None and bs.numel() != n:
             raise ValueError(f"expected {n} {name}, got {bs.numel()}")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     if out is None:
         out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
     elif out.is_cuda or out.dtype != torch.bfloat16 or out.shape != q.shape or not out.is_contiguous():

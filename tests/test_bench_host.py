@@ -51,3 +51,23 @@ def test_varlen_random_selection():
             row += 1
     idx2, num2, _ = I.varlen_random_selection(q_lens, kv_lens, 3, 0.5, 7)
     assert np.array_equal(idx, idx2) and np.array_equal(num, num2)
+
+
+def test_forward_host_binding_rejects_bad_tensors():
+    """The host-buffer binding checks dtypes, devices and shapes before it
+    touches the GPU."""
+    import pytest
+    import torch
+
+    from block_sparse_attention_15_b200 import binding as vsa
+
+    q = torch.zeros((1, 2, 128, 64), dtype=torch.bfloat16)
+    k = torch.zeros((1, 2, 192, 64), dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        vsa.vsa_forward_host(q.float(), k, k, topk=1)
+    with pytest.raises(ValueError):
+        vsa.vsa_forward_host(q, k, k[:, :, :128], topk=1)               # v shape != k shape
+    with pytest.raises(ValueError):
+        vsa.vsa_forward_host(q, k, k, torch.zeros((1, 128, 3, 64), dtype=torch.bfloat16), topk=1)
+    with pytest.raises(ValueError):
+        vsa.vsa_forward_host(q, k, k, topk=1, q_block_sizes=[64])     # 2 query blocks
