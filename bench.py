@@ -77,22 +77,27 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def profiled_traffic():
-    """DRAM bytes per launch of the block-sparse kernel from the committed ncu
-    summary, if the kernel sources still hash to what was profiled."""
-    path = os.path.join(ROOT, "profiles", "sparse_fwd_h3.md")
-    if not os.path.exists(path):
-        return None
-    text = open(path).read()
-    m_t = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
-    m_h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
-    if not (m_t and m_h):
-        return None
+def sparse_source_hash() -> str:
     h = hashlib.sha256()
     for rel in SPARSE_SOURCES:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
-    return int(m_t.group(1)) if h.hexdigest() == m_h.group(1) else None
+    return h.hexdigest()
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the block-sparse kernel on the default workload,
+    from the committed record of an ncu capture (a JSON data file beside the
+    capture's summary), if the kernel sources still hash to what was
+    profiled; else None."""
+    path = os.path.join(ROOT, "profiles", "sparse_fwd_h3_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("kernel_source_sha256") != sparse_source_hash():
+        return None
+    return int(rec["traffic_bytes_per_launch"])
 
 
 # ---------------------------------------------------------------------------
@@ -112,6 +117,7 @@ class ClockSampler:
         self.proc = None
         self.lines = []          # (monotonic time, line)
         self.t0 = self.t1 = None
+        self.nvml = NvmlSampler(device_index)
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
             ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
@@ -137,8 +143,12 @@ class ClockSampler:
 
     def stop(self) -> dict:
         self.t1 = time.monotonic()
+        fast = self.nvml.stop(self.t0 if self.t0 is not None else self.t1, self.t1)
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            res = {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            if fast:
+                res["nvml_5ms"] = fast
+            return res
         time.sleep(0.12)
         self.proc.terminate()
         try:
@@ -147,7 +157,58 @@ class ClockSampler:
             self.proc.kill()
         self.reader.join(timeout=5)
         t0 = self.t0 if self.t0 is not None else self.t1
-        return summarize_clock_lines(self.lines, t0, self.t1, self.NAMES)
+        res = summarize_clock_lines(self.lines, t0, self.t1, self.NAMES)
+        if fast:
+            res["nvml_5ms"] = fast
+        return res
+
+
+class NvmlSampler:
+    """SM clock and throttle reasons read through NVML every 5 ms on a thread
+    (read-only queries), so that a timed region of a few tens of ms still
+    holds several samples; None where NVML is unavailable."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, device_index: int):
+        self.samples = []   # (monotonic time, sm MHz, reason bits)
+        self.stop_flag = False
+        self.thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(ident)
+            self.nv = pynvml
+        except Exception:  # noqa: BLE001 - best effort
+            self.handle = None
+            return
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag:
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((time.monotonic(), float(mhz), int(bits)))
+            except Exception:  # noqa: BLE001
+                return
+            time.sleep(0.005)
+
+    def stop(self, t0: float, t1: float):
+        if self.thread is None:
+            return None
+        self.stop_flag = True
+        self.thread.join(timeout=2)
+        inside = [(m, b) for t, m, b in self.samples if t0 <= t <= t1]
+        if not inside:
+            return None
+        reasons = sorted(n for n, bit in self.REASONS.items() if any(b & bit for _, b in inside))
+        return {"sm_mhz": statistics.median(m for m, _ in inside), "samples": len(inside),
+                "min_mhz": min(m for m, _ in inside), "reasons": reasons}
 
 
 def summarize_clock_lines(lines, t0: float, t1: float, names) -> dict:
@@ -258,6 +319,23 @@ def config_of(wl: I.Workload, flushed: bool) -> dict:
 # ---------------------------------------------------------------------------
 # the two arms
 # ---------------------------------------------------------------------------
+def clock_normalised(ms_per_step: float, ms_sparse: float, clocks: dict) -> dict | None:
+    """Time x median SM clock over the timed region, and the times that
+    product gives at the maximum clock: a run that the power cap slowed
+    (sustained behaviour) and one at full clock (burst) then compare like for
+    like."""
+    fast = clocks.get("nvml_5ms") or {}
+    mhz = fast.get("sm_mhz") or clocks.get("sm_mhz")
+    mx = clocks.get("sm_max_mhz")
+    if not mhz:
+        return None
+    res = {"sm_mhz_median": mhz, "ms_x_mhz": ms_per_step * mhz, "sparse_ms_x_mhz": ms_sparse * mhz}
+    if mx:
+        res["ms_per_step_at_max_clock"] = ms_per_step * mhz / mx
+        res["sparse_ms_at_max_clock"] = ms_sparse * mhz / mx
+    return res
+
+
 def max_over_ranks(values, world: int, device):
     """Element-wise maximum of per-rank timings (every rank gets the result;
     the slowest rank sets the job's time)."""
@@ -463,6 +541,7 @@ def run_ours(args, wl):
             "gpu_launches": 3 * K,
             "clocks": clocks,
         }
+        line["clock_normalised"] = clock_normalised(ms_per_step, k_sparse, clocks)
         # pooling streams q, k and v once: algorithmic bytes = their real tokens
         pool_bytes = 2 * wl.B * wl.H * wl.D * (sum(wl.q_block_sizes) + 2 * sum(wl.kv_block_sizes))
         line["pool_gbs"] = pool_bytes / (k_pool * 1e-3) / 1e9

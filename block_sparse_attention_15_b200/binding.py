@@ -63,6 +63,7 @@ SIGNATURES = {
     "vsa_scatter_tokens": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int64, _c_int64,
                                     _c_int64, _c_int, _c_void_p]),
     "vsa_selftest_umma": (_c_int, [_c_int, _c_int, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "vsa_selftest_exp2": (_c_int, [_c_void_p, _c_void_p, _c_int64, _c_void_p, _c_void_p]),
     "vsa_set_profile_events": (_c_int, [ctypes.POINTER(_c_void_p)]),
 }
 
@@ -406,6 +407,17 @@ def selftest_umma(mode: int, a, b, *, stream=None):
     _check("vsa_selftest_umma", lib().vsa_selftest_umma(mode, D, _ptr(a), _ptr(b), _ptr(c),
                                                         _stream(stream)))
     return c
+
+
+def selftest_exp2(x, *, stream=None):
+    """The sparse kernel's FMA-pipe 2^x on a device fp32 tensor; returns
+    (y, number of elements whose packed halves disagree)."""
+    _require(x, torch.float32, "x")
+    y = torch.empty_like(x)
+    mism = torch.zeros(1, dtype=torch.int32, device=x.device)
+    _check("vsa_selftest_exp2", lib().vsa_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _ptr(mism),
+                                                        _stream(stream)))
+    return y, int(mism.item())
 
 
 def set_profile_events(events):

@@ -5,6 +5,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
 #include <vector>
 
 #include "vsa.h"
@@ -15,10 +16,16 @@ namespace vsa {
 // Device status word: kernels record the first error of a launch sequence.
 __device__ int g_device_status = 0;
 
+// The address is looked up once per device and cached (under a lock, so
+// concurrent first calls from several host threads are safe).  The cache
+// assumes the device's context lives as long as the process: a
+// cudaDeviceReset between calls is not supported.
 int* device_status_ptr() {
+  static std::mutex mu;
   static int* cached[64] = {nullptr};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (!cached[dev]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_device_status) != cudaSuccess) return nullptr;
@@ -37,12 +44,124 @@ static inline bool aligned16(const void* p) {
 static cudaEvent_t g_prof_events[4] = {nullptr, nullptr, nullptr, nullptr};
 static bool g_prof_on = false;
 
-static inline void prof_record(int i, cudaStream_t st) {
-  if (g_prof_on) cudaEventRecord(g_prof_events[i], st);
+float resolve_scale(float scale, int D) {
+  return scale > 0.f ? scale : 1.0f / sqrtf((float)D);
 }
 
-static inline float resolve_scale(float scale, int D) {
-  return scale > 0.f ? scale : 1.0f / sqrtf((float)D);
+
+int check_forward_args(const ForwardArgs& a) {
+  if (!a.q || !a.k || !a.v || !a.out || !a.q2k_idx || !a.q2k_num) return VSA_ERR_INVALID_ARG;
+  if (a.B <= 0 || a.H <= 0 || a.Sq_pad <= 0 || a.Skv_pad <= 0 || a.topk < 1 || !(a.scale == a.scale))
+    return VSA_ERR_INVALID_ARG;
+  if (a.D != 64 && a.D != 128) return VSA_ERR_UNSUPPORTED;
+  if (a.Sq_pad % 64 || a.Skv_pad % 64) return VSA_ERR_SHAPE;
+  const int nq = a.Sq_pad / 64, nkv = a.Skv_pad / 64;
+  if (nq > VSA_MAX_BLOCKS || nkv > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
+  const int k_eff = a.topk < nkv ? a.topk : nkv;
+  if (a.idx_stride < k_eff) return VSA_ERR_SHAPE;
+  if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.out) ||
+      (a.gate && !aligned16(a.gate)) || (a.out_c && !aligned16(a.out_c)))
+    return VSA_ERR_INVALID_ARG;
+  return VSA_OK;
+}
+
+// The three launches of the forward on checked arguments, with the scratch
+// regions carved from `scratch` (vsa_forward_workspace_size bytes, 256-byte
+// aligned) in the documented order.  Every region is written in full by the
+// kernel that produces it before any kernel reads it.
+int launch_forward(const ForwardArgs& a, void* scratch, bool profile, cudaStream_t st) {
+  const int B = a.B, H = a.H, D = a.D;
+  const int nq = a.Sq_pad / 64, nkv = a.Skv_pad / 64;
+  const int k_eff = a.topk < nkv ? a.topk : nkv;
+  int* status = device_status_ptr();
+  if (!status) return VSA_ERR_CUDA;
+  const bool prof = profile && g_prof_on;
+
+  const size_t g = (size_t)B * H * D * sizeof(float);
+  char* ws = static_cast<char*>(scratch);
+  float* qc = reinterpret_cast<float*>(ws);
+  ws += align256(g * nq);
+  float* kc = reinterpret_cast<float*>(ws);
+  ws += align256(g * nkv);
+  float* vc = reinterpret_cast<float*>(ws);
+  ws += align256(g * nkv);
+  float* oc = a.out_c ? a.out_c : reinterpret_cast<float*>(ws);
+  ws += align256(g * nq);
+  // block row norms and the per-query-block logit bound
+  const size_t G = (size_t)B * H;
+  float* qn = reinterpret_cast<float*>(ws);
+  float* kn = qn + G * nq;
+  float* qk_bound = kn + G * nkv;
+
+  PoolParams pp;
+  pp.q = static_cast<const __nv_bfloat16*>(a.q);
+  pp.k = static_cast<const __nv_bfloat16*>(a.k);
+  pp.v = static_cast<const __nv_bfloat16*>(a.v);
+  pp.q_bs = a.q_block_sizes;
+  pp.kv_bs = a.kv_block_sizes;
+  pp.groups = B * H;
+  pp.nq = nq;
+  pp.nkv = nkv;
+  pp.qc = qc;
+  pp.kc = kc;
+  pp.vc = vc;
+  pp.qn = qn;
+  pp.kn = kn;
+  pp.status = status;
+  if (prof) cudaEventRecord(g_prof_events[0], st);
+  int rc = launch_pool(pp, D, st);
+  if (rc != VSA_OK) return rc;
+  if (prof) cudaEventRecord(g_prof_events[1], st);
+
+  const float sc = resolve_scale(a.scale, D);
+  CoarseParams cp;
+  cp.qc = qc;
+  cp.kc = kc;
+  cp.vc = vc;
+  cp.groups = B * H;
+  cp.nq = nq;
+  cp.nkv = nkv;
+  cp.scale = sc;
+  cp.topk = k_eff;
+  cp.idx_stride = a.idx_stride;
+  cp.q2k_idx = a.q2k_idx;
+  cp.q2k_num = a.q2k_num;
+  cp.out_c = oc;
+  cp.qn = qn;
+  cp.kn = kn;
+  cp.qk_bound = qk_bound;
+  cp.bound_scale = sc * kLog2e * (1.f + 0x1p-8f);
+  cp.status = status;
+  rc = launch_coarse_topk(cp, D, st);
+  if (rc != VSA_OK) return rc;
+  if (prof) cudaEventRecord(g_prof_events[2], st);
+
+  SparseParams sp;
+  memset(&sp, 0, sizeof(sp));
+  sp.out = static_cast<__nv_bfloat16*>(a.out);
+  sp.gate = static_cast<const __nv_bfloat16*>(a.gate);
+  sp.out_c = oc;
+  sp.q2k_idx = a.q2k_idx;
+  sp.q2k_num = a.q2k_num;
+  sp.idx_stride = a.idx_stride;
+  sp.q_bs = a.q_block_sizes;
+  sp.kv_bs = a.kv_block_sizes;
+  sp.B = B;
+  sp.H = H;
+  sp.nq = nq;
+  sp.nkv = nkv;
+  sp.q_rows_per_group = a.Sq_pad;
+  sp.kv_rows_per_group = a.Skv_pad;
+  sp.gate_seq = a.Sq_pad;
+  sp.scale_log2 = sc * kLog2e;
+  sp.qk_bound = qk_bound;
+  sp.varlen = 0;
+  sp.status = status;
+  rc = launch_sparse(sp, a.q, a.k, a.v, (long long)B * H * a.Sq_pad, (long long)B * H * a.Skv_pad,
+                     D, /*combine=*/true, /*gated=*/a.gate != nullptr, st);
+  if (rc != VSA_OK) return rc;
+  if (prof) cudaEventRecord(g_prof_events[3], st);
+  return VSA_OK;
 }
 
 }  // namespace vsa
@@ -92,110 +211,18 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
                 int Sq_pad, int Skv_pad, int D, int topk, float scale, void* out,
                 int32_t* q2k_idx, int32_t* q2k_num, int idx_stride, float* out_c,
                 void* workspace, size_t workspace_bytes, void* stream) {
-  if (!q || !k || !v || !out || !q2k_idx || !q2k_num) return VSA_ERR_INVALID_ARG;
-  if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || topk < 1 || !(scale == scale))
-    return VSA_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
-  if (Sq_pad % 64 || Skv_pad % 64) return VSA_ERR_SHAPE;
-  const int nq = Sq_pad / 64, nkv = Skv_pad / 64;
-  if (nq > VSA_MAX_BLOCKS || nkv > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
-  const int k_eff = topk < nkv ? topk : nkv;
-  if (idx_stride < k_eff) return VSA_ERR_SHAPE;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-      (gate && !aligned16(gate)) || (out_c && !aligned16(out_c)))
-    return VSA_ERR_INVALID_ARG;
-  const size_t need = vsa_forward_workspace_size(B, H, nq, nkv, D);
+  ForwardArgs a;
+  a.q = q; a.k = k; a.v = v; a.gate = gate;
+  a.q_block_sizes = q_block_sizes; a.kv_block_sizes = kv_block_sizes;
+  a.B = B; a.H = H; a.Sq_pad = Sq_pad; a.Skv_pad = Skv_pad; a.D = D; a.topk = topk;
+  a.scale = scale; a.out = out; a.q2k_idx = q2k_idx; a.q2k_num = q2k_num;
+  a.idx_stride = idx_stride; a.out_c = out_c;
+  int rc = check_forward_args(a);
+  if (rc != VSA_OK) return rc;
+  const size_t need = vsa_forward_workspace_size(B, H, Sq_pad / 64, Skv_pad / 64, D);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return VSA_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int* status = device_status_ptr();
-  if (!status) return VSA_ERR_CUDA;
-
-  const size_t g = (size_t)B * H * D * sizeof(float);
-  char* ws = static_cast<char*>(workspace);
-  float* qc = reinterpret_cast<float*>(ws);
-  ws += align256(g * nq);
-  float* kc = reinterpret_cast<float*>(ws);
-  ws += align256(g * nkv);
-  float* vc = reinterpret_cast<float*>(ws);
-  ws += align256(g * nkv);
-  float* oc = out_c ? out_c : reinterpret_cast<float*>(ws);
-  ws += align256(g * nq);
-  // block row norms and the per-query-block logit bound
-  const size_t G = (size_t)B * H;
-  float* qn = reinterpret_cast<float*>(ws);
-  float* kn = qn + G * nq;
-  float* qk_bound = kn + G * nkv;
-
-  PoolParams pp;
-  pp.q = static_cast<const __nv_bfloat16*>(q);
-  pp.k = static_cast<const __nv_bfloat16*>(k);
-  pp.v = static_cast<const __nv_bfloat16*>(v);
-  pp.q_bs = q_block_sizes;
-  pp.kv_bs = kv_block_sizes;
-  pp.groups = B * H;
-  pp.nq = nq;
-  pp.nkv = nkv;
-  pp.qc = qc;
-  pp.kc = kc;
-  pp.vc = vc;
-  pp.qn = qn;
-  pp.kn = kn;
-  pp.status = status;
-  prof_record(0, st);
-  int rc = launch_pool(pp, D, st);
-  if (rc != VSA_OK) return rc;
-  prof_record(1, st);
-
-  const float sc = resolve_scale(scale, D);
-  CoarseParams cp;
-  cp.qc = qc;
-  cp.kc = kc;
-  cp.vc = vc;
-  cp.groups = B * H;
-  cp.nq = nq;
-  cp.nkv = nkv;
-  cp.scale = sc;
-  cp.topk = k_eff;
-  cp.idx_stride = idx_stride;
-  cp.q2k_idx = q2k_idx;
-  cp.q2k_num = q2k_num;
-  cp.out_c = oc;
-  cp.qn = qn;
-  cp.kn = kn;
-  cp.qk_bound = qk_bound;
-  cp.bound_scale = sc * 1.4426950408889634f * (1.f + 0x1p-8f);
-  cp.status = status;
-  rc = launch_coarse_topk(cp, D, st);
-  if (rc != VSA_OK) return rc;
-  prof_record(2, st);
-
-  SparseParams sp;
-  memset(&sp, 0, sizeof(sp));
-  sp.out = static_cast<__nv_bfloat16*>(out);
-  sp.gate = static_cast<const __nv_bfloat16*>(gate);
-  sp.out_c = oc;
-  sp.q2k_idx = q2k_idx;
-  sp.q2k_num = q2k_num;
-  sp.idx_stride = idx_stride;
-  sp.q_bs = q_block_sizes;
-  sp.kv_bs = kv_block_sizes;
-  sp.B = B;
-  sp.H = H;
-  sp.nq = nq;
-  sp.nkv = nkv;
-  sp.q_rows_per_group = Sq_pad;
-  sp.kv_rows_per_group = Skv_pad;
-  sp.gate_seq = Sq_pad;
-  sp.scale_log2 = sc * 1.4426950408889634f;
-  sp.qk_bound = qk_bound;
-  sp.varlen = 0;
-  sp.status = status;
-  rc = launch_sparse(sp, q, k, v, (long long)B * H * Sq_pad, (long long)B * H * Skv_pad, D,
-                     /*combine=*/true, /*gated=*/gate != nullptr, st);
-  if (rc != VSA_OK) return rc;
-  prof_record(3, st);
-  return VSA_OK;
+  return launch_forward(a, workspace, /*profile=*/true, static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------
@@ -231,7 +258,7 @@ int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
   sp.nkv = nkv;
   sp.q_rows_per_group = Sq_pad;
   sp.kv_rows_per_group = Skv_pad;
-  sp.scale_log2 = sc * 1.4426950408889634f;
+  sp.scale_log2 = sc * kLog2e;
   sp.status = status;
   return launch_sparse(sp, q, k, v, (long long)B * H * Sq_pad, (long long)B * H * Skv_pad, D,
                        false, false, static_cast<cudaStream_t>(stream));
@@ -362,7 +389,7 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
   bp.nkvb = nkvb;
   bp.total_q = total_q;
   bp.total_kv = total_kv;
-  bp.bound_scale = sc * 1.4426950408889634f * (1.f + 0x1p-8f);
+  bp.bound_scale = sc * kLog2e * (1.f + 0x1p-8f);
   bp.qn = qn;
   bp.kn = qn + (size_t)H * nqb;
   bp.qk_bound = bp.kn + (size_t)H * nkvb;
@@ -385,7 +412,7 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
   sp.nkv = nkvb;
   sp.q_rows_per_group = total_q;
   sp.kv_rows_per_group = total_kv;
-  sp.scale_log2 = sc * 1.4426950408889634f;
+  sp.scale_log2 = sc * kLog2e;
   sp.qk_bound = bp.qk_bound;
   sp.varlen = 1;
   sp.status = status;
@@ -471,6 +498,12 @@ int vsa_set_profile_events(void* const* events) {
   for (int i = 0; i < 4; ++i) g_prof_events[i] = static_cast<cudaEvent_t>(events[i]);
   g_prof_on = true;
   return VSA_OK;
+}
+
+int vsa_selftest_exp2(const float* x, float* y, int64_t n, int* mismatch, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y || !mismatch))) return VSA_ERR_INVALID_ARG;
+  if (n > (int64_t)1 << 40) return VSA_ERR_UNSUPPORTED;
+  return launch_selftest_exp2(x, y, (long long)n, mismatch, static_cast<cudaStream_t>(stream));
 }
 
 int vsa_selftest_umma(int mode, int D, const void* a, const void* b, float* c, void* stream) {

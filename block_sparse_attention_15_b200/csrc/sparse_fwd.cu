@@ -194,9 +194,13 @@ __device__ __forceinline__ float red_op(float a, float b) {
 // softmax group; the 32 results land in fin[0..31] (shared memory, visible to
 // the group on return).  Warp stage: recursive halving with shuffles, after
 // which lane l holds column l; then the four warps combine through `red`.
+// The first barrier also ORs the warps' abort flags: if any warp of the group
+// gave up a wait, every warp returns true there (and nothing is reduced), so
+// the group leaves its loop together instead of leaving a warp behind at a
+// barrier that the others never reach.
 template <bool IsMax>
-__device__ __forceinline__ void col_reduce32(const float (&v)[32], float* red, float* fin, int wq,
-                                             int lane, int t128, uint32_t bar_id) {
+__device__ __forceinline__ bool col_reduce32(const float (&v)[32], float* red, float* fin, int wq,
+                                             int lane, int t128, uint32_t bar_id, bool aborted) {
   float a[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
@@ -225,12 +229,13 @@ __device__ __forceinline__ void col_reduce32(const float (&v)[32], float* red, f
   const bool hi = lane & 1;
   const float e = red_op<IsMax>(hi ? d[1] : d[0], __shfl_xor_sync(0xffffffffu, hi ? d[0] : d[1], 1));
   red[wq * 32 + lane] = e;
-  named_barrier_sync(bar_id, 128);
+  if (bar_red_or(bar_id, 128, aborted)) return true;
   if (t128 < 32) {
     fin[t128] = red_op<IsMax>(red_op<IsMax>(red[t128], red[32 + t128]),
                               red_op<IsMax>(red[64 + t128], red[96 + t128]));
   }
   named_barrier_sync(bar_id, 128);
+  return false;
 }
 
 // Probabilities of one key row for 32 query columns: p = 2^x (0 for a
@@ -269,12 +274,15 @@ __device__ __forceinline__ void store_probs(const uint32_t (&pk)[16], uint8_t* p
 // column maxima over this step's valid key rows, the new running maxima
 // (published in mns), the factors 2^(old - new) (in asc) and O^T rescaled by
 // them once the PV products so far are done.  Out of line so that its
-// registers do not weigh on the common path.  False if a wait gave up.
+// registers do not weigh on the common path.  Returns false when the group
+// agreed to abort (some warp had given up a wait); a wait given up here sets
+// `aborted`, which the group's next barrier reports.
 __device__ __noinline__ bool rescale_step(uint32_t t_s0, uint32_t t_s1, bool two, bool valid0,
                                           bool valid1, float c, float* red, float* fin,
                                           float* mns, float* asc, int wq, int lane, int t128,
                                           uint32_t bar_red, uint64_t* pempty, uint32_t pparity,
-                                          uint32_t t_o, volatile int* abort_flag, int* status) {
+                                          uint32_t t_o, bool& aborted, volatile int* abort_flag,
+                                          int* status) {
   {
     uint32_t x[32];
     float masked[32];
@@ -286,7 +294,7 @@ __device__ __noinline__ bool rescale_step(uint32_t t_s0, uint32_t t_s1, bool two
 #pragma unroll
       for (int q = 0; q < 32; ++q) masked[q] = fmaxf(masked[q], valid1 ? __uint_as_float(x[q]) * c : -INFINITY);
     }
-    col_reduce32<true>(masked, red, fin, wq, lane, t128, bar_red);
+    if (col_reduce32<true>(masked, red, fin, wq, lane, t128, bar_red, aborted)) return false;
   }
   if (t128 < 32) {
     const float old = -mns[t128];
@@ -295,7 +303,7 @@ __device__ __noinline__ bool rescale_step(uint32_t t_s0, uint32_t t_s1, bool two
     mns[t128] = -nm;
   }
   named_barrier_sync(bar_red, 128);
-  if (!warp_wait(pempty, pparity, abort_flag, status)) return false;
+  if (!aborted && !warp_wait(pempty, pparity, abort_flag, status)) aborted = true;
   tc_fence_after_sync();
   uint32_t ov[32];
   tmem_ld32(t_o, ov);
@@ -596,6 +604,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.scale_log2;
     uint32_t gp = 0, n = 0;
     bool ok = true;
+    // A wait that gives up only sets `aborted` (this warp then skips its later
+    // waits); the group's next barrier ORs the flag, and there every warp of
+    // the group leaves the loop together (see col_reduce32).
+    bool aborted = false;
+    auto wwait = [&](uint64_t* bar, uint32_t parity) {
+      if (!aborted && !warp_wait(bar, parity, abort_flag, p.status)) aborted = true;
+    };
     // minus the running max per query column (log2 units): the same for all
     // threads of the group, so it lives in shared memory and is read as
     // broadcast 16-byte loads (it changes only at a rescale)
@@ -630,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // its barrier covers both products (and both key-count records)
         {
           const uint32_t gl = two ? g1 : g0;
-          if (!warp_wait(bars + L::kSFull + (int)(gl % kNS), (uint32_t)((gl / kNS) & 1), abort_flag, p.status)) return false;
+          wwait(bars + L::kSFull + (int)(gl % kNS), (uint32_t)((gl / kNS) & 1));
         }
         {
           const int2 l0 = smeta[g0 % kNS];
@@ -661,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float b = valid1 ? __uint_as_float(x1[q]) * c : -INFINITY;
             fm[q] = fmaxf(a, b);
           }
-          col_reduce32<true>(fm, red, fin, wq, lane, t128, bar_red);
+          if (col_reduce32<true>(fm, red, fin, wq, lane, t128, bar_red, aborted)) return false;
           // later offsets are at most bound - max: if that is within the
           // limit for every column of the group, later steps need no vote
           bool fits = true;
@@ -698,7 +713,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float worst = fmaxf(valid0 ? w0 : -INFINITY, valid1 ? w1 : -INFINITY);
           // does any logit exceed the running max by more than the limit?
-          if (vote && i > 0) rescale = bar_red_or(bar_vote, 128, worst > kOffsetLimit);
+          if (vote && i > 0 && bar_red_or(bar_vote, 128, aborted || worst > kOffsetLimit)) {
+            // rare: a refresh, or some warp of the group gave up a wait
+            if (bar_red_or(bar_vote, 128, aborted)) return false;
+            rescale = true;
+          }
         }
         if (vote && rescale) {
           // rare step, out of line: new running maxima (shared memory), the
@@ -707,8 +726,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t gq = g0 - 1;
           if (!rescale_step(t_lane + s0_col, t_lane + s1_col, two, valid0, valid1, c, red, fin, mns,
                             asc, wq, lane, t128, bar_red, bars + L::kPEmpty + (int)(gq % kNP),
-                            (uint32_t)((gq / kNP) & 1), t_lane + kTmemO + 64u * o + col0, abort_flag,
-                            p.status)) return false;
+                            (uint32_t)((gq / kNP) & 1), t_lane + kTmemO + 64u * o + col0, aborted,
+                            abort_flag, p.status)) return false;
 #pragma unroll
           for (int q = 0; q < 32; ++q) lp[q] *= asc[q];
           tmem_ld32(t_lane + s0_col, x0);
@@ -736,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the barrier of the later one covers both
         if (g0 + 1 >= kNP) {
           const uint32_t gq = g0 + 1 - kNP;
-          if (!warp_wait(bars + L::kPEmpty + (int)(gq % kNP), (uint32_t)((gq / kNP) & 1), abort_flag, p.status)) return false;
+          wwait(bars + L::kPEmpty + (int)(gq % kNP), (uint32_t)((gq / kNP) & 1));
         }
         store_probs(pk0, smem + L::kPOff + (int)(g0 % kNP) * L::kP, Lr, grp);
         if (two) store_probs(pk1, smem + L::kPOff + (int)(g1 % kNP) * L::kP, Lr, grp);
@@ -758,15 +777,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // end of item: 1 / row sums for the epilogue
-      if (n >= 2 && !warp_wait(bars + L::kOEmpty + o, (uint32_t)(((n - 2) >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
-      col_reduce32<false>(lp, red, fin, wq, lane, t128, bar_red);
+      if (n >= 2) wwait(bars + L::kOEmpty + o, (uint32_t)(((n - 2) >> 1) & 1));
+      if (col_reduce32<false>(lp, red, fin, wq, lane, t128, bar_red, aborted)) { ok = false; break; }
       if (t128 < 32) inv_l[o * 64 + col0 + t128] = fin[t128] > 0.f ? 1.f / fin[t128] : 0.f;
       named_barrier_sync(bar_red, 128);
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + L::kLFull + o);
     }
     // drain: the last PV products' releases of the P^T buffers land before exit
-    if (ok) {
+    if (ok && !aborted) {
       for (uint32_t g = (gp > (uint32_t)kNP ? gp - kNP : 0u); g < gp; ++g) {
         if (!warp_wait(bars + L::kPEmpty + (int)(g % kNP), (uint32_t)((g / kNP) & 1), abort_flag, p.status)) break;
       }
@@ -790,8 +809,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (long long it = it0; it < n_items; it += it_step, ++n) {
       const Item x = load_item(p, it);
       const int o = (int)(n & 1);
-      if (!warp_wait(bars + L::kOFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status)) break;
-      if (!warp_wait(bars + L::kLFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status)) break;
+      // the four warps agree before their first named barrier of the item,
+      // so a warp that gave up a wait never leaves the others at one
+      bool bad = !warp_wait(bars + L::kOFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status);
+      if (!bad) bad = !warp_wait(bars + L::kLFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status);
+      if (bar_red_or(5, 128, bad)) break;
       float4 oc = make_float4(0.f, 0.f, 0.f, 0.f);
       if (COMBINE) oc = *reinterpret_cast<const float4*>(p.out_c + (x.group * p.nq + x.a) * (long long)D + d0);
       const long long orow0 = x.group * p.q_rows_per_group + x.q_tok;
@@ -935,6 +957,17 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// Self-test of the FMA-pipe exponential: y[i] = exp2_fma2(x[i]) (the lower
+// half of the pair; the upper half gets x[i] too and must agree).
+__global__ void selftest_exp2_kernel(const float* x, float* y, long long n, int* mismatch) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float lo, hi;
+  upk2(exp2_fma2(x[i], x[i]), lo, hi);
+  y[i] = lo;
+  if (__float_as_uint(lo) != __float_as_uint(hi)) atomicAdd(mismatch, 1);
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -1019,6 +1052,13 @@ int launch_sparse(const SparseParams& p, const void* q, const void* k, const voi
   if (!combine) return launch_sparse_t<64, false, false>(p, mq, mk, mv, stream);
   if (gated) return launch_sparse_t<64, true, true>(p, mq, mk, mv, stream);
   return launch_sparse_t<64, true, false>(p, mq, mk, mv, stream);
+}
+
+int launch_selftest_exp2(const float* x, float* y, long long n, int* mismatch,
+                         cudaStream_t stream) {
+  if (n <= 0) return VSA_OK;
+  selftest_exp2_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(x, y, n, mismatch);
+  return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
 int launch_selftest_umma(int mode, int D, const void* a, const void* b, float* c,

@@ -404,17 +404,19 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // 2^x for a pair of floats on the FMA pipe, so that part of the
 // exponentials leaves the MUFU unit (which does 16 per cycle per SM) alone.
 // Range reduction x = j + f with j = round(x) (added to the exponent field)
-// and f in [-1/2, 1/2]; 2^f by a cubic fitted by weighted least squares to
-// the relative error on that interval (max relative error 7.5e-5, far below
-// the bf16 rounding of the probabilities).  x is clamped to >= -120, where
-// the result (< 2^-120) is negligible next to the row maximum's 1.
+// and f in [-1/2, 1/2]; 2^f by the cubic that minimises the largest relative
+// error on that interval (Remez exchange; block_sparse_attention_15_b200/
+// exp2_fit.py computes these float32 coefficients and models these steps:
+// max relative error 7.49e-5 over [-120, 32], far below the bf16 rounding of
+// the probabilities).  x is clamped to >= -120, where the result (2^-120) is
+// negligible next to the row maximum's 1.
 __device__ __forceinline__ uint64_t exp2_fma2(float x0, float x1) {
   constexpr float kRound = 12582912.f;  // 1.5 * 2^23: adding it rounds to an integer
   const uint64_t xx = pk2(fmaxf(x0, -120.f), fmaxf(x1, -120.f));
   const uint64_t t = fadd2(xx, pk2(kRound, kRound));
   const uint64_t j = fadd2(t, pk2(-kRound, -kRound));
   const uint64_t f = ffma2(j, pk2(-1.f, -1.f), xx);
-  uint64_t q = ffma2(f, pk2(0x1.c3f75ep-5f, 0x1.c3f75ep-5f), pk2(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
+  uint64_t q = ffma2(f, pk2(0x1.c3f760p-5f, 0x1.c3f760p-5f), pk2(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
   q = ffma2(q, f, pk2(0x1.62f31ap-1f, 0x1.62f31ap-1f));
   q = ffma2(q, f, pk2(0x1.fff692p-1f, 0x1.fff692p-1f));
   float q0, q1, t0, t1;

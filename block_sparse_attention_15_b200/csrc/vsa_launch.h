@@ -82,6 +82,8 @@ int launch_sparse(const SparseParams& p, const void* q, const void* k, const voi
                   bool gated, cudaStream_t stream);
 int launch_selftest_umma(int mode, int D, const void* a, const void* b, float* c,
                          cudaStream_t stream);
+int launch_selftest_exp2(const float* x, float* y, long long n, int* mismatch,
+                         cudaStream_t stream);
 
 // varlen / metadata helpers (vsa_varlen.cu)
 // Logit bound for the varlen entry (same meaning as CoarseParams::qk_bound):
@@ -121,5 +123,34 @@ EncodeTiledFn get_encode_fn();
 
 // Device status word of the current device (address via cudaGetSymbolAddress).
 int* device_status_ptr();
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Softmax scale: the given one, or 1/sqrt(D) when it is <= 0.
+float resolve_scale(float scale, int D);
+
+// Arguments of the whole forward (vsa_forward and vsa_forward_noalloc share
+// the checks and the launch sequence; only the source of the scratch differs).
+struct ForwardArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* gate;
+  const int32_t* q_block_sizes;
+  const int32_t* kv_block_sizes;
+  int B, H, Sq_pad, Skv_pad, D, topk;
+  float scale;
+  void* out;
+  int32_t* q2k_idx;
+  int32_t* q2k_num;
+  int idx_stride;
+  float* out_c;
+};
+// Host checks of vsa_forward's arguments (everything but the workspace).
+int check_forward_args(const ForwardArgs& a);
+// Pool, coarse + top-k and the sparse kernel with the fused combine, on
+// `stream`, with scratch of vsa_forward_workspace_size bytes at `scratch`.
+// `profile`: record the profiling events when the hook is set.
+int launch_forward(const ForwardArgs& a, void* scratch, bool profile, cudaStream_t stream);
 
 }  // namespace vsa

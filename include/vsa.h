@@ -32,7 +32,10 @@
  *   device on first use, kept for the process, and a few events per call.)
  * - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *   asynchronous on that stream and never synchronise it, except
- *   vsa_get_device_status.
+ *   vsa_get_device_status, and except that block_sparse_attn_varlen (its
+ *   block tables) and vsa_forward_host (the block sizes) copy a small table
+ *   from pageable host memory with cudaMemcpyAsync, which the CUDA runtime
+ *   may serialise with the stream.
  * - Every call returns a vsa status code.  Argument problems detectable on
  *   the host are returned before anything is launched.  Problems found inside
  *   kernels (an out-of-range index, a bad block size, a barrier wait that ran
@@ -367,6 +370,15 @@ int vsa_set_profile_events(void* const* events);
  * transposed-output product.  a, b device bf16; c device fp32.  D 64 or 128.
  */
 int vsa_selftest_umma(int mode, int D, const void* a, const void* b, float* c, void* stream);
+
+/*
+ * vsa_selftest_exp2 -- evaluate the sparse kernel's FMA-pipe exponential
+ * (2^x by range reduction and a fitted cubic; the pages fix no such routine,
+ * it is an implementation detail of the softmax) on x[0 .. n): y[i] is its
+ * value, and *mismatch (device int32, added to) counts elements where the two
+ * halves of the packed evaluation disagree.  x, y device fp32 [n].
+ */
+int vsa_selftest_exp2(const float* x, float* y, int64_t n, int* mismatch, void* stream);
 
 #ifdef __cplusplus
 }

@@ -20,7 +20,7 @@ Sources (FastVideo pages):
              (PR #1408)
   [readme]   fastvideo-kernel README
 
-Readings where the pages leave a step open (each also listed in the design doc):
+Readings where the pages leave a step open:
   R1  the coarse softmax uses the same scale as the fine one, 1/sqrt(D);
   R2  top-k ranks the scaled coarse logits; equal logits go to the lower KV
       block index;

@@ -1,7 +1,10 @@
 """GPU parity at the workloads' full sizes, in the launch configuration the
-benchmark times.  Indices are checked in full; outputs on sampled query
-blocks that the oracle computes one by one (the full fp64 oracle would take
-minutes)."""
+benchmark times.  Indices are checked in full.  Outputs are checked against
+the fp64 oracle on every query block of every head for the H3-like, the
+video-tiled and the varlen workloads (the oracle needs about half a minute
+for the largest), and on every head x 32 query blocks for the long
+(32768-token) workloads, whose dense case alone would take the oracle many
+minutes in full."""
 import numpy as np
 import pytest
 import torch
@@ -15,18 +18,32 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _sample_items(rng, B, H, nq, n):
-    items = {(0, 0, 0), (B - 1, H - 1, nq - 1)}
-    while len(items) < n:
-        items.add((int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(nq))))
-    return sorted(items)
+def _all_items(B, H, nq):
+    return [(b, h, a) for b in range(B) for h in range(H) for a in range(nq)]
+
+
+def _per_head_items(rng, B, H, nq, per_head):
+    """per_head distinct query blocks of every (batch, head), the first and
+    last block always among them."""
+    items = []
+    for b in range(B):
+        for h in range(H):
+            blocks = {0, nq - 1}
+            blocks.update(int(a) for a in rng.choice(nq, size=min(nq, per_head) - 2, replace=False))
+            while len(blocks) < min(nq, per_head):
+                blocks.add(int(rng.integers(nq)))
+            items += [(b, h, a) for a in sorted(blocks)]
+    return items
 
 
 def _rows_of(items, q_sizes):
     return [(b, h, np.arange(64 * a, 64 * a + q_sizes[a])) for b, h, a in items]
 
 
-def _run_forward_case(wl: I.Workload, q, k, v, gate, n_items, seed):
+def _run_forward_case(wl: I.Workload, q, k, v, gate, seed, per_head=None):
+    """Forward on the GPU; stage by stage against the oracle.  Outputs are
+    compared on every query block (per_head None) or on per_head blocks of
+    every head."""
     out, idx, num, out_c = vsa.vsa_forward(
         q.to(DEV), k.to(DEV), v.to(DEV), None if gate is None else gate.to(DEV),
         None if all(s == 64 for s in wl.q_block_sizes) else wl.q_block_sizes,
@@ -42,7 +59,8 @@ def _run_forward_case(wl: I.Workload, q, k, v, gate, n_items, seed):
     idx_np, num_np = P.to_np(idx), P.to_np(num)
     P.check_topk(idx_np, num_np, scores, wl.topk)
     rng = np.random.default_rng(seed)
-    items = _sample_items(rng, wl.B, wl.H, wl.nq, n_items)
+    items = (_all_items(wl.B, wl.H, wl.nq) if per_head is None
+             else _per_head_items(rng, wl.B, wl.H, wl.nq, per_head))
     o_s = O.block_sparse_attention(qn, kn, vn, idx_np, num_np, wl.q_block_sizes,
                                    wl.kv_block_sizes, scale, items=items)
     want = O.combine(oc, o_s, None if gate is None else P.to_np(gate), wl.q_block_sizes)
@@ -72,7 +90,7 @@ def test_h3_like_full():
     """B1 H56 D128 S15488 (242 blocks), top-48, gated: the benchmark's shape."""
     wl = I.workload_h3()
     q, k, v, gate = _inputs(wl)
-    _run_forward_case(wl, q, k, v, gate, n_items=24, seed=1)
+    _run_forward_case(wl, q, k, v, gate, seed=1)
 
 
 def test_video_tiled_full():
@@ -88,7 +106,7 @@ def test_video_tiled_full():
     q, k, v = (vsa.gather_tokens(t.reshape(wl.H, N, wl.D).to(DEV), slot).reshape(1, wl.H, -1, wl.D).cpu()
                for t in toks)
     gate = I.gate_bf16((1, 64 * wl.nq, wl.H, wl.D), wl.seed)
-    got, _, _ = _run_forward_case(wl, q, k, v, gate, n_items=24, seed=2)
+    got, _, _ = _run_forward_case(wl, q, k, v, gate, seed=2)
     # back to token order
     back = vsa.scatter_tokens(torch.from_numpy(got).to(torch.bfloat16).reshape(wl.H, -1, wl.D).to(DEV),
                               slot, N)
@@ -101,7 +119,7 @@ def test_long_sequence(frac, gated):
     """B1 H40 D128 S32768 (512 blocks) at top 5% / 10% / 100%."""
     wl = I.workload_long(frac, gated)
     q, k, v, gate = _inputs(wl)
-    got, idx, num = _run_forward_case(wl, q, k, v, gate, n_items=12, seed=3)
+    got, idx, num = _run_forward_case(wl, q, k, v, gate, seed=3, per_head=32)
     if frac == 1.0:
         # dense: every block selected, so the sparse branch is full attention;
         # brute force on sampled rows (fp64, all 32768 keys)
@@ -138,7 +156,6 @@ def test_varlen_full():
     nq = [-(-n // 64) for n in q_lens]
     idx, num, ks = I.varlen_random_selection(q_lens, kv_lens, H, 0.15, seed)
     assert ks == [7, 16, 21, 30]
-    rng = np.random.default_rng(seed + 1)
     out, pq, pkv, reb = vsa.block_sparse_attn_varlen(
         q.to(DEV), k.to(DEV), v.to(DEV), cu_q, cu_kv, torch.from_numpy(idx).to(DEV),
         torch.from_numpy(num).to(DEV), return_aux=True)
@@ -153,7 +170,7 @@ def test_varlen_full():
     qp = O.pack_tokens(P.to_np(q), lay["pack_index_q"])
     kp = O.pack_tokens(P.to_np(k), lay["pack_index_kv"])
     vp = O.pack_tokens(P.to_np(v), lay["pack_index_kv"])
-    items = _sample_items(rng, 1, H, sum(nq), 24)
+    items = _all_items(1, H, sum(nq))
     o = O.block_sparse_attention(qp, kp, vp, reb_want[None], num[None], lay["q_block_sizes"],
                                  lay["kv_block_sizes"], O.default_scale(D), items=items)
     got = P.to_np(out)
