@@ -658,6 +658,68 @@ def run_varlen(args):
     return 0
 
 
+def run_entry(args, wl):
+    """Other entry points on the same workload, one call per step, the whole
+    call timed: ``indices`` = block_sparse_attn_from_indices (with its
+    logit-bound pass) on the selection the forward makes; ``bshd`` = the
+    whole forward on BSHD tensors (video_sparse_attn_bshd)."""
+    from block_sparse_attention_15_b200 import binding as vsa
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--entry other than forward runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    q_h, k_h, v_h, g_h = host_inputs(wl)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    gate = None if g_h is None else g_h.to(dev)
+    qbs = None if all(s == 64 for s in wl.q_block_sizes) else wl.q_block_sizes
+    kbs = None if all(s == 64 for s in wl.kv_block_sizes) else wl.kv_block_sizes
+    out, idx, num = vsa.vsa_forward(q, k, v, gate, qbs, kbs, topk=wl.topk)
+    if args.entry == "indices":
+        def step():
+            vsa.block_sparse_attn_from_indices(q, k, v, idx, num, qbs, kbs, out=out)
+        what = "block_sparse_attn_from_indices with its logit-bound pass, on the forward's selection"
+        launches = 3
+    else:
+        qb, kb, vb = (x.transpose(1, 2).contiguous() for x in (q, k, v))
+        del q, k, v
+        out_b = torch.empty_like(qb)
+
+        def step():
+            vsa.video_sparse_attn_bshd(qb, kb, vb, gate, qbs, kbs, topk=wl.topk, out=out_b)
+        what = "whole forward on BSHD q/k/v/out (video_sparse_attn_bshd)"
+        launches = 3
+    sampler = ClockSampler(local)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    vsa.check_device_status()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    vsa.check_device_status()
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tflops = wl.flops / (ms * 1e-3) / 1e12
+    line = {"metric": METRIC + f" [{args.entry} entry]", "value": tflops, "unit": "TFLOP/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": {**config_of(wl, False), "entry": what},
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tflops / peak, "traffic": None, "kernel": f"whole call: {what}",
+                         "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS)"},
+            "gpu_launches": launches * args.steps, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -670,6 +732,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-items", type=int, default=24,
                     help="query blocks per reference-arm step (bounded CPU sample)")
+    ap.add_argument("--entry", choices=["forward", "indices", "bshd"], default="forward",
+                    help="entry point timed on the workload (forward: the headline line)")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (smaller cases for profiler captures)")
     args = ap.parse_args(argv)
@@ -685,6 +749,8 @@ def main(argv=None):
         wl.name += f" [H overridden to {args.heads}]"
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.entry != "forward":
+        return run_entry(args, wl)
     return run_ours(args, wl)
 
 

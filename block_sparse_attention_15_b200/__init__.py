@@ -7,6 +7,7 @@ package is its Python binding plus the seeded input generator
 """
 from .binding import (  # noqa: F401
     VSAError,
+    block_sparse_attn,
     block_sparse_attn_from_indices,
     block_sparse_attn_varlen,
     build_vsa_metadata,
@@ -17,10 +18,11 @@ from .binding import (  # noqa: F401
     scatter_tokens,
     vsa_forward,
     vsa_forward_host,
+    video_sparse_attn_bshd,
 )
 
 __all__ = [
-    "VSAError", "block_sparse_attn_from_indices", "block_sparse_attn_varlen", "build_vsa_metadata",
+    "VSAError", "block_sparse_attn", "block_sparse_attn_from_indices", "block_sparse_attn_varlen", "build_vsa_metadata",
     "check_device_status", "gather_tokens", "get_device_status", "lib", "scatter_tokens",
-    "vsa_forward", "vsa_forward_host",
+    "vsa_forward", "vsa_forward_host", "video_sparse_attn_bshd",
 ]

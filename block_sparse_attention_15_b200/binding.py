@@ -34,6 +34,21 @@ _c_float = ctypes.c_float
 _P32 = ctypes.POINTER(ctypes.c_int32)
 _P64 = ctypes.POINTER(ctypes.c_int64)
 
+
+class VsaStrides(ctypes.Structure):
+    """vsa_strides: element strides over (batch, head, sequence slot)."""
+    _fields_ = [("batch", ctypes.c_int64), ("head", ctypes.c_int64), ("seq", ctypes.c_int64)]
+
+
+class VsaLayout(ctypes.Structure):
+    """vsa_layout: the strides of q, k, v, out and the gate of one call."""
+    _fields_ = [("q", VsaStrides), ("k", VsaStrides), ("v", VsaStrides), ("out", VsaStrides),
+                ("gate", VsaStrides)]
+
+
+_PL = ctypes.POINTER(VsaLayout)
+VSA_LAYOUT_BHSD, VSA_LAYOUT_BSHD = 0, 1
+
 # name -> (restype, argtypes); mirrors include/vsa.h
 SIGNATURES = {
     "vsa_status_string": (ctypes.c_char_p, [_c_int]),
@@ -43,6 +58,13 @@ SIGNATURES = {
     "vsa_forward": (_c_int, [_c_void_p] * 4 + [_c_void_p, _c_void_p] + [_c_int] * 6 +
                     [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p,
                      _c_size_t, _c_void_p]),
+    "vsa_make_layout": (_c_int, [_c_int] * 6 + [_PL]),
+    "vsa_forward_strided": (_c_int, [_c_void_p] * 4 + [_PL, _c_void_p, _c_void_p] + [_c_int] * 6 +
+                            [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p,
+                             _c_void_p, _c_size_t, _c_void_p]),
+    "vsa_forward_bshd": (_c_int, [_c_void_p] * 4 + [_c_void_p, _c_void_p] + [_c_int] * 6 +
+                         [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p,
+                          _c_size_t, _c_void_p]),
     "vsa_forward_noalloc": (_c_int, [_c_void_p] * 4 + [_c_void_p, _c_void_p] + [_c_int] * 6 +
                             [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p,
                              _c_void_p]),
@@ -50,8 +72,13 @@ SIGNATURES = {
     "vsa_forward_host": (_c_int, [_c_void_p] * 4 + [_c_void_p, _c_void_p] + [_c_int] * 6 +
                          [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_int,
                           _c_void_p, _c_size_t, _c_void_p]),
+    "block_sparse_attn_from_indices_workspace_size": (_c_size_t, [_c_int] * 4),
     "block_sparse_attn_from_indices": (_c_int, [_c_void_p] * 7 + [_c_int] * 6 +
-                                       [_c_float, _c_void_p, _c_void_p]),
+                                       [_c_float, _c_void_p, _PL, _c_void_p, _c_size_t,
+                                        _c_void_p]),
+    "block_sparse_attn": (_c_int, [_c_void_p] * 6 + [_c_int] * 5 +
+                          [_c_float, _c_void_p, _c_void_p, _c_void_p, _PL, _c_void_p, _c_size_t,
+                           _c_void_p]),
     "block_sparse_attn_varlen_workspace_size": (_c_size_t, [_c_int] * 4),
     "block_sparse_attn_varlen": (_c_int, [_c_void_p] * 3 + [_P32, _P32, _P32, _P32, _P32, _P32] +
                                  [_c_int] * 3 + [_c_void_p, _c_void_p, _c_int, _c_float,
@@ -116,6 +143,38 @@ def _require(t, dtype, name, device=True):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _require_view(t, name):
+    """A bf16 CUDA tensor whose last (head-dim) axis is contiguous and whose
+    other strides are multiples of 8 elements (any layout: BHSD, BSHD, a
+    slice of a fused tensor, a transposed view)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be torch.bfloat16, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError(f"{name} must be a 4-D view with a contiguous last axis")
+    for ax in range(3):
+        if t.shape[ax] > 1 and (t.stride(ax) <= 0 or t.stride(ax) % 8):
+            raise ValueError(f"{name}: stride {t.stride(ax)} of axis {ax} is not a positive "
+                             "multiple of 8 elements")
+    if t.data_ptr() % 16:
+        raise ValueError(f"{name} must start on a 16-byte boundary")
+
+
+def _strides_bhsd(t):
+    """vsa_strides of a [B, H, S, D] view."""
+    return VsaStrides(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _layout(q, k, v, out, gate_bshd=None):
+    """vsa_layout of [B, H, S, D] views q, k, v, out and a [B, S, H, D] gate."""
+    g = (VsaStrides(gate_bshd.stride(0), gate_bshd.stride(2), gate_bshd.stride(1))
+         if gate_bshd is not None else VsaStrides(0, 0, 0))
+    return VsaLayout(_strides_bhsd(q), _strides_bhsd(k), _strides_bhsd(v), _strides_bhsd(out), g)
+
+
 def _block_sizes_tensor(bs, n, device):
     if bs is None:
         return None
@@ -142,20 +201,23 @@ def vsa_forward(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=None, *, 
                 scale: float | None = None, idx_stride: int | None = None, out=None,
                 return_out_c: bool = False, return_pooled: bool = False, workspace=None,
                 stream=None):
-    """Full VSA forward through ``vsa_forward`` (see include/vsa.h).
+    """Full VSA forward through ``vsa_forward_strided`` (see include/vsa.h).
 
     q: [B, H, Sq_pad, D] bf16; k, v: [B, H, Skv_pad, D]; gate: [B, Sq_pad, H, D]
-    or None.  Returns ``(out, q2k_idx, q2k_num)`` plus ``out_c`` and the pooled
-    (qc, kc, vc) when asked.
+    or None.  Any of them may be a strided view (head dim contiguous, other
+    strides multiples of 8): a BSHD tensor transposed to [B, H, S, D], a
+    slice of a fused QKV tensor.  ``out`` (allocated like q if None) may be a
+    view too.  Returns ``(out, q2k_idx, q2k_num)`` plus ``out_c`` and the
+    pooled (qc, kc, vc) when asked.
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _require(t, torch.bfloat16, n)
+        _require_view(t, n)
     B, H, Sq, D = q.shape
     Skv = k.shape[2]
     if k.shape != (B, H, Skv, D) or v.shape != k.shape:
         raise ValueError("k and v must be [B, H, Skv_pad, D] matching q")
     if gate is not None:
-        _require(gate, torch.bfloat16, "gate")
+        _require_view(gate, "gate")
         if gate.shape != (B, Sq, H, D):
             raise ValueError(f"gate must be [B, Sq_pad, H, D] = {(B, Sq, H, D)}, got {tuple(gate.shape)}")
     nq, nkv = Sq // 64, Skv // 64
@@ -166,6 +228,9 @@ def vsa_forward(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=None, *, 
     kbs = _block_sizes_tensor(kv_block_sizes, nkv, dev)
     if out is None:
         out = torch.empty_like(q)
+    _require_view(out, "out")
+    if out.shape != q.shape:
+        raise ValueError("out must be shaped like q")
     q2k_idx = torch.empty((B, H, nq, stride), dtype=torch.int32, device=dev)
     q2k_num = torch.empty((B, H, nq), dtype=torch.int32, device=dev)
     out_c = torch.empty((B, H, nq, D), dtype=torch.float32, device=dev) if return_out_c else None
@@ -173,10 +238,11 @@ def vsa_forward(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=None, *, 
     ws_bytes = L.vsa_forward_workspace_size(B, H, nq, nkv, D)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
-    _check("vsa_forward", L.vsa_forward(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(qbs), _ptr(kbs), B, H, Sq, Skv, D, int(topk),
-        float(scale) if scale is not None else 0.0, _ptr(out), _ptr(q2k_idx), _ptr(q2k_num), stride,
-        _ptr(out_c), _ptr(workspace), workspace.numel(), _stream(stream)))
+    lay = _layout(q, k, v, out, gate)
+    _check("vsa_forward_strided", L.vsa_forward_strided(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gate), ctypes.byref(lay), _ptr(qbs), _ptr(kbs), B, H, Sq,
+        Skv, D, int(topk), float(scale) if scale is not None else 0.0, _ptr(out), _ptr(q2k_idx),
+        _ptr(q2k_num), stride, _ptr(out_c), _ptr(workspace), workspace.numel(), _stream(stream)))
     res = [out, q2k_idx, q2k_num]
     if return_out_c:
         res.append(out_c)
@@ -261,29 +327,96 @@ def pooled_views(workspace, B, H, nq, nkv, D):
     return tuple(views)
 
 
-def block_sparse_attn_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes=None,
-                                   kv_block_sizes=None, *, scale: float | None = None, out=None,
-                                   stream=None):
-    """Block-sparse attention over the listed tiles (``block_sparse_attn_from_indices``)."""
+def _sparse_common(q, k, v, out):
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _require(t, torch.bfloat16, n)
-    _require(q2k_idx, torch.int32, "q2k_idx")
-    _require(q2k_num, torch.int32, "q2k_num")
+        _require_view(t, n)
     B, H, Sq, D = q.shape
     Skv = k.shape[2]
+    if k.shape != (B, H, Skv, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H, Skv_pad, D] matching q")
+    if out is None:
+        out = torch.empty_like(q)
+    _require_view(out, "out")
+    if out.shape != q.shape:
+        raise ValueError("out must be shaped like q")
+    return B, H, Sq, Skv, D, out
+
+
+def block_sparse_attn_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes=None,
+                                   kv_block_sizes=None, *, scale: float | None = None, out=None,
+                                   logit_bound: bool = True, stream=None):
+    """Block-sparse attention over the listed tiles (``block_sparse_attn_from_indices``).
+
+    q, k, v, out: [B, H, S, D] views (see :func:`vsa_forward`).  With
+    ``logit_bound`` (default) a workspace is passed, so the library bounds
+    each query block's logits first and the kernel skips its running-max
+    check where the bound allows (same results)."""
+    B, H, Sq, Skv, D, out = _sparse_common(q, k, v, out)
+    _require(q2k_idx, torch.int32, "q2k_idx")
+    _require(q2k_num, torch.int32, "q2k_num")
     nq, nkv = Sq // 64, Skv // 64
     if q2k_idx.dim() != 4 or q2k_idx.shape[:3] != (B, H, nq) or q2k_num.shape != (B, H, nq):
         raise ValueError("q2k_idx must be [B, H, n_q_blocks, stride], q2k_num [B, H, n_q_blocks]")
     dev = q.device
     qbs = _block_sizes_tensor(q_block_sizes, nq, dev)
     kbs = _block_sizes_tensor(kv_block_sizes, nkv, dev)
-    if out is None:
-        out = torch.empty_like(q)
-    _check("block_sparse_attn_from_indices", lib().block_sparse_attn_from_indices(
+    L = lib()
+    ws = None
+    if logit_bound:
+        ws = torch.empty(max(L.block_sparse_attn_from_indices_workspace_size(B, H, nq, nkv), 256),
+                         dtype=torch.uint8, device=dev)
+    lay = _layout(q, k, v, out)
+    _check("block_sparse_attn_from_indices", L.block_sparse_attn_from_indices(
         _ptr(q), _ptr(k), _ptr(v), _ptr(q2k_idx), _ptr(q2k_num), _ptr(qbs), _ptr(kbs), B, H, Sq,
         Skv, D, q2k_idx.shape[3], float(scale) if scale is not None else 0.0, _ptr(out),
-        _stream(stream)))
+        ctypes.byref(lay), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
     return out
+
+
+def block_sparse_attn(q, k, v, block_map, q_block_sizes=None, kv_block_sizes=None, *,
+                      scale: float | None = None, out=None, return_indices: bool = False,
+                      stream=None):
+    """Block-sparse attention from a bool block map [B, H, n_q_blocks,
+    n_kv_blocks] (``block_sparse_attn``): converted on the device to index
+    rows, then the index-native kernel.  With ``return_indices`` also
+    returns the (q2k_idx, q2k_num) it produced."""
+    B, H, Sq, Skv, D, out = _sparse_common(q, k, v, out)
+    nq, nkv = Sq // 64, Skv // 64
+    if not isinstance(block_map, torch.Tensor) or block_map.dtype != torch.bool:
+        raise TypeError("block_map must be a torch.bool tensor")
+    if tuple(block_map.shape) != (B, H, nq, nkv) or not block_map.is_cuda or not block_map.is_contiguous():
+        raise ValueError(f"block_map must be a contiguous CUDA [B, H, n_q_blocks, n_kv_blocks] = "
+                         f"{(B, H, nq, nkv)} tensor")
+    dev = q.device
+    qbs = _block_sizes_tensor(q_block_sizes, nq, dev)
+    kbs = _block_sizes_tensor(kv_block_sizes, nkv, dev)
+    q2k_idx = torch.empty((B, H, nq, nkv), dtype=torch.int32, device=dev)
+    q2k_num = torch.empty((B, H, nq), dtype=torch.int32, device=dev)
+    L = lib()
+    ws = torch.empty(max(L.block_sparse_attn_from_indices_workspace_size(B, H, nq, nkv), 256),
+                     dtype=torch.uint8, device=dev)
+    lay = _layout(q, k, v, out)
+    _check("block_sparse_attn", L.block_sparse_attn(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(block_map), _ptr(qbs), _ptr(kbs), B, H, Sq, Skv, D,
+        float(scale) if scale is not None else 0.0, _ptr(out), _ptr(q2k_idx), _ptr(q2k_num),
+        ctypes.byref(lay), _ptr(ws), ws.numel(), _stream(stream)))
+    return (out, q2k_idx, q2k_num) if return_indices else out
+
+
+def video_sparse_attn_bshd(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=None, *,
+                           topk: int, scale: float | None = None, idx_stride: int | None = None,
+                           out=None, return_out_c: bool = False, workspace=None, stream=None):
+    """The whole VSA forward on BSHD tensors: q [B, Sq_pad, H, D], k and v
+    [B, Skv_pad, H, D], gate [B, Sq_pad, H, D]; the output is BSHD too.  The
+    library reads and writes the BSHD memory in place (strided views, no
+    transposed copies).  Returns ``(out, q2k_idx, q2k_num)`` (+ ``out_c``)."""
+    if out is None and isinstance(q, torch.Tensor):
+        out = torch.empty_like(q)
+    res = vsa_forward(q.transpose(1, 2), k.transpose(1, 2), v.transpose(1, 2), gate,
+                      q_block_sizes, kv_block_sizes, topk=topk, scale=scale, idx_stride=idx_stride,
+                      out=None if out is None else out.transpose(1, 2), return_out_c=return_out_c,
+                      workspace=workspace, stream=stream)
+    return (out,) + tuple(res[1:])
 
 
 def _host_i32(xs):

@@ -48,6 +48,51 @@ float resolve_scale(float scale, int D) {
   return scale > 0.f ? scale : 1.0f / sqrtf((float)D);
 }
 
+static Strides3 to_strides(const vsa_strides& s) { return Strides3{s.batch, s.head, s.seq}; }
+
+Strides3 bhsd_strides(int H, long long S, int D) {
+  return Strides3{(long long)H * S * D, S * D, (long long)D};
+}
+
+Strides3 gate_strides(int H, long long S, int D) {
+  return Strides3{S * H * D, (long long)D, (long long)H * D};
+}
+
+// A view is usable when every stride of an axis longer than one is a
+// positive multiple of 8 elements (16 bytes: TMA and 16-byte loads).
+static bool strides_ok(const Strides3& st, int B, int H, long long S) {
+  auto ok = [](long long stride, long long extent) {
+    return extent <= 1 || (stride > 0 && stride % 8 == 0);
+  };
+  return ok(st.b, B) && ok(st.h, H) && ok(st.s, S);
+}
+
+static bool layout_ok(const vsa_layout& L, int B, int H, long long Sq, long long Skv, bool gated) {
+  return strides_ok(to_strides(L.q), B, H, Sq) && strides_ok(to_strides(L.k), B, H, Skv) &&
+         strides_ok(to_strides(L.v), B, H, Skv) && strides_ok(to_strides(L.out), B, H, Sq) &&
+         (!gated || strides_ok(to_strides(L.gate), B, H, Sq));
+}
+
+static void fill_layout(int kind, int B, int H, int Sq, int Skv, int D, vsa_layout* L) {
+  (void)B;
+  auto set = [](vsa_strides& s, long long b, long long h, long long q) {
+    s.batch = b; s.head = h; s.seq = q;
+  };
+  if (kind == VSA_LAYOUT_BSHD) {
+    set(L->q, (long long)Sq * H * D, D, (long long)H * D);
+    set(L->out, (long long)Sq * H * D, D, (long long)H * D);
+    set(L->k, (long long)Skv * H * D, D, (long long)H * D);
+    set(L->v, (long long)Skv * H * D, D, (long long)H * D);
+  } else {
+    set(L->q, (long long)H * Sq * D, (long long)Sq * D, D);
+    set(L->out, (long long)H * Sq * D, (long long)Sq * D, D);
+    set(L->k, (long long)H * Skv * D, (long long)Skv * D, D);
+    set(L->v, (long long)H * Skv * D, (long long)Skv * D, D);
+  }
+  // the gate ("compress_attn_weight") is [B, Sq, H, D] memory in both
+  set(L->gate, (long long)Sq * H * D, D, (long long)H * D);
+}
+
 
 int check_forward_args(const ForwardArgs& a) {
   if (!a.q || !a.k || !a.v || !a.out || !a.q2k_idx || !a.q2k_num) return VSA_ERR_INVALID_ARG;
@@ -62,6 +107,10 @@ int check_forward_args(const ForwardArgs& a) {
   if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.out) ||
       (a.gate && !aligned16(a.gate)) || (a.out_c && !aligned16(a.out_c)))
     return VSA_ERR_INVALID_ARG;
+  if (!strides_ok(a.q_st, a.B, a.H, a.Sq_pad) || !strides_ok(a.k_st, a.B, a.H, a.Skv_pad) ||
+      !strides_ok(a.v_st, a.B, a.H, a.Skv_pad) || !strides_ok(a.out_st, a.B, a.H, a.Sq_pad) ||
+      (a.gate && !strides_ok(a.gate_st, a.B, a.H, a.Sq_pad)))
+    return VSA_ERR_UNSUPPORTED;
   return VSA_OK;
 }
 
@@ -97,9 +146,13 @@ int launch_forward(const ForwardArgs& a, void* scratch, bool profile, cudaStream
   pp.q = static_cast<const __nv_bfloat16*>(a.q);
   pp.k = static_cast<const __nv_bfloat16*>(a.k);
   pp.v = static_cast<const __nv_bfloat16*>(a.v);
+  pp.q_st = a.q_st;
+  pp.k_st = a.k_st;
+  pp.v_st = a.v_st;
   pp.q_bs = a.q_block_sizes;
   pp.kv_bs = a.kv_block_sizes;
   pp.groups = B * H;
+  pp.H = H;
   pp.nq = nq;
   pp.nkv = nkv;
   pp.qc = qc;
@@ -139,7 +192,9 @@ int launch_forward(const ForwardArgs& a, void* scratch, bool profile, cudaStream
   SparseParams sp;
   memset(&sp, 0, sizeof(sp));
   sp.out = static_cast<__nv_bfloat16*>(a.out);
+  sp.out_st = a.out_st;
   sp.gate = static_cast<const __nv_bfloat16*>(a.gate);
+  sp.gate_st = a.gate_st;
   sp.out_c = oc;
   sp.q2k_idx = a.q2k_idx;
   sp.q2k_num = a.q2k_num;
@@ -150,15 +205,12 @@ int launch_forward(const ForwardArgs& a, void* scratch, bool profile, cudaStream
   sp.H = H;
   sp.nq = nq;
   sp.nkv = nkv;
-  sp.q_rows_per_group = a.Sq_pad;
-  sp.kv_rows_per_group = a.Skv_pad;
-  sp.gate_seq = a.Sq_pad;
   sp.scale_log2 = sc * kLog2e;
   sp.qk_bound = qk_bound;
   sp.varlen = 0;
   sp.status = status;
-  rc = launch_sparse(sp, a.q, a.k, a.v, (long long)B * H * a.Sq_pad, (long long)B * H * a.Skv_pad,
-                     D, /*combine=*/true, /*gated=*/a.gate != nullptr, st);
+  rc = launch_sparse(sp, a.q, a.q_st, a.Sq_pad, a.k, a.k_st, a.v, a.v_st, a.Skv_pad, D,
+                     /*combine=*/true, /*gated=*/a.gate != nullptr, st);
   if (rc != VSA_OK) return rc;
   if (prof) cudaEventRecord(g_prof_events[3], st);
   return VSA_OK;
@@ -185,7 +237,7 @@ const char* vsa_status_string(int status) {
   }
 }
 
-int vsa_abi_version(void) { return (1 << 16) | 1; }
+int vsa_abi_version(void) { return (2 << 16) | 0; }
 
 int vsa_get_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return VSA_ERR_CUDA;
@@ -206,13 +258,24 @@ size_t vsa_forward_workspace_size(int B, int H, int n_q_blocks, int n_kv_blocks,
   return align256(g * n_q_blocks) * 2 + align256(g * n_kv_blocks) * 2 + align256(norms);
 }
 
-int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
-                const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B, int H,
-                int Sq_pad, int Skv_pad, int D, int topk, float scale, void* out,
-                int32_t* q2k_idx, int32_t* q2k_num, int idx_stride, float* out_c,
-                void* workspace, size_t workspace_bytes, void* stream) {
+int vsa_make_layout(int kind, int B, int H, int Sq_pad, int Skv_pad, int D, vsa_layout* layout) {
+  if (!layout || (kind != VSA_LAYOUT_BHSD && kind != VSA_LAYOUT_BSHD)) return VSA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || D <= 0) return VSA_ERR_INVALID_ARG;
+  fill_layout(kind, B, H, Sq_pad, Skv_pad, D, layout);
+  return VSA_OK;
+}
+
+int vsa_forward_strided(const void* q, const void* k, const void* v, const void* gate,
+                        const vsa_layout* layout, const int32_t* q_block_sizes,
+                        const int32_t* kv_block_sizes, int B, int H, int Sq_pad, int Skv_pad,
+                        int D, int topk, float scale, void* out, int32_t* q2k_idx,
+                        int32_t* q2k_num, int idx_stride, float* out_c, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!layout) return VSA_ERR_INVALID_ARG;
   ForwardArgs a;
   a.q = q; a.k = k; a.v = v; a.gate = gate;
+  a.q_st = to_strides(layout->q); a.k_st = to_strides(layout->k); a.v_st = to_strides(layout->v);
+  a.out_st = to_strides(layout->out); a.gate_st = to_strides(layout->gate);
   a.q_block_sizes = q_block_sizes; a.kv_block_sizes = kv_block_sizes;
   a.B = B; a.H = H; a.Sq_pad = Sq_pad; a.Skv_pad = Skv_pad; a.D = D; a.topk = topk;
   a.scale = scale; a.out = out; a.q2k_idx = q2k_idx; a.q2k_num = q2k_num;
@@ -225,14 +288,49 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
   return launch_forward(a, workspace, /*profile=*/true, static_cast<cudaStream_t>(stream));
 }
 
+int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
+                const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B, int H,
+                int Sq_pad, int Skv_pad, int D, int topk, float scale, void* out,
+                int32_t* q2k_idx, int32_t* q2k_num, int idx_stride, float* out_c,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || D <= 0) return VSA_ERR_INVALID_ARG;
+  vsa_layout L;
+  fill_layout(VSA_LAYOUT_BHSD, B, H, Sq_pad, Skv_pad, D, &L);
+  return vsa_forward_strided(q, k, v, gate, &L, q_block_sizes, kv_block_sizes, B, H, Sq_pad,
+                             Skv_pad, D, topk, scale, out, q2k_idx, q2k_num, idx_stride, out_c,
+                             workspace, workspace_bytes, stream);
+}
+
+int vsa_forward_bshd(const void* q, const void* k, const void* v, const void* gate,
+                     const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B, int H,
+                     int Sq_pad, int Skv_pad, int D, int topk, float scale, void* out,
+                     int32_t* q2k_idx, int32_t* q2k_num, int idx_stride, float* out_c,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || D <= 0) return VSA_ERR_INVALID_ARG;
+  vsa_layout L;
+  fill_layout(VSA_LAYOUT_BSHD, B, H, Sq_pad, Skv_pad, D, &L);
+  return vsa_forward_strided(q, k, v, gate, &L, q_block_sizes, kv_block_sizes, B, H, Sq_pad,
+                             Skv_pad, D, topk, scale, out, q2k_idx, q2k_num, idx_stride, out_c,
+                             workspace, workspace_bytes, stream);
+}
+
 // ---------------------------------------------------------------------------
 // block_sparse_attn_from_indices
 // ---------------------------------------------------------------------------
-int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
-                                   const int32_t* q2k_idx, const int32_t* q2k_num,
-                                   const int32_t* q_block_sizes, const int32_t* kv_block_sizes,
-                                   int B, int H, int Sq_pad, int Skv_pad, int D, int idx_stride,
-                                   float scale, void* out, void* stream) {
+size_t block_sparse_attn_from_indices_workspace_size(int B, int H, int n_q_blocks,
+                                                     int n_kv_blocks) {
+  if (B <= 0 || H <= 0 || n_q_blocks <= 0 || n_kv_blocks <= 0) return 0;
+  return align256(index_bound_bytes(B * H, n_q_blocks, n_kv_blocks));
+}
+
+// Shared by block_sparse_attn_from_indices and block_sparse_attn: checks,
+// the optional logit-bound pass, then the sparse kernel.
+static int sparse_from_indices(const void* q, const void* k, const void* v,
+                               const int32_t* q2k_idx, const int32_t* q2k_num,
+                               const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B,
+                               int H, int Sq_pad, int Skv_pad, int D, int idx_stride, float scale,
+                               void* out, const vsa_layout* layout, void* workspace,
+                               size_t workspace_bytes, cudaStream_t st) {
   if (!q || !k || !v || !out || !q2k_idx || !q2k_num) return VSA_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || idx_stride < 1 || !(scale == scale))
     return VSA_ERR_INVALID_ARG;
@@ -241,12 +339,49 @@ int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
   const int nq = Sq_pad / 64, nkv = Skv_pad / 64;
   if (idx_stride > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return VSA_ERR_INVALID_ARG;
+  vsa_layout L;
+  if (layout) L = *layout;
+  else fill_layout(VSA_LAYOUT_BHSD, B, H, Sq_pad, Skv_pad, D, &L);
+  if (!layout_ok(L, B, H, Sq_pad, Skv_pad, false)) return VSA_ERR_UNSUPPORTED;
+  if (workspace) {
+    const size_t need = block_sparse_attn_from_indices_workspace_size(B, H, nq, nkv);
+    if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+      return VSA_ERR_WORKSPACE;
+  }
   int* status = device_status_ptr();
   if (!status) return VSA_ERR_CUDA;
   const float sc = resolve_scale(scale, D);
+  const float* qk_bound = nullptr;
+  if (workspace) {
+    // logit bound of every item from block row norms and its selection
+    BoundParams bp;
+    memset(&bp, 0, sizeof(bp));
+    bp.q = static_cast<const __nv_bfloat16*>(q);
+    bp.k = static_cast<const __nv_bfloat16*>(k);
+    bp.q_st = to_strides(L.q);
+    bp.k_st = to_strides(L.k);
+    bp.q_seq = Sq_pad;
+    bp.kv_seq = Skv_pad;
+    bp.kv_len = kv_block_sizes;
+    bp.q2k_idx = q2k_idx;
+    bp.q2k_num = q2k_num;
+    bp.idx_stride = idx_stride;
+    bp.B = B;
+    bp.H = H;
+    bp.nqb = nq;
+    bp.nkvb = nkv;
+    bp.bound_scale = sc * kLog2e * (1.f + 0x1p-8f);
+    bp.qn = static_cast<float*>(workspace);
+    bp.kn = bp.qn + (size_t)B * H * nq;
+    bp.qk_bound = bp.kn + (size_t)B * H * nkv;
+    int rc = launch_index_bound(bp, D, st);
+    if (rc != VSA_OK) return rc;
+    qk_bound = bp.qk_bound;
+  }
   SparseParams sp;
   memset(&sp, 0, sizeof(sp));
   sp.out = static_cast<__nv_bfloat16*>(out);
+  sp.out_st = to_strides(L.out);
   sp.q2k_idx = q2k_idx;
   sp.q2k_num = q2k_num;
   sp.idx_stride = idx_stride;
@@ -256,12 +391,43 @@ int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
   sp.H = H;
   sp.nq = nq;
   sp.nkv = nkv;
-  sp.q_rows_per_group = Sq_pad;
-  sp.kv_rows_per_group = Skv_pad;
   sp.scale_log2 = sc * kLog2e;
+  sp.qk_bound = qk_bound;
   sp.status = status;
-  return launch_sparse(sp, q, k, v, (long long)B * H * Sq_pad, (long long)B * H * Skv_pad, D,
-                       false, false, static_cast<cudaStream_t>(stream));
+  return launch_sparse(sp, q, to_strides(L.q), Sq_pad, k, to_strides(L.k), v, to_strides(L.v),
+                       Skv_pad, D, false, false, st);
+}
+
+int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
+                                   const int32_t* q2k_idx, const int32_t* q2k_num,
+                                   const int32_t* q_block_sizes, const int32_t* kv_block_sizes,
+                                   int B, int H, int Sq_pad, int Skv_pad, int D, int idx_stride,
+                                   float scale, void* out, const vsa_layout* layout,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  return sparse_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes, kv_block_sizes, B, H,
+                             Sq_pad, Skv_pad, D, idx_stride, scale, out, layout, workspace,
+                             workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// block_sparse_attn (bool block map)
+// ---------------------------------------------------------------------------
+int block_sparse_attn(const void* q, const void* k, const void* v, const uint8_t* block_map,
+                      const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B, int H,
+                      int Sq_pad, int Skv_pad, int D, float scale, void* out, int32_t* q2k_idx,
+                      int32_t* q2k_num, const vsa_layout* layout, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  if (!block_map || !q2k_idx || !q2k_num) return VSA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0) return VSA_ERR_INVALID_ARG;
+  if (Sq_pad % 64 || Skv_pad % 64) return VSA_ERR_SHAPE;
+  const int nq = Sq_pad / 64, nkv = Skv_pad / 64;
+  if (nkv > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc = launch_mask_to_indices(block_map, (long long)B * H * nq, nkv, q2k_idx, q2k_num, st);
+  if (rc != VSA_OK) return rc;
+  return sparse_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes, kv_block_sizes, B, H,
+                             Sq_pad, Skv_pad, D, nkv, scale, out, layout, workspace,
+                             workspace_bytes, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -375,28 +541,41 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
   const long long total_q = cu_seqlens_q[n_seqs], total_kv = cu_seqlens_kv[n_seqs];
   const float sc = resolve_scale(scale, D);
   // logit bound (lets the sparse kernel skip its running-max check where it
-  // proves the check unneeded): block row norms, then per query block
+  // proves the check unneeded): block row norms, then per query block over
+  // the blocks it selected
   float* qn = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                        align256(sizeof(int32_t) * table.size()));
-  VarlenBoundParams bp;
+  // token-packed [H, total, D] tensors as [1, H, total, D] views
+  const Strides3 q_st{0, total_q * D, D}, kv_st{0, total_kv * D, D};
+  BoundParams bp;
+  memset(&bp, 0, sizeof(bp));
+  bp.q = static_cast<const __nv_bfloat16*>(q);
+  bp.k = static_cast<const __nv_bfloat16*>(k);
+  bp.q_st = q_st;
+  bp.k_st = kv_st;
+  bp.q_seq = total_q;
+  bp.kv_seq = total_kv;
   bp.q_tok = d_qtok;
   bp.kv_tok = d_ktok;
   bp.kv_len = d_klen;
   bp.q_kv_base = d_kvbase;
   bp.q_kv_count = d_kvcount;
+  bp.q2k_idx = q2k_idx;
+  bp.q2k_num = q2k_num;
+  bp.idx_stride = idx_stride;
+  bp.B = 1;
   bp.H = H;
   bp.nqb = nqb;
   bp.nkvb = nkvb;
-  bp.total_q = total_q;
-  bp.total_kv = total_kv;
   bp.bound_scale = sc * kLog2e * (1.f + 0x1p-8f);
   bp.qn = qn;
   bp.kn = qn + (size_t)H * nqb;
   bp.qk_bound = bp.kn + (size_t)H * nkvb;
-  if ((rc = launch_varlen_bound(q, k, bp, D, st)) != VSA_OK) return rc;
+  if ((rc = launch_index_bound(bp, D, st)) != VSA_OK) return rc;
   SparseParams sp;
   memset(&sp, 0, sizeof(sp));
   sp.out = static_cast<__nv_bfloat16*>(out);
+  sp.out_st = q_st;
   sp.q2k_idx = q2k_idx;
   sp.q2k_num = q2k_num;
   sp.idx_stride = idx_stride;
@@ -410,14 +589,11 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
   sp.H = H;
   sp.nq = nqb;
   sp.nkv = nkvb;
-  sp.q_rows_per_group = total_q;
-  sp.kv_rows_per_group = total_kv;
   sp.scale_log2 = sc * kLog2e;
   sp.qk_bound = bp.qk_bound;
   sp.varlen = 1;
   sp.status = status;
-  return launch_sparse(sp, q, k, v, (long long)H * total_q, (long long)H * total_kv, D, false,
-                       false, st);
+  return launch_sparse(sp, q, q_st, total_q, k, kv_st, v, kv_st, total_kv, D, false, false, st);
 }
 
 // ---------------------------------------------------------------------------

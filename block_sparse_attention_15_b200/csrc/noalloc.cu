@@ -57,6 +57,9 @@ extern "C" int vsa_forward_noalloc(const void* q, const void* k, const void* v, 
                                    int idx_stride, float* out_c, void* stream) {
   ForwardArgs a;
   a.q = q; a.k = k; a.v = v; a.gate = gate;
+  a.q_st = a.out_st = bhsd_strides(H, Sq_pad, D);
+  a.k_st = a.v_st = bhsd_strides(H, Skv_pad, D);
+  a.gate_st = gate_strides(H, Sq_pad, D);
   a.q_block_sizes = q_block_sizes; a.kv_block_sizes = kv_block_sizes;
   a.B = B; a.H = H; a.Sq_pad = Sq_pad; a.Skv_pad = Skv_pad; a.D = D; a.topk = topk;
   a.scale = scale; a.out = out; a.q2k_idx = q2k_idx; a.q2k_num = q2k_num;

@@ -33,32 +33,37 @@ __global__ void __launch_bounds__(256, 8) pool_kernel(PoolParams p) {
   __shared__ float red[RPP][D + 1];
   __shared__ float wmax[8];
 
-  long long item = blockIdx.x;
-  const long long nq_items = (long long)p.groups * p.nq;
-  const long long nkv_items = (long long)p.groups * p.nkv;
+  // 32-bit index arithmetic: the launcher caps the grid below 2^31 CTAs
+  int item = (int)blockIdx.x;
+  const int nq_items = p.groups * p.nq;
+  const int nkv_items = p.groups * p.nkv;
   const __nv_bfloat16* src;
+  Strides3 st;
   const int32_t* bs;
   float* dst;
   float* nrm;        // largest row norm of the block, or null
   bool all_rows;     // the norm covers the padding rows too (query side)
   int nblocks;
   if (item < nq_items) {
-    src = p.q; bs = p.q_bs; dst = p.qc; nblocks = p.nq; nrm = p.qn; all_rows = true;
+    src = p.q; st = p.q_st; bs = p.q_bs; dst = p.qc; nblocks = p.nq; nrm = p.qn; all_rows = true;
   } else if (item < nq_items + nkv_items) {
     item -= nq_items;
-    src = p.k; bs = p.kv_bs; dst = p.kc; nblocks = p.nkv; nrm = p.kn; all_rows = false;
+    src = p.k; st = p.k_st; bs = p.kv_bs; dst = p.kc; nblocks = p.nkv; nrm = p.kn; all_rows = false;
   } else {
     item -= nq_items + nkv_items;
-    src = p.v; bs = p.kv_bs; dst = p.vc; nblocks = p.nkv; nrm = nullptr; all_rows = false;
+    src = p.v; st = p.v_st; bs = p.kv_bs; dst = p.vc; nblocks = p.nkv; nrm = nullptr; all_rows = false;
   }
-  const int blk = (int)(item % nblocks);
+  const int group = item / nblocks;
+  const int blk = item - group * nblocks;
+  const int b = group / p.H, h = group - b * p.H;
   int m = bs ? bs[blk] : 64;
   if (m < 1 || m > 64) {
     if (threadIdx.x == 0) set_status(p.status, VSA_ERR_BLOCK_SIZE);
     m = m < 1 ? 1 : 64;
   }
   const int lim = (nrm && all_rows) ? 64 : m;  // rows read
-  const __nv_bfloat16* base = src + item * 64 * D;  // item = group*nblocks + blk
+  // first slot of the block in the strided view (item = group*nblocks + blk)
+  const __nv_bfloat16* base = src + b * st.b + h * st.h + 64LL * blk * st.s;
   const int chunk = threadIdx.x % CPR;
   const int r0 = threadIdx.x / CPR;
 
@@ -67,7 +72,7 @@ __global__ void __launch_bounds__(256, 8) pool_kernel(PoolParams p) {
   for (int ps = 0; ps < PASSES; ++ps) {
     const int row = r0 + ps * RPP;
     if (row < lim) {
-      buf[ps] = __ldcs(reinterpret_cast<const uint4*>(base + (long long)row * D) + chunk);
+      buf[ps] = __ldcs(reinterpret_cast<const uint4*>(base + (long long)row * st.s) + chunk);
     } else {
       buf[ps] = make_uint4(0u, 0u, 0u, 0u);
     }
@@ -114,7 +119,7 @@ __global__ void __launch_bounds__(256, 8) pool_kernel(PoolParams p) {
     float s = 0.f;
 #pragma unroll
     for (int r = 0; r < RPP; ++r) s += red[r][threadIdx.x];
-    dst[item * D + threadIdx.x] = __fdiv_rn(s, (float)m);
+    dst[(long long)item * D + threadIdx.x] = __fdiv_rn(s, (float)m);
   }
   if (nrm && threadIdx.x == 0) {
     float mx = wmax[0];

@@ -340,6 +340,18 @@ __device__ __forceinline__ Item load_item(const SparseParams& p, long long it) {
   return x;
 }
 
+// A 64 x 64 tile of a strided [B, H, S, D] view through its 4-D tensor map:
+// head dims d0 .. d0+63 of sequence slots s .. s+63 of (b, h).  Slots past the
+// view's end arrive as zeros.
+__device__ __forceinline__ void load_view_tile(void* dst, const CUtensorMap* map, TmaAxes ax,
+                                               uint64_t* bar, int d0, int s, int h, int b,
+                                               uint64_t hint) {
+  const int c1 = ax.s == 1 ? s : (ax.h == 1 ? h : b);
+  const int c2 = ax.s == 2 ? s : (ax.h == 2 ? h : b);
+  const int c3 = ax.s == 3 ? s : (ax.h == 3 ? h : b);
+  tma_load_4d(dst, map, bar, d0, c1, c2, c3, hint);
+}
+
 // Report a work item whose count or query block size is out of range.
 __device__ __forceinline__ void check_item(const SparseParams& p, long long it) {
   const long long t = it / p.nq;
@@ -442,18 +454,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = mbar_wait(bars + L::kQEmpty, (uint32_t)((n - 1) & 1), abort_flag, p.status);
             if (ok) {
               mbar_arrive_expect_tx(bars + L::kQFull, L::kQ);
-              const int q_row = (int)(x.group * p.q_rows_per_group + x.q_tok);
 #pragma unroll
               for (int dh = 0; dh < L::DH; ++dh)
-                tma_load_2d(smem + L::kQOff + dh * 8192, &tm_q, bars + L::kQFull, dh * 64, q_row,
-                            pol_q);
+                load_view_tile(smem + L::kQOff + dh * 8192, &tm_q, p.q_ax, bars + L::kQFull, dh * 64,
+                               (int)x.q_tok, x.h, x.b, pol_q);
             }
           }
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
         const int32_t* idx_row = p.q2k_idx + (x.group * p.nq + x.a) * (long long)p.idx_stride;
         const int np = (x.num + 1) / 2;
-        const long long kv_row0 = x.group * p.kv_rows_per_group;
         for (int j0 = 0; ok && j0 < x.num; j0 += 32) {
           int row, len;
           resolve_entry(p, x, idx_row, j0 + lane, row, len);
@@ -486,16 +496,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                   mbar_arrive_expect_tx(full, L::kK2);
 #pragma unroll
                   for (int dh = 0; dh < L::DH; ++dh) {
-                    tma_load_2d(dst + k_slot_off<D>(dh, 0), &tm_k, full, dh * 64, (int)(kv_row0 + r0), pol_kv);
-                    tma_load_2d(dst + k_slot_off<D>(dh, 1), &tm_k, full, dh * 64, (int)(kv_row0 + r1), pol_kv);
+                    load_view_tile(dst + k_slot_off<D>(dh, 0), &tm_k, p.k_ax, full, dh * 64, r0, x.h, x.b, pol_kv);
+                    load_view_tile(dst + k_slot_off<D>(dh, 1), &tm_k, p.k_ax, full, dh * 64, r1, x.h, x.b, pol_kv);
                   }
                 } else {
                   uint8_t* dst = smem + L::kVOff + st * L::kV2;
                   mbar_arrive_expect_tx(full, L::kV2);
 #pragma unroll
                   for (int dh = 0; dh < L::DH; ++dh) {
-                    tma_load_2d(dst + v_slot_off<D>(0, dh), &tm_v, full, dh * 64, (int)(kv_row0 + r0), pol_kv);
-                    tma_load_2d(dst + v_slot_off<D>(1, dh), &tm_v, full, dh * 64, (int)(kv_row0 + r1), pol_kv);
+                    load_view_tile(dst + v_slot_off<D>(0, dh), &tm_v, p.v_ax, full, dh * 64, r0, x.h, x.b, pol_kv);
+                    load_view_tile(dst + v_slot_off<D>(1, dh), &tm_v, p.v_ax, full, dh * 64, r1, x.h, x.b, pol_kv);
                   }
                   *reinterpret_cast<volatile int*>(smem + L::kVIssuedOff) = (int)(gp + 1);
                 }
@@ -816,8 +826,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (bar_red_or(5, 128, bad)) break;
       float4 oc = make_float4(0.f, 0.f, 0.f, 0.f);
       if (COMBINE) oc = *reinterpret_cast<const float4*>(p.out_c + (x.group * p.nq + x.a) * (long long)D + d0);
-      const long long orow0 = x.group * p.q_rows_per_group + x.q_tok;
-      const long long grow0 = ((long long)x.b * p.gate_seq + x.q_tok) * p.H + x.h;
+      // element offsets of the block's first token in out and gate
+      __nv_bfloat16* orow0 = p.out + x.b * p.out_st.b + x.h * p.out_st.h + x.q_tok * p.out_st.s + d0;
+      const __nv_bfloat16* grow0 =
+          GATED ? p.gate + x.b * p.gate_st.b + x.h * p.gate_st.h + x.q_tok * p.gate_st.s + d0 : nullptr;
       for (int rnd = 0; rnd < 4; ++rnd) {
         if (active) {
           uint32_t ov[16];
@@ -850,7 +862,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float v0 = v4.x, v1 = v4.y, v2 = v4.z, v3 = v4.w;
             if (COMBINE) {
               if (GATED) {
-                const uint2 graw = *reinterpret_cast<const uint2*>(p.gate + (grow0 + (long long)q * p.H) * D + d0);
+                const uint2 graw = *reinterpret_cast<const uint2*>(grow0 + q * p.gate_st.s);
                 const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&graw.x));
                 const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&graw.y));
                 v0 = fmaf(oc.x, g01.x, v0);
@@ -861,10 +873,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 v0 += oc.x; v1 += oc.y; v2 += oc.z; v3 += oc.w;
               }
             }
-            *reinterpret_cast<uint2*>(p.out + (orow0 + q) * D + d0) =
+            *reinterpret_cast<uint2*>(orow0 + q * p.out_st.s) =
                 make_uint2(pack_bf16x2(v0, v1), pack_bf16x2(v2, v3));
           } else if (!p.varlen) {
-            *reinterpret_cast<uint2*>(p.out + (orow0 + q) * D + d0) = make_uint2(0u, 0u);
+            *reinterpret_cast<uint2*>(orow0 + q * p.out_st.s) = make_uint2(0u, 0u);
           }
         }
         named_barrier_sync(5, 128);
@@ -985,15 +997,41 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// Row-major [rows][D] bf16 tensor, 64x64 boxes, 128-byte swizzle.
-static bool make_tile_map(CUtensorMap* map, const void* base, long long rows, int D) {
+// 4-D map of a strided [B, H, S, D] bf16 view: dimension 0 is the head dim,
+// dimensions 1..3 the sequence, head and batch axes in increasing stride
+// order (an axis of extent 1 goes last, with the stride an outer contiguous
+// axis would have); 64 x 1 x 64 x 1 boxes (64 head dims of 64 slots of one
+// head and batch), 128-byte swizzle.  The caller checked that every stride
+// is a multiple of 8 elements (16 bytes) and the base 16-byte aligned.
+static bool make_view_map(CUtensorMap* map, TmaAxes* ax, const void* base, int D, long long S,
+                          int H, int B, Strides3 st) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, 64};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+  struct A { int id; long long ext, str; } a[3] = {{0, S, st.s}, {1, H, st.h}, {2, B, st.b}};
+  // order: axes of extent > 1 by stride, then the rest
+  for (int i = 0; i < 3; ++i)
+    for (int j = i + 1; j < 3; ++j) {
+      const bool ai = a[i].ext > 1, aj = a[j].ext > 1;
+      if ((!ai && aj) || (ai == aj && ai && a[j].str < a[i].str)) { A t = a[i]; a[i] = a[j]; a[j] = t; }
+    }
+  cuuint64_t dims[4] = {(cuuint64_t)D, 0, 0, 0};
+  cuuint64_t strides[3];
+  long long outer = (long long)D * 2;  // bytes spanned so far
+  for (int i = 0; i < 3; ++i) {
+    long long sb = a[i].str * 2;
+    if (a[i].ext <= 1 || sb <= 0) sb = outer;  // never stepped: any valid stride
+    dims[i + 1] = (cuuint64_t)a[i].ext;
+    strides[i] = (cuuint64_t)sb;
+    outer = sb * a[i].ext > outer ? sb * a[i].ext : outer;
+    const int slot = i + 1;
+    if (a[i].id == 0) ax->s = slot;
+    else if (a[i].id == 1) ax->h = slot;
+    else ax->b = slot;
+  }
+  cuuint32_t box[4] = {64, 1, 1, 1};
+  box[ax->s] = 64;
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -1034,15 +1072,17 @@ static int launch_sparse_t(const SparseParams& p, const CUtensorMap& mq, const C
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
-int launch_sparse(const SparseParams& p, const void* q, const void* k, const void* v,
-                  long long q_rows_total, long long kv_rows_total, int D, bool combine,
-                  bool gated, cudaStream_t stream) {
-  if (p.nq <= 0 || p.H <= 0 || p.B <= 0) return VSA_OK;
-  if (q_rows_total + 64 > 0x7FFFFFFFLL || kv_rows_total + 64 > 0x7FFFFFFFLL)
-    return VSA_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
+int launch_sparse(const SparseParams& p_in, const void* q, Strides3 q_st, long long q_seq,
+                  const void* k, Strides3 k_st, const void* v, Strides3 v_st, long long kv_seq,
+                  int D, bool combine, bool gated, cudaStream_t stream) {
+  if (p_in.nq <= 0 || p_in.H <= 0 || p_in.B <= 0) return VSA_OK;
+  if (q_seq + 64 > 0x7FFFFFFFLL || kv_seq + 64 > 0x7FFFFFFFLL)
+    return VSA_ERR_UNSUPPORTED;  // TMA coordinates are 32-bit
+  SparseParams p = p_in;
   CUtensorMap mq, mk, mv;
-  if (!make_tile_map(&mq, q, q_rows_total, D) || !make_tile_map(&mk, k, kv_rows_total, D) ||
-      !make_tile_map(&mv, v, kv_rows_total, D))
+  if (!make_view_map(&mq, &p.q_ax, q, D, q_seq, p.H, p.B, q_st) ||
+      !make_view_map(&mk, &p.k_ax, k, D, kv_seq, p.H, p.B, k_st) ||
+      !make_view_map(&mv, &p.v_ax, v, D, kv_seq, p.H, p.B, v_st))
     return VSA_ERR_CUDA;
   if (D == 128) {
     if (!combine) return launch_sparse_t<128, false, false>(p, mq, mk, mv, stream);

@@ -9,13 +9,28 @@
 
 namespace vsa {
 
+// Element strides of a [batch][head][sequence slot][head dim] view whose head
+// dim is contiguous.
+struct Strides3 {
+  long long b, h, s;
+};
+
+// Tensor-map dimension (1..3) that holds each of the sequence, head and
+// batch axes of a 4D tile map (dimension 0 is the head dim): the three axes
+// are ordered by stride on the host.
+struct TmaAxes {
+  int s, h, b;
+};
+
 struct PoolParams {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
+  Strides3 q_st, k_st, v_st;
   const int32_t* q_bs;   // [nq] or null (all 64)
   const int32_t* kv_bs;  // [nkv] or null
   int groups;            // B * H
+  int H;
   int nq, nkv;
   float* qc;             // [groups, nq, D]
   float* kc;             // [groups, nkv, D]
@@ -47,13 +62,16 @@ struct CoarseParams {
 };
 
 // One launch of the block-sparse kernel.  Work item = (query block a, head h,
-// batch b); "group" = b * H + h.  Rows of q/out are addressed as
-//   group * q_rows_per_group + q_tok(a) + t
-// and rows of k/v as group * kv_rows_per_group + kv_tok(c) + t, where
-// q_tok(a) = 64 a unless a varlen table is given.
+// batch b); "group" = b * H + h.  Token t of query block a is sequence slot
+// q_tok(a) + t of (b, h) in q and out, token t of KV block c is slot
+// kv_tok(c) + t in k and v, where q_tok(a) = 64 a and kv_tok(c) = 64 c unless
+// a varlen table is given.  Every tensor is a strided [B, H, S, D] view.
 struct SparseParams {
   __nv_bfloat16* out;
-  const __nv_bfloat16* gate;  // [B, gate_seq, H, D] or null
+  Strides3 out_st;
+  const __nv_bfloat16* gate;  // strided [B, H, Sq, D] view or null
+  Strides3 gate_st;
+  TmaAxes q_ax, k_ax, v_ax;   // filled by launch_sparse
   const float* out_c;         // [groups, nq, D] or null (no combine)
   const int32_t* q2k_idx;     // [groups, nq, idx_stride]
   const int32_t* q2k_num;     // [groups, nq]
@@ -65,9 +83,6 @@ struct SparseParams {
   const int32_t* q_kv_base;   // varlen: first kv block of the q block's sequence
   const int32_t* q_kv_count;  // varlen: kv blocks of the q block's sequence
   int B, H, nq, nkv;
-  long long q_rows_per_group;
-  long long kv_rows_per_group;
-  int gate_seq;
   float scale_log2;           // softmax scale * log2(e)
   const float* qk_bound;      // [groups, nq] bound on scale_log2 * q.k (CoarseParams), or null
   int varlen;                 // write only real rows
@@ -76,34 +91,43 @@ struct SparseParams {
 
 int launch_pool(const PoolParams& p, int D, cudaStream_t stream);
 int launch_coarse_topk(const CoarseParams& p, int D, cudaStream_t stream);
-// q, k, v: base pointers of the row-major [rows, D] bf16 views.
-int launch_sparse(const SparseParams& p, const void* q, const void* k, const void* v,
-                  long long q_rows_total, long long kv_rows_total, int D, bool combine,
-                  bool gated, cudaStream_t stream);
+// q, k, v: strided [B, H, S, D] bf16 views with S = q_seq / kv_seq slots
+// (element strides multiples of 8, bases 16-byte aligned).
+int launch_sparse(const SparseParams& p, const void* q, Strides3 q_st, long long q_seq,
+                  const void* k, Strides3 k_st, const void* v, Strides3 v_st, long long kv_seq,
+                  int D, bool combine, bool gated, cudaStream_t stream);
 int launch_selftest_umma(int mode, int D, const void* a, const void* b, float* c,
                          cudaStream_t stream);
 int launch_selftest_exp2(const float* x, float* y, long long n, int* mismatch,
                          cudaStream_t stream);
 
 // varlen / metadata helpers (vsa_varlen.cu)
-// Logit bound for the varlen entry (same meaning as CoarseParams::qk_bound):
-// block row norms of the packed q and k, then per (head, query block) the
-// bound over its sequence's KV blocks.
-struct VarlenBoundParams {
-  const int32_t* q_tok;       // [nqb] first packed row of each query block
-  const int32_t* kv_tok;      // [nkvb]
-  const int32_t* kv_len;      // [nkvb] real rows
-  const int32_t* q_kv_base;   // [nqb] first KV block of the query block's sequence
-  const int32_t* q_kv_count;  // [nqb]
-  int H, nqb, nkvb;
-  long long total_q, total_kv;  // packed rows per head
+// Logit bound for the entries that take indices (same meaning as
+// CoarseParams::qk_bound): block row norms of q and k, then per (group,
+// query block) bound_scale * its query norm * the largest key norm among the
+// KV blocks it lists in q2k_idx.
+struct BoundParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  Strides3 q_st, k_st;
+  long long q_seq, kv_seq;    // sequence slots of q and k per (b, h)
+  const int32_t* q_tok;       // [nqb] first slot of each query block, or null (64 a)
+  const int32_t* kv_tok;      // [nkvb] or null (64 c)
+  const int32_t* kv_len;      // [nkvb] real rows, or null (64)
+  const int32_t* q_kv_base;   // [nqb] first KV block of the query block's sequence, or null (0)
+  const int32_t* q_kv_count;  // [nqb] or null (nkvb)
+  const int32_t* q2k_idx;     // [groups, nqb, idx_stride] (indices local to the sequence)
+  const int32_t* q2k_num;     // [groups, nqb]
+  int idx_stride;
+  int B, H, nqb, nkvb;
   float bound_scale;
-  float* qn;                  // [H, nqb]
-  float* kn;                  // [H, nkvb]
-  float* qk_bound;            // [H, nqb]
+  float* qn;                  // [groups, nqb]
+  float* kn;                  // [groups, nkvb]
+  float* qk_bound;            // [groups, nqb]
 };
-int launch_varlen_bound(const void* q, const void* k, const VarlenBoundParams& p, int D,
-                        cudaStream_t stream);
+int launch_index_bound(const BoundParams& p, int D, cudaStream_t stream);
+// Scratch bytes launch_index_bound needs for its norms and bound.
+size_t index_bound_bytes(int groups, int nqb, int nkvb);
 int launch_varlen_aux(const int32_t* blk_tok, const int32_t* blk_len, int n_blocks,
                       int64_t* pack_index, cudaStream_t stream);
 int launch_rebase(const int32_t* q2k_idx, const int32_t* q2k_num, const int32_t* q_kv_base,
@@ -129,13 +153,15 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Softmax scale: the given one, or 1/sqrt(D) when it is <= 0.
 float resolve_scale(float scale, int D);
 
-// Arguments of the whole forward (vsa_forward and vsa_forward_noalloc share
-// the checks and the launch sequence; only the source of the scratch differs).
+// Arguments of the whole forward (vsa_forward, vsa_forward_strided and
+// vsa_forward_noalloc share the checks and the launch sequence; only the
+// layout and the source of the scratch differ).
 struct ForwardArgs {
   const void* q;
   const void* k;
   const void* v;
   const void* gate;
+  Strides3 q_st, k_st, v_st, out_st, gate_st;
   const int32_t* q_block_sizes;
   const int32_t* kv_block_sizes;
   int B, H, Sq_pad, Skv_pad, D, topk;
@@ -146,6 +172,15 @@ struct ForwardArgs {
   int idx_stride;
   float* out_c;
 };
+// Strides of contiguous [B, H, S, D] tensors, and of the gate's [B, S, H, D]
+// memory seen as a [B, H, S, D] view.
+Strides3 bhsd_strides(int H, long long S, int D);
+Strides3 gate_strides(int H, long long S, int D);
+// Bool block map [rows, nkv] (1 byte per entry, nonzero = selected) to
+// ascending q2k_idx rows of width nkv (-1 after the selected blocks) and
+// q2k_num.
+int launch_mask_to_indices(const uint8_t* block_map, long long rows, int nkv, int32_t* q2k_idx,
+                           int32_t* q2k_num, cudaStream_t stream);
 // Host checks of vsa_forward's arguments (everything but the workspace).
 int check_forward_args(const ForwardArgs& a);
 // Pool, coarse + top-k and the sparse kernel with the fused combine, on

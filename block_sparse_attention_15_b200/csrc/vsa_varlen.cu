@@ -72,45 +72,49 @@ __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint4* src, ui
   }
 }
 
-// Largest row L2 norm of one packed block per (head, block): query blocks
-// over the 64 rows from the block's first token (the rows the sparse kernel's
-// query tile holds, clipped at the end of the tensor), key blocks over their
-// real rows.  One CTA of 256 threads per (head, block); the squared norms of
-// a row's D/8 16-byte chunks add up across consecutive lanes.
+// Largest row L2 norm of one block per (group, block): query blocks over the
+// 64 slots from the block's first token (the rows the sparse kernel's query
+// tile holds, clipped at the end of the sequence), key blocks over their real
+// rows.  One CTA of 256 threads per (group, block); the squared norms of a
+// row's D/8 16-byte chunks add up across consecutive lanes.
 template <int D>
-__global__ void __launch_bounds__(256, 8) varlen_norm_kernel(const __nv_bfloat16* q,
-                                                          const __nv_bfloat16* k, VarlenBoundParams p) {
+__global__ void __launch_bounds__(256, 8) block_norm_kernel(BoundParams p) {
   constexpr int CPR = D / 8, RPP = 256 / CPR, PASSES = 64 / RPP;
   __shared__ float wmax[8];
-  const long long item = blockIdx.x;  // h * (nqb + nkvb) + block
-  const int per_head = p.nqb + p.nkvb;
-  const int h = (int)(item / per_head), blk = (int)(item % per_head);
+  const long long item = blockIdx.x;  // group * (nqb + nkvb) + block
+  const int per_group = p.nqb + p.nkvb;
+  const long long group = item / per_group;
+  const int blk = (int)(item % per_group);
+  const int b = (int)(group / p.H), h = (int)(group % p.H);
   const bool is_q = blk < p.nqb;
-  const __nv_bfloat16* src;
-  long long row0, rows_end;
+  const __nv_bfloat16* base;
+  long long s0, s_end, st;
   int rows;
   float* dst;
   if (is_q) {
-    src = q;
-    row0 = (long long)h * p.total_q + p.q_tok[blk];
-    rows_end = (long long)p.H * p.total_q;
+    base = p.q + b * p.q_st.b + h * p.q_st.h;
+    st = p.q_st.s;
+    s0 = p.q_tok ? p.q_tok[blk] : 64LL * blk;
+    s_end = p.q_seq;
     rows = 64;
-    dst = p.qn + (long long)h * p.nqb + blk;
+    dst = p.qn + group * p.nqb + blk;
   } else {
     const int c = blk - p.nqb;
-    src = k;
-    row0 = (long long)h * p.total_kv + p.kv_tok[c];
-    rows_end = (long long)p.H * p.total_kv;
-    rows = p.kv_len[c];
-    dst = p.kn + (long long)h * p.nkvb + c;
+    base = p.k + b * p.k_st.b + h * p.k_st.h;
+    st = p.k_st.s;
+    s0 = p.kv_tok ? p.kv_tok[c] : 64LL * c;
+    s_end = p.kv_seq;
+    rows = p.kv_len ? p.kv_len[c] : 64;
+    rows = rows < 0 ? 0 : (rows > 64 ? 64 : rows);
+    dst = p.kn + group * p.nkvb + c;
   }
   const int chunk = threadIdx.x % CPR, r0 = threadIdx.x / CPR;
   uint4 buf[PASSES];  // every load issued before any use
 #pragma unroll
   for (int ps = 0; ps < PASSES; ++ps) {
     const int r = r0 + ps * RPP;
-    buf[ps] = (r < rows && row0 + r < rows_end)
-                  ? __ldcs(reinterpret_cast<const uint4*>(src + (row0 + r) * D) + chunk)
+    buf[ps] = (r < rows && s0 + r < s_end)
+                  ? __ldcs(reinterpret_cast<const uint4*>(base + (s0 + r) * st) + chunk)
                   : make_uint4(0u, 0u, 0u, 0u);
   }
   float mx = 0.f;
@@ -140,31 +144,77 @@ __global__ void __launch_bounds__(256, 8) varlen_norm_kernel(const __nv_bfloat16
   }
 }
 
-// Per (head, query block): bound_scale * its query norm * the largest key
-// norm among its sequence's KV blocks.
-__global__ void varlen_bound_kernel(VarlenBoundParams p) {
+// Per (group, query block): bound_scale * its query norm * the largest key
+// norm among the KV blocks its q2k_idx row lists (entries outside the
+// sequence's blocks are skipped here; the sparse kernel reports them).  A
+// tighter bound than the largest key norm of the whole head, so more items
+// take the vote-free step.
+__global__ void index_bound_kernel(BoundParams p) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (long long)p.H * p.nqb) return;
-  const int h = (int)(i / p.nqb), a = (int)(i % p.nqb);
-  const float* kn = p.kn + (long long)h * p.nkvb + p.q_kv_base[a];
+  if (i >= (long long)p.B * p.H * p.nqb) return;
+  const long long group = i / p.nqb;
+  const int a = (int)(i % p.nqb);
+  const int base = p.q_kv_base ? p.q_kv_base[a] : 0;
+  const int count = p.q_kv_count ? p.q_kv_count[a] : p.nkvb;
+  const float* kn = p.kn + group * p.nkvb + base;
+  const int32_t* idx = p.q2k_idx + i * p.idx_stride;
+  int num = p.q2k_num[i];
+  num = num < 0 ? 0 : (num > p.idx_stride ? p.idx_stride : num);
   float km = 0.f;
-  for (int j = 0; j < p.q_kv_count[a]; ++j) km = fmaxf(km, kn[j]);
+  for (int j = 0; j < num; ++j) {
+    const int c = idx[j];
+    if (c >= 0 && c < count) km = fmaxf(km, kn[c]);
+  }
   p.qk_bound[i] = p.bound_scale * p.qn[i] * km;
 }
 
-int launch_varlen_bound(const void* q, const void* k, const VarlenBoundParams& p, int D,
-                        cudaStream_t stream) {
-  const unsigned grid = (unsigned)((long long)p.H * (p.nqb + p.nkvb));
-  if (grid == 0) return VSA_OK;
-  if (D == 128)
-    varlen_norm_kernel<128><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q),
-                                                       static_cast<const __nv_bfloat16*>(k), p);
-  else
-    varlen_norm_kernel<64><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q),
-                                                      static_cast<const __nv_bfloat16*>(k), p);
+size_t index_bound_bytes(int groups, int nqb, int nkvb) {
+  return sizeof(float) * (size_t)groups * (2 * (size_t)nqb + nkvb);
+}
+
+int launch_index_bound(const BoundParams& p, int D, cudaStream_t stream) {
+  const long long groups = (long long)p.B * p.H;
+  const long long grid = groups * (p.nqb + p.nkvb);
+  if (grid <= 0) return VSA_OK;
+  if (grid > 0x7FFFFFFFLL) return VSA_ERR_UNSUPPORTED;
+  if (D == 128) block_norm_kernel<128><<<(unsigned)grid, 256, 0, stream>>>(p);
+  else block_norm_kernel<64><<<(unsigned)grid, 256, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return VSA_ERR_CUDA;
-  const long long n = (long long)p.H * p.nqb;
-  varlen_bound_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(p);
+  const long long n = groups * p.nqb;
+  index_bound_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+// One warp per row of the block map: the selected KV blocks in ascending
+// order by ballot compaction, 32 columns at a time ("[chore] release
+// fastvideo-kernel 0.3.0", Block-sparse / VSA attention improvements: the
+// legacy bool block_map API becomes a wrapper over the index-native kernel).
+__global__ void __launch_bounds__(256) mask_to_indices_kernel(const uint8_t* block_map, long long rows,
+                                                              int nkv, int32_t* q2k_idx,
+                                                              int32_t* q2k_num) {
+  const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= rows) return;
+  const uint8_t* m = block_map + row * nkv;
+  int32_t* out = q2k_idx + row * nkv;
+  int n = 0;
+  for (int c0 = 0; c0 < nkv; c0 += 32) {
+    const int c = c0 + lane;
+    const bool sel = c < nkv && m[c] != 0;
+    const uint32_t ball = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[n + __popc(ball & ((1u << lane) - 1u))] = c;
+    n += __popc(ball);
+  }
+  for (int j = n + lane; j < nkv; j += 32) out[j] = -1;
+  if (lane == 0) q2k_num[row] = n;
+}
+
+int launch_mask_to_indices(const uint8_t* block_map, long long rows, int nkv, int32_t* q2k_idx,
+                           int32_t* q2k_num, cudaStream_t stream) {
+  if (rows <= 0 || nkv <= 0) return VSA_OK;
+  const long long grid = (rows + 7) / 8;
+  if (grid > 0x7FFFFFFFLL) return VSA_ERR_UNSUPPORTED;
+  mask_to_indices_kernel<<<(unsigned)grid, 256, 0, stream>>>(block_map, rows, nkv, q2k_idx, q2k_num);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 

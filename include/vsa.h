@@ -73,6 +73,33 @@ extern "C" {
  * per query block (the coarse stage keeps a full score row on chip). */
 #define VSA_MAX_BLOCKS 2048
 
+/* ---- strided views ------------------------------------------------------ */
+/*
+ * Element strides (not bytes) of a tensor seen as [batch][head][sequence
+ * slot][head dim] with the head dim contiguous.  Every stride of an axis
+ * longer than one must be a positive multiple of 8 elements (16 bytes;
+ * VSA_ERR_UNSUPPORTED otherwise); a stride of an axis of length one is never
+ * used.  Views must not overlap the output.
+ */
+typedef struct vsa_strides {
+  int64_t batch, head, seq;
+} vsa_strides;
+
+/* Strides of every tensor of one call.  `gate` describes the gate as a
+ * [B, H, Sq, D] view of its memory: for the pages' [B, S, H, D] gate
+ * ("compress_attn_weight", passed to the BHSD kernel as a transposed view in
+ * PR #1813's follow-up) that is {S*H*D, D, H*D}. */
+typedef struct vsa_layout {
+  vsa_strides q, k, v, out, gate;
+} vsa_layout;
+
+#define VSA_LAYOUT_BHSD 0 /* q, k, v, out contiguous [B, H, S, D] */
+#define VSA_LAYOUT_BSHD 1 /* q, k, v, out contiguous [B, S, H, D] */
+
+/* Fill `layout` for contiguous tensors of the given kind; the gate is
+ * contiguous [B, Sq_pad, H, D] memory in both kinds.  Host only. */
+int vsa_make_layout(int kind, int B, int H, int Sq_pad, int Skv_pad, int D, vsa_layout* layout);
+
 /* Human-readable name of a status code (static string). */
 const char* vsa_status_string(int status);
 
@@ -137,6 +164,36 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
                 int Sq_pad, int Skv_pad, int D, int topk, float scale, void* out,
                 int32_t* q2k_idx, int32_t* q2k_num, int idx_stride, float* out_c,
                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * vsa_forward_strided -- vsa_forward on strided views: q, k, v, out and gate
+ * are read and written through the strides in `layout` (host pointer), so
+ * BSHD tensors, slices of a fused QKV tensor and a transposed gate view need
+ * no copy.  Same results as vsa_forward on the same values.
+ *
+ * Defined by: release 0.3.0, "Block-sparse / VSA attention improvements"
+ * (the BSHD-native `video_sparse_attn_bshd` entry, the "skip the bool-mask
+ * round-trip" item) and PR #1813's follow-up (the gate passed as a
+ * transposed view of its [B, S, H, D] memory).  All other arguments as in
+ * vsa_forward; the workspace is the same size.
+ */
+int vsa_forward_strided(const void* q, const void* k, const void* v, const void* gate,
+                        const vsa_layout* layout, const int32_t* q_block_sizes,
+                        const int32_t* kv_block_sizes, int B, int H, int Sq_pad, int Skv_pad,
+                        int D, int topk, float scale, void* out, int32_t* q2k_idx,
+                        int32_t* q2k_num, int idx_stride, float* out_c, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/*
+ * vsa_forward_bshd -- vsa_forward with q, k, v and out contiguous
+ * [B, S_pad, H, D] (the layout of release 0.3.0's `video_sparse_attn_bshd`)
+ * and the gate [B, Sq_pad, H, D]; arguments otherwise as in vsa_forward.
+ */
+int vsa_forward_bshd(const void* q, const void* k, const void* v, const void* gate,
+                     const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B, int H,
+                     int Sq_pad, int Skv_pad, int D, int topk, float scale, void* out,
+                     int32_t* q2k_idx, int32_t* q2k_num, int idx_stride, float* out_c,
+                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * vsa_forward_noalloc -- vsa_forward for callers that cannot allocate device
@@ -229,12 +286,50 @@ int vsa_forward_host(const void* q, const void* k, const void* v, const void* ga
  * q2k_num  device int32 [B, H, n_q_blocks], each in [0, idx_stride]
  * idx_stride  1 .. VSA_MAX_BLOCKS
  * out      device bf16 [B, H, Sq_pad, D]
+ * layout   host, strides of q, k, v and out (gate unused), or NULL for
+ *          contiguous BHSD
+ * workspace  device, >= block_sparse_attn_from_indices_workspace_size(...)
+ *          bytes, 256-aligned, or NULL.  With it, one extra pass takes block
+ *          row norms of q and k and bounds every query block's logits by
+ *          its query norm times the largest key norm among the blocks it
+ *          lists; where the bound shows no logit can exceed the first tile
+ *          pair's maxima by 2^32, the sparse kernel skips its running-max
+ *          check (same results, fewer instructions).  Without it every step
+ *          keeps the check.
+ * (ABI 2.0 added layout and workspace.)
  */
+size_t block_sparse_attn_from_indices_workspace_size(int B, int H, int n_q_blocks,
+                                                     int n_kv_blocks);
 int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
                                    const int32_t* q2k_idx, const int32_t* q2k_num,
                                    const int32_t* q_block_sizes, const int32_t* kv_block_sizes,
                                    int B, int H, int Sq_pad, int Skv_pad, int D, int idx_stride,
-                                   float scale, void* out, void* stream);
+                                   float scale, void* out, const vsa_layout* layout,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * block_sparse_attn -- block-sparse attention from a bool block map:
+ * block_map[b, h, a, c] != 0 selects KV block c for query block a.  The map
+ * is converted on the device to ascending index rows, written to q2k_idx
+ * (row width n_kv_blocks, -1 after the selected blocks) and q2k_num, and
+ * those run exactly as in block_sparse_attn_from_indices (so the results are
+ * bit-identical to that call on the same indices).
+ *
+ * Defined by: release 0.3.0, "Block-sparse / VSA attention improvements" and
+ * "New / changed public API": the legacy `block_sparse_attn(..., block_map,
+ * ...)` bool-mask API kept as a wrapper over the index-native kernel.
+ *
+ * block_map  device uint8 (torch.bool) [B, H, n_q_blocks, n_kv_blocks]
+ * q2k_idx    device int32 [B, H, n_q_blocks, n_kv_blocks], written
+ * q2k_num    device int32 [B, H, n_q_blocks], written
+ * everything else as in block_sparse_attn_from_indices (the workspace size
+ * is block_sparse_attn_from_indices_workspace_size's).
+ */
+int block_sparse_attn(const void* q, const void* k, const void* v, const uint8_t* block_map,
+                      const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B, int H,
+                      int Sq_pad, int Skv_pad, int D, float scale, void* out, int32_t* q2k_idx,
+                      int32_t* q2k_num, const vsa_layout* layout, void* workspace,
+                      size_t workspace_bytes, void* stream);
 
 /* ======================================================================== *
  * a6: varlen block-sparse attention

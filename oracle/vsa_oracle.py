@@ -184,6 +184,28 @@ def block_sparse_attention(q, k, v, q2k_idx, q2k_num, q_block_sizes, kv_block_si
     return out
 
 
+def block_map_to_indices(block_map):
+    """Selections of a bool block map as index rows.
+
+    [release] "Block-sparse / VSA attention improvements" and "New / changed
+    public API": the legacy ``block_sparse_attn(..., block_map, ...)`` bool
+    mask is kept as a wrapper over the index-native kernel.  Row
+    ``block_map[..., a, :]`` selects KV block ``c`` where it is True; the
+    index row lists those blocks in ascending order (R3), ``-1`` after them,
+    and the count is the number of True entries.
+
+    block_map: bool [..., nq, nkv]  ->  (q2k_idx int32 [..., nq, nkv],
+    q2k_num int32 [..., nq]).
+    """
+    bm = np.asarray(block_map, dtype=bool)
+    idx = np.full(bm.shape, -1, dtype=np.int32)
+    num = bm.sum(axis=-1).astype(np.int32)
+    for pos in np.ndindex(*bm.shape[:-1]):
+        chosen = np.flatnonzero(bm[pos])
+        idx[pos][:len(chosen)] = chosen
+    return idx, num
+
+
 # ---------------------------------------------------------------------------
 # a5: coarse/sparse combine
 # ---------------------------------------------------------------------------

@@ -496,10 +496,52 @@ def check_page_figures(O):
     assert np.array_equal(out[0, 0, :, 0], np.repeat(np.arange(len(sizes)), g["block"]))
 
 
+def check_block_map_to_indices(O):
+    """Bool block maps to index rows: against a plain per-entry loop on
+    random maps (all-False and all-True rows included), the round trip
+    indices -> map -> indices on a top-k selection, and attention from the
+    map's indices against masked dense attention (torch SDPA, fp64)."""
+    rng = _rng(21)
+    bm = rng.random((2, 3, 5, 37)) < 0.3
+    bm[0, 0, 0] = False
+    bm[1, 2, 4] = True
+    idx, num = O.block_map_to_indices(bm)
+    for pos in np.ndindex(*bm.shape[:-1]):
+        want = [c for c in range(bm.shape[-1]) if bm[pos][c]]
+        assert num[pos] == len(want)
+        assert list(idx[pos][:len(want)]) == want
+        assert np.all(idx[pos][len(want):] == -1)
+    # round trip with a top-k selection
+    scores = rng.standard_normal((1, 2, 6, 11))
+    sel, sn = O.select_topk(scores, 4)
+    back = np.zeros((1, 2, 6, 11), dtype=bool)
+    for b, h, a in np.ndindex(1, 2, 6):
+        back[b, h, a, sel[b, h, a, :sn[b, h, a]]] = True
+    idx2, num2 = O.block_map_to_indices(back)
+    assert np.array_equal(num2, sn) and np.array_equal(idx2[..., :4], sel)
+    # attention through the map equals masked dense attention
+    B, H, D = 1, 2, 16
+    q_sizes, kv_sizes = [64, 40, 64], [64, 9, 64, 64, 30]
+    q = _padded(rng, B, H, q_sizes, D)
+    k = _padded(rng, B, H, kv_sizes, D, pad_value=3.0)
+    v = _padded(rng, B, H, kv_sizes, D, pad_value=3.0)
+    bm = rng.random((B, H, len(q_sizes), len(kv_sizes))) < 0.5
+    bm[..., 0] = True
+    idx, num = O.block_map_to_indices(bm)
+    got = O.block_sparse_attention(q, k, v, idx, num, q_sizes, kv_sizes, 0.25)
+    mask = np.zeros((B, H, BLOCK * len(q_sizes), BLOCK * len(kv_sizes)), dtype=bool)
+    for b, h, a, c in zip(*np.nonzero(bm)):
+        mask[b, h, BLOCK * a:BLOCK * (a + 1), BLOCK * c:BLOCK * c + kv_sizes[c]] = True
+    want = _sdpa(q, k, v, 0.25, mask)
+    qr = _real_rows(q_sizes)
+    assert np.allclose(got[:, :, qr], want[:, :, qr], atol=1e-12)
+
+
 ALL_CHECKS = [
     check_pool_closed_forms, check_coarse_special_cases, check_coarse_vs_library,
     check_topk_brute_force, check_topk_edge_cases, check_sparse_dense_equivalence,
     check_sparse_vs_masked_library, check_sparse_invariants, check_combine,
     check_forward_dense_limit, check_varlen_pack_indices, check_varlen_equals_per_sequence,
     check_varlen_dense_vs_library, check_metadata, check_page_figures,
+    check_block_map_to_indices,
 ]

@@ -60,7 +60,7 @@ def test_status_strings():
     lib = _lib()
     assert lib.vsa_status_string(0) == b"ok"
     assert b"range" in lib.vsa_status_string(6)
-    assert lib.vsa_abi_version() >> 16 == 1
+    assert lib.vsa_abi_version() >> 16 == 2
 
 
 def _fwd(lib, **kw):
@@ -197,3 +197,43 @@ def test_metadata_rejects_bad_tiles():
                                   ctypes.byref(n)) == 1          # tile volume 128 > 64
     assert lib.build_vsa_metadata(0, 4, 4, 4, 4, 4, None, None, None, None, None,
                                   ctypes.byref(n)) == 1
+
+
+def test_layouts_and_strided_argument_checks():
+    """vsa_make_layout fills the documented strides; a view stride that is not
+    a multiple of 8 elements and a missing layout come back as status codes
+    before any CUDA call."""
+    from block_sparse_attention_15_b200.binding import VsaLayout
+    lib = _lib()
+    L = VsaLayout()
+    B, H, Sq, Skv, D = 2, 3, 128, 192, 64
+    assert lib.vsa_make_layout(1, B, H, Sq, Skv, D, ctypes.byref(L)) == 0
+    assert (L.q.batch, L.q.head, L.q.seq) == (Sq * H * D, D, H * D)
+    assert (L.k.batch, L.k.head, L.k.seq) == (Skv * H * D, D, H * D)
+    assert (L.gate.batch, L.gate.head, L.gate.seq) == (Sq * H * D, D, H * D)
+    assert lib.vsa_make_layout(0, B, H, Sq, Skv, D, ctypes.byref(L)) == 0
+    assert (L.out.batch, L.out.head, L.out.seq) == (H * Sq * D, Sq * D, D)
+    assert lib.vsa_make_layout(7, B, H, Sq, Skv, D, ctypes.byref(L)) == 1
+    fake = ctypes.c_void_p(1 << 20)
+
+    def fwd(layout):
+        return lib.vsa_forward_strided(fake, fake, fake, None, layout, None, None, B, H, Sq, Skv, D,
+                                       1, 0.0, fake, fake, fake, 1, None, None, 0, None)
+    assert fwd(None) == 1
+    L.q.seq = 68   # 136 bytes: not a TMA stride
+    assert fwd(ctypes.byref(L)) == 3
+    lib.vsa_make_layout(0, B, H, Sq, Skv, D, ctypes.byref(L))
+    assert fwd(ctypes.byref(L)) == 7   # valid layout: next check is the missing workspace
+
+
+def test_bool_mask_entry_argument_checks():
+    lib = _lib()
+    fake = ctypes.c_void_p(1 << 20)
+
+    def call(bm=fake, idx=fake, num=fake, Sq=128, Skv=128, D=128):
+        return lib.block_sparse_attn(fake, fake, fake, bm, None, None, 1, 1, Sq, Skv, D, 0.0, fake,
+                                     idx, num, None, None, 0, None)
+    assert call(bm=None) == 1
+    assert call(idx=None) == 1
+    assert call(Sq=100) == 2
+    assert call(Skv=64 * 4096) == 3

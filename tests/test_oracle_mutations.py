@@ -13,6 +13,10 @@ ORACLE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))
 
 # (name, exact source fragment, replacement)
 MUTATIONS = [
+    ("block map rows not ascending", "idx[pos][:len(chosen)] = chosen",
+     "idx[pos][:len(chosen)] = chosen[::-1]"),
+    ("block map counts all entries", "num = bm.sum(axis=-1).astype(np.int32)",
+     "num = np.full(bm.shape[:-1], bm.shape[-1], dtype=np.int32)"),
     ("pool divides by 64", "sum(axis=2) / m", "sum(axis=2) / BLOCK"),
     ("pool includes padding", "x[:, :, BLOCK * j:BLOCK * j + m, :].sum(axis=2)",
      "x[:, :, BLOCK * j:BLOCK * j + BLOCK, :].sum(axis=2)"),
