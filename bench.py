@@ -53,6 +53,8 @@ def make_workload(name: str) -> I.Workload:
         return I.workload_tiny()
     if name == "h3":
         return I.workload_h3()
+    if name == "vsa128":
+        return I.workload_vsa128()
     m = re.fullmatch(r"long(\d+)(-ungated)?", name)
     if m:
         return I.workload_long(int(m.group(1)) / 100.0, gated=m.group(2) is None)
@@ -260,9 +262,10 @@ def oracle_sample(wl: I.Workload, q, k, v, gate, head: int, n_items: int):
     vn = v[:, head:head + 1].float().numpy()
     gn = None if gate is None else gate[:, :, head:head + 1].float().numpy()
     items = [(0, 0, a) for a in range(min(n_items, wl.nq))]
-    O.vsa_forward(qn, kn, vn, gn, wl.q_block_sizes, wl.kv_block_sizes, wl.topk, items=items)
+    O.vsa_forward(qn, kn, vn, gn, wl.q_block_sizes, wl.kv_block_sizes, wl.topk, items=items,
+                  block=wl.block)
     dt = time.perf_counter() - t0
-    flops = 4.0 * 64 * 64 * wl.D * min(wl.topk, wl.nkv) * len(items)
+    flops = 4.0 * wl.block * wl.block * wl.D * min(wl.topk, wl.nkv) * len(items)
     return dt, flops
 
 
@@ -286,7 +289,7 @@ def cpu_baseline(wl, q, k, v, gate, budget_s=15.0):
 # inputs
 # ---------------------------------------------------------------------------
 def host_inputs(wl: I.Workload):
-    Sq, Skv = 64 * wl.nq, 64 * wl.nkv
+    Sq, Skv = wl.block * wl.nq, wl.block * wl.nkv
     if "meta" in wl.extra:
         meta = wl.extra["meta"]
         N = int(sum(wl.q_block_sizes))
@@ -300,16 +303,17 @@ def host_inputs(wl: I.Workload):
             padded.append(x)
         q, k, v = padded
     else:
-        q = I.padded_normal_bhsd(wl.B, wl.H, wl.q_block_sizes, wl.D, wl.seed, I.STREAM_Q)
-        k = I.padded_normal_bhsd(wl.B, wl.H, wl.kv_block_sizes, wl.D, wl.seed, I.STREAM_K)
-        v = I.padded_normal_bhsd(wl.B, wl.H, wl.kv_block_sizes, wl.D, wl.seed, I.STREAM_V)
+        q = I.padded_normal_bhsd(wl.B, wl.H, wl.q_block_sizes, wl.D, wl.seed, I.STREAM_Q, block=wl.block)
+        k = I.padded_normal_bhsd(wl.B, wl.H, wl.kv_block_sizes, wl.D, wl.seed, I.STREAM_K, block=wl.block)
+        v = I.padded_normal_bhsd(wl.B, wl.H, wl.kv_block_sizes, wl.D, wl.seed, I.STREAM_V, block=wl.block)
     gate = I.gate_bf16((wl.B, Sq, wl.H, wl.D), wl.seed) if wl.gated else None
     return q, k, v, gate
 
 
 def config_of(wl: I.Workload, flushed: bool) -> dict:
-    return {"workload": wl.name, "B": wl.B, "H": wl.H, "D": wl.D, "seq_q_slots": 64 * wl.nq,
-            "seq_kv_slots": 64 * wl.nkv, "q_blocks": wl.nq, "kv_blocks": wl.nkv,
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "D": wl.D, "block": wl.block,
+            "seq_q_slots": wl.block * wl.nq, "seq_kv_slots": wl.block * wl.nkv,
+            "q_blocks": wl.nq, "kv_blocks": wl.nkv,
             "topk": min(wl.topk, wl.nkv), "gated": wl.gated,
             "selected_tiles_per_gpu": wl.selected_tiles,
             "l2": "L2 flushed between steps" if flushed else
@@ -437,8 +441,8 @@ def run_ours(args, wl):
     flush = None
     if 2 * in_bytes < 2 * L2_BYTES:
         flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
-    qbs = None if all(s == 64 for s in wl.q_block_sizes) else torch.tensor(wl.q_block_sizes, dtype=torch.int32, device=dev)
-    kbs = None if all(s == 64 for s in wl.kv_block_sizes) else torch.tensor(wl.kv_block_sizes, dtype=torch.int32, device=dev)
+    qbs = None if all(s == wl.block for s in wl.q_block_sizes) else torch.tensor(wl.q_block_sizes, dtype=torch.int32, device=dev)
+    kbs = None if all(s == wl.block for s in wl.kv_block_sizes) else torch.tensor(wl.kv_block_sizes, dtype=torch.int32, device=dev)
     k_eff = min(wl.topk, wl.nkv)
     qbs_list = None if qbs is None else list(wl.q_block_sizes)
     kbs_list = None if kbs is None else list(wl.kv_block_sizes)
@@ -450,7 +454,7 @@ def run_ours(args, wl):
     def step():
         if flush is not None:
             flush.fill_(1)
-        vsa.vsa_forward(q, k, v, gate, qbs, kbs, topk=wl.topk, out=out, workspace=ws)
+        vsa.vsa_forward(q, k, v, gate, qbs, kbs, topk=wl.topk, out=out, workspace=ws, block=wl.block)
 
     sampler = ClockSampler(local)  # nvidia-smi starts up during the warm-up
     for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
@@ -496,11 +500,26 @@ def run_ours(args, wl):
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     gh = pin[3] if g_h is not None else None
     host_ws = torch.empty(vsa.lib().vsa_forward_host_workspace_size(
-        wl.B, wl.H, wl.nq, wl.nkv, wl.D, k_eff, 1 if gh is not None else 0, 0), dtype=torch.uint8, device=dev)
+        wl.B, wl.H, wl.nq, wl.nkv, wl.D, k_eff, 1 if gh is not None else 0, 0)
+        if wl.block == 64 else 256, dtype=torch.uint8, device=dev)
 
     def e2e_step():
         vsa.vsa_forward_host(pin[0], pin[1], pin[2], gh, qbs_list, kbs_list, topk=wl.topk, out=out_h,
                              workspace=host_ws, device=dev)
+
+    if wl.block != 64:
+        # the host-buffer entry chunks 64-slot forwards; for other block sizes
+        # the step copies the pinned inputs in, runs the forward and copies
+        # the output back, in sequence on the stream
+        def e2e_step():  # noqa: F811
+            q.copy_(pin[0], non_blocking=True)
+            k.copy_(pin[1], non_blocking=True)
+            v.copy_(pin[2], non_blocking=True)
+            if gh is not None:
+                gate.copy_(gh, non_blocking=True)
+            vsa.vsa_forward(q, k, v, gate, qbs, kbs, topk=wl.topk, out=out, workspace=ws,
+                            block=wl.block)
+            out_h.copy_(out, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize(dev)

@@ -59,7 +59,7 @@ SIGNATURES = {
                     [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p,
                      _c_size_t, _c_void_p]),
     "vsa_make_layout": (_c_int, [_c_int] * 6 + [_PL]),
-    "vsa_forward_strided": (_c_int, [_c_void_p] * 4 + [_PL, _c_void_p, _c_void_p] + [_c_int] * 6 +
+    "vsa_forward_strided": (_c_int, [_c_void_p] * 4 + [_PL, _c_void_p, _c_void_p] + [_c_int] * 7 +
                             [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p,
                              _c_void_p, _c_size_t, _c_void_p]),
     "vsa_forward_bshd": (_c_int, [_c_void_p] * 4 + [_c_void_p, _c_void_p] + [_c_int] * 6 +
@@ -73,10 +73,10 @@ SIGNATURES = {
                          [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_int,
                           _c_void_p, _c_size_t, _c_void_p]),
     "block_sparse_attn_from_indices_workspace_size": (_c_size_t, [_c_int] * 4),
-    "block_sparse_attn_from_indices": (_c_int, [_c_void_p] * 7 + [_c_int] * 6 +
+    "block_sparse_attn_from_indices": (_c_int, [_c_void_p] * 7 + [_c_int] * 7 +
                                        [_c_float, _c_void_p, _PL, _c_void_p, _c_size_t,
                                         _c_void_p]),
-    "block_sparse_attn": (_c_int, [_c_void_p] * 6 + [_c_int] * 5 +
+    "block_sparse_attn": (_c_int, [_c_void_p] * 6 + [_c_int] * 6 +
                           [_c_float, _c_void_p, _c_void_p, _c_void_p, _PL, _c_void_p, _c_size_t,
                            _c_void_p]),
     "block_sparse_attn_varlen_workspace_size": (_c_size_t, [_c_int] * 4),
@@ -200,15 +200,16 @@ def check_device_status(stream=None):
 def vsa_forward(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=None, *, topk: int,
                 scale: float | None = None, idx_stride: int | None = None, out=None,
                 return_out_c: bool = False, return_pooled: bool = False, workspace=None,
-                stream=None):
+                block: int = 64, stream=None):
     """Full VSA forward through ``vsa_forward_strided`` (see include/vsa.h).
 
     q: [B, H, Sq_pad, D] bf16; k, v: [B, H, Skv_pad, D]; gate: [B, Sq_pad, H, D]
     or None.  Any of them may be a strided view (head dim contiguous, other
     strides multiples of 8): a BSHD tensor transposed to [B, H, S, D], a
     slice of a fused QKV tensor.  ``out`` (allocated like q if None) may be a
-    view too.  Returns ``(out, q2k_idx, q2k_num)`` plus ``out_c`` and the
-    pooled (qc, kc, vc) when asked.
+    view too.  ``block``: slots per block, 64 or 128 (VSA-128 tiles; S is then
+    padded to multiples of 128).  Returns ``(out, q2k_idx, q2k_num)`` plus
+    ``out_c`` and the pooled (qc, kc, vc) when asked.
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _require_view(t, n)
@@ -220,7 +221,7 @@ def vsa_forward(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=None, *, 
         _require_view(gate, "gate")
         if gate.shape != (B, Sq, H, D):
             raise ValueError(f"gate must be [B, Sq_pad, H, D] = {(B, Sq, H, D)}, got {tuple(gate.shape)}")
-    nq, nkv = Sq // 64, Skv // 64
+    nq, nkv = Sq // block, Skv // block
     k_eff = min(int(topk), nkv)
     stride = k_eff if idx_stride is None else int(idx_stride)
     dev = q.device
@@ -241,7 +242,7 @@ def vsa_forward(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=None, *, 
     lay = _layout(q, k, v, out, gate)
     _check("vsa_forward_strided", L.vsa_forward_strided(
         _ptr(q), _ptr(k), _ptr(v), _ptr(gate), ctypes.byref(lay), _ptr(qbs), _ptr(kbs), B, H, Sq,
-        Skv, D, int(topk), float(scale) if scale is not None else 0.0, _ptr(out), _ptr(q2k_idx),
+        Skv, D, int(block), int(topk), float(scale) if scale is not None else 0.0, _ptr(out), _ptr(q2k_idx),
         _ptr(q2k_num), stride, _ptr(out_c), _ptr(workspace), workspace.numel(), _stream(stream)))
     res = [out, q2k_idx, q2k_num]
     if return_out_c:
@@ -344,7 +345,7 @@ def _sparse_common(q, k, v, out):
 
 def block_sparse_attn_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes=None,
                                    kv_block_sizes=None, *, scale: float | None = None, out=None,
-                                   logit_bound: bool = True, stream=None):
+                                   logit_bound: bool = True, block: int = 64, stream=None):
     """Block-sparse attention over the listed tiles (``block_sparse_attn_from_indices``).
 
     q, k, v, out: [B, H, S, D] views (see :func:`vsa_forward`).  With
@@ -354,7 +355,7 @@ def block_sparse_attn_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes=None
     B, H, Sq, Skv, D, out = _sparse_common(q, k, v, out)
     _require(q2k_idx, torch.int32, "q2k_idx")
     _require(q2k_num, torch.int32, "q2k_num")
-    nq, nkv = Sq // 64, Skv // 64
+    nq, nkv = Sq // block, Skv // block
     if q2k_idx.dim() != 4 or q2k_idx.shape[:3] != (B, H, nq) or q2k_num.shape != (B, H, nq):
         raise ValueError("q2k_idx must be [B, H, n_q_blocks, stride], q2k_num [B, H, n_q_blocks]")
     dev = q.device
@@ -368,20 +369,20 @@ def block_sparse_attn_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes=None
     lay = _layout(q, k, v, out)
     _check("block_sparse_attn_from_indices", L.block_sparse_attn_from_indices(
         _ptr(q), _ptr(k), _ptr(v), _ptr(q2k_idx), _ptr(q2k_num), _ptr(qbs), _ptr(kbs), B, H, Sq,
-        Skv, D, q2k_idx.shape[3], float(scale) if scale is not None else 0.0, _ptr(out),
+        Skv, D, int(block), q2k_idx.shape[3], float(scale) if scale is not None else 0.0, _ptr(out),
         ctypes.byref(lay), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
     return out
 
 
 def block_sparse_attn(q, k, v, block_map, q_block_sizes=None, kv_block_sizes=None, *,
                       scale: float | None = None, out=None, return_indices: bool = False,
-                      stream=None):
+                      block: int = 64, stream=None):
     """Block-sparse attention from a bool block map [B, H, n_q_blocks,
     n_kv_blocks] (``block_sparse_attn``): converted on the device to index
     rows, then the index-native kernel.  With ``return_indices`` also
     returns the (q2k_idx, q2k_num) it produced."""
     B, H, Sq, Skv, D, out = _sparse_common(q, k, v, out)
-    nq, nkv = Sq // 64, Skv // 64
+    nq, nkv = Sq // block, Skv // block
     if not isinstance(block_map, torch.Tensor) or block_map.dtype != torch.bool:
         raise TypeError("block_map must be a torch.bool tensor")
     if tuple(block_map.shape) != (B, H, nq, nkv) or not block_map.is_cuda or not block_map.is_contiguous():
@@ -398,14 +399,15 @@ def block_sparse_attn(q, k, v, block_map, q_block_sizes=None, kv_block_sizes=Non
     lay = _layout(q, k, v, out)
     _check("block_sparse_attn", L.block_sparse_attn(
         _ptr(q), _ptr(k), _ptr(v), _ptr(block_map), _ptr(qbs), _ptr(kbs), B, H, Sq, Skv, D,
-        float(scale) if scale is not None else 0.0, _ptr(out), _ptr(q2k_idx), _ptr(q2k_num),
+        int(block), float(scale) if scale is not None else 0.0, _ptr(out), _ptr(q2k_idx), _ptr(q2k_num),
         ctypes.byref(lay), _ptr(ws), ws.numel(), _stream(stream)))
     return (out, q2k_idx, q2k_num) if return_indices else out
 
 
 def video_sparse_attn_bshd(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=None, *,
                            topk: int, scale: float | None = None, idx_stride: int | None = None,
-                           out=None, return_out_c: bool = False, workspace=None, stream=None):
+                           out=None, return_out_c: bool = False, workspace=None, block: int = 64,
+                           stream=None):
     """The whole VSA forward on BSHD tensors: q [B, Sq_pad, H, D], k and v
     [B, Skv_pad, H, D], gate [B, Sq_pad, H, D]; the output is BSHD too.  The
     library reads and writes the BSHD memory in place (strided views, no
@@ -415,7 +417,7 @@ def video_sparse_attn_bshd(q, k, v, gate=None, q_block_sizes=None, kv_block_size
     res = vsa_forward(q.transpose(1, 2), k.transpose(1, 2), v.transpose(1, 2), gate,
                       q_block_sizes, kv_block_sizes, topk=topk, scale=scale, idx_stride=idx_stride,
                       out=None if out is None else out.transpose(1, 2), return_out_c=return_out_c,
-                      workspace=workspace, stream=stream)
+                      workspace=workspace, block=block, stream=stream)
     return (out,) + tuple(res[1:])
 
 
@@ -534,9 +536,9 @@ def selftest_umma(mode: int, a, b, *, stream=None):
     """Run one tensor-core product of the sparse kernel on global operands."""
     _require(a, torch.bfloat16, "a")
     _require(b, torch.bfloat16, "b")
-    D = a.shape[1]
-    rows = 128 if mode == 0 else D
-    c = torch.empty((rows, 64), dtype=torch.float32, device=a.device)
+    D = b.shape[1] if mode >= 2 else a.shape[1]
+    shape = {0: (128, 64), 1: (D, 64), 2: (128, 128), 3: (128, D)}[mode]
+    c = torch.empty(shape, dtype=torch.float32, device=a.device)
     _check("vsa_selftest_umma", lib().vsa_selftest_umma(mode, D, _ptr(a), _ptr(b), _ptr(c),
                                                         _stream(stream)))
     return c

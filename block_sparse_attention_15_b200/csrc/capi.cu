@@ -99,8 +99,9 @@ int check_forward_args(const ForwardArgs& a) {
   if (a.B <= 0 || a.H <= 0 || a.Sq_pad <= 0 || a.Skv_pad <= 0 || a.topk < 1 || !(a.scale == a.scale))
     return VSA_ERR_INVALID_ARG;
   if (a.D != 64 && a.D != 128) return VSA_ERR_UNSUPPORTED;
-  if (a.Sq_pad % 64 || a.Skv_pad % 64) return VSA_ERR_SHAPE;
-  const int nq = a.Sq_pad / 64, nkv = a.Skv_pad / 64;
+  if (a.block != 64 && a.block != 128) return VSA_ERR_UNSUPPORTED;
+  if (a.Sq_pad % a.block || a.Skv_pad % a.block) return VSA_ERR_SHAPE;
+  const int nq = a.Sq_pad / a.block, nkv = a.Skv_pad / a.block;
   if (nq > VSA_MAX_BLOCKS || nkv > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
   const int k_eff = a.topk < nkv ? a.topk : nkv;
   if (a.idx_stride < k_eff) return VSA_ERR_SHAPE;
@@ -120,7 +121,10 @@ int check_forward_args(const ForwardArgs& a) {
 // kernel that produces it before any kernel reads it.
 int launch_forward(const ForwardArgs& a, void* scratch, bool profile, cudaStream_t st) {
   const int B = a.B, H = a.H, D = a.D;
-  const int nq = a.Sq_pad / 64, nkv = a.Skv_pad / 64;
+  const int nq = a.Sq_pad / a.block, nkv = a.Skv_pad / a.block;
+  // the logit bound serves the 64-slot kernel's vote-free step; the 128-slot
+  // kernel keeps its row maxima in-thread and needs none
+  const bool bound = a.block == 64;
   const int k_eff = a.topk < nkv ? a.topk : nkv;
   int* status = device_status_ptr();
   if (!status) return VSA_ERR_CUDA;
@@ -153,13 +157,14 @@ int launch_forward(const ForwardArgs& a, void* scratch, bool profile, cudaStream
   pp.kv_bs = a.kv_block_sizes;
   pp.groups = B * H;
   pp.H = H;
+  pp.block = a.block;
   pp.nq = nq;
   pp.nkv = nkv;
   pp.qc = qc;
   pp.kc = kc;
   pp.vc = vc;
-  pp.qn = qn;
-  pp.kn = kn;
+  pp.qn = bound ? qn : nullptr;
+  pp.kn = bound ? kn : nullptr;
   pp.status = status;
   if (prof) cudaEventRecord(g_prof_events[0], st);
   int rc = launch_pool(pp, D, st);
@@ -182,7 +187,7 @@ int launch_forward(const ForwardArgs& a, void* scratch, bool profile, cudaStream
   cp.out_c = oc;
   cp.qn = qn;
   cp.kn = kn;
-  cp.qk_bound = qk_bound;
+  cp.qk_bound = bound ? qk_bound : nullptr;
   cp.bound_scale = sc * kLog2e * (1.f + 0x1p-8f);
   cp.status = status;
   rc = launch_coarse_topk(cp, D, st);
@@ -206,11 +211,14 @@ int launch_forward(const ForwardArgs& a, void* scratch, bool profile, cudaStream
   sp.nq = nq;
   sp.nkv = nkv;
   sp.scale_log2 = sc * kLog2e;
-  sp.qk_bound = qk_bound;
+  sp.qk_bound = bound ? qk_bound : nullptr;
   sp.varlen = 0;
   sp.status = status;
-  rc = launch_sparse(sp, a.q, a.q_st, a.Sq_pad, a.k, a.k_st, a.v, a.v_st, a.Skv_pad, D,
-                     /*combine=*/true, /*gated=*/a.gate != nullptr, st);
+  rc = a.block == 128
+           ? launch_sparse128(sp, a.q, a.q_st, a.Sq_pad, a.k, a.k_st, a.v, a.v_st, a.Skv_pad, D,
+                              /*combine=*/true, /*gated=*/a.gate != nullptr, st)
+           : launch_sparse(sp, a.q, a.q_st, a.Sq_pad, a.k, a.k_st, a.v, a.v_st, a.Skv_pad, D,
+                           /*combine=*/true, /*gated=*/a.gate != nullptr, st);
   if (rc != VSA_OK) return rc;
   if (prof) cudaEventRecord(g_prof_events[3], st);
   return VSA_OK;
@@ -268,11 +276,12 @@ int vsa_make_layout(int kind, int B, int H, int Sq_pad, int Skv_pad, int D, vsa_
 int vsa_forward_strided(const void* q, const void* k, const void* v, const void* gate,
                         const vsa_layout* layout, const int32_t* q_block_sizes,
                         const int32_t* kv_block_sizes, int B, int H, int Sq_pad, int Skv_pad,
-                        int D, int topk, float scale, void* out, int32_t* q2k_idx,
+                        int D, int block_size, int topk, float scale, void* out, int32_t* q2k_idx,
                         int32_t* q2k_num, int idx_stride, float* out_c, void* workspace,
                         size_t workspace_bytes, void* stream) {
   if (!layout) return VSA_ERR_INVALID_ARG;
   ForwardArgs a;
+  a.block = block_size;
   a.q = q; a.k = k; a.v = v; a.gate = gate;
   a.q_st = to_strides(layout->q); a.k_st = to_strides(layout->k); a.v_st = to_strides(layout->v);
   a.out_st = to_strides(layout->out); a.gate_st = to_strides(layout->gate);
@@ -282,7 +291,7 @@ int vsa_forward_strided(const void* q, const void* k, const void* v, const void*
   a.idx_stride = idx_stride; a.out_c = out_c;
   int rc = check_forward_args(a);
   if (rc != VSA_OK) return rc;
-  const size_t need = vsa_forward_workspace_size(B, H, Sq_pad / 64, Skv_pad / 64, D);
+  const size_t need = vsa_forward_workspace_size(B, H, Sq_pad / block_size, Skv_pad / block_size, D);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return VSA_ERR_WORKSPACE;
   return launch_forward(a, workspace, /*profile=*/true, static_cast<cudaStream_t>(stream));
@@ -297,7 +306,7 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
   vsa_layout L;
   fill_layout(VSA_LAYOUT_BHSD, B, H, Sq_pad, Skv_pad, D, &L);
   return vsa_forward_strided(q, k, v, gate, &L, q_block_sizes, kv_block_sizes, B, H, Sq_pad,
-                             Skv_pad, D, topk, scale, out, q2k_idx, q2k_num, idx_stride, out_c,
+                             Skv_pad, D, 64, topk, scale, out, q2k_idx, q2k_num, idx_stride, out_c,
                              workspace, workspace_bytes, stream);
 }
 
@@ -310,7 +319,7 @@ int vsa_forward_bshd(const void* q, const void* k, const void* v, const void* ga
   vsa_layout L;
   fill_layout(VSA_LAYOUT_BSHD, B, H, Sq_pad, Skv_pad, D, &L);
   return vsa_forward_strided(q, k, v, gate, &L, q_block_sizes, kv_block_sizes, B, H, Sq_pad,
-                             Skv_pad, D, topk, scale, out, q2k_idx, q2k_num, idx_stride, out_c,
+                             Skv_pad, D, 64, topk, scale, out, q2k_idx, q2k_num, idx_stride, out_c,
                              workspace, workspace_bytes, stream);
 }
 
@@ -328,15 +337,16 @@ size_t block_sparse_attn_from_indices_workspace_size(int B, int H, int n_q_block
 static int sparse_from_indices(const void* q, const void* k, const void* v,
                                const int32_t* q2k_idx, const int32_t* q2k_num,
                                const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B,
-                               int H, int Sq_pad, int Skv_pad, int D, int idx_stride, float scale,
-                               void* out, const vsa_layout* layout, void* workspace,
+                               int H, int Sq_pad, int Skv_pad, int D, int block, int idx_stride,
+                               float scale, void* out, const vsa_layout* layout, void* workspace,
                                size_t workspace_bytes, cudaStream_t st) {
   if (!q || !k || !v || !out || !q2k_idx || !q2k_num) return VSA_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || idx_stride < 1 || !(scale == scale))
     return VSA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
-  if (Sq_pad % 64 || Skv_pad % 64) return VSA_ERR_SHAPE;
-  const int nq = Sq_pad / 64, nkv = Skv_pad / 64;
+  if (block != 64 && block != 128) return VSA_ERR_UNSUPPORTED;
+  if (Sq_pad % block || Skv_pad % block) return VSA_ERR_SHAPE;
+  const int nq = Sq_pad / block, nkv = Skv_pad / block;
   if (idx_stride > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return VSA_ERR_INVALID_ARG;
   vsa_layout L;
@@ -352,7 +362,7 @@ static int sparse_from_indices(const void* q, const void* k, const void* v,
   if (!status) return VSA_ERR_CUDA;
   const float sc = resolve_scale(scale, D);
   const float* qk_bound = nullptr;
-  if (workspace) {
+  if (workspace && block == 64) {
     // logit bound of every item from block row norms and its selection
     BoundParams bp;
     memset(&bp, 0, sizeof(bp));
@@ -394,6 +404,9 @@ static int sparse_from_indices(const void* q, const void* k, const void* v,
   sp.scale_log2 = sc * kLog2e;
   sp.qk_bound = qk_bound;
   sp.status = status;
+  if (block == 128)
+    return launch_sparse128(sp, q, to_strides(L.q), Sq_pad, k, to_strides(L.k), v, to_strides(L.v),
+                            Skv_pad, D, false, false, st);
   return launch_sparse(sp, q, to_strides(L.q), Sq_pad, k, to_strides(L.k), v, to_strides(L.v),
                        Skv_pad, D, false, false, st);
 }
@@ -401,12 +414,13 @@ static int sparse_from_indices(const void* q, const void* k, const void* v,
 int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
                                    const int32_t* q2k_idx, const int32_t* q2k_num,
                                    const int32_t* q_block_sizes, const int32_t* kv_block_sizes,
-                                   int B, int H, int Sq_pad, int Skv_pad, int D, int idx_stride,
-                                   float scale, void* out, const vsa_layout* layout,
-                                   void* workspace, size_t workspace_bytes, void* stream) {
+                                   int B, int H, int Sq_pad, int Skv_pad, int D, int block_size,
+                                   int idx_stride, float scale, void* out,
+                                   const vsa_layout* layout, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
   return sparse_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes, kv_block_sizes, B, H,
-                             Sq_pad, Skv_pad, D, idx_stride, scale, out, layout, workspace,
-                             workspace_bytes, static_cast<cudaStream_t>(stream));
+                             Sq_pad, Skv_pad, D, block_size, idx_stride, scale, out, layout,
+                             workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------
@@ -414,19 +428,20 @@ int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
 // ---------------------------------------------------------------------------
 int block_sparse_attn(const void* q, const void* k, const void* v, const uint8_t* block_map,
                       const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B, int H,
-                      int Sq_pad, int Skv_pad, int D, float scale, void* out, int32_t* q2k_idx,
-                      int32_t* q2k_num, const vsa_layout* layout, void* workspace,
-                      size_t workspace_bytes, void* stream) {
+                      int Sq_pad, int Skv_pad, int D, int block_size, float scale, void* out,
+                      int32_t* q2k_idx, int32_t* q2k_num, const vsa_layout* layout,
+                      void* workspace, size_t workspace_bytes, void* stream) {
   if (!block_map || !q2k_idx || !q2k_num) return VSA_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0) return VSA_ERR_INVALID_ARG;
-  if (Sq_pad % 64 || Skv_pad % 64) return VSA_ERR_SHAPE;
-  const int nq = Sq_pad / 64, nkv = Skv_pad / 64;
+  if (block_size != 64 && block_size != 128) return VSA_ERR_UNSUPPORTED;
+  if (Sq_pad % block_size || Skv_pad % block_size) return VSA_ERR_SHAPE;
+  const int nq = Sq_pad / block_size, nkv = Skv_pad / block_size;
   if (nkv > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int rc = launch_mask_to_indices(block_map, (long long)B * H * nq, nkv, q2k_idx, q2k_num, st);
   if (rc != VSA_OK) return rc;
   return sparse_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes, kv_block_sizes, B, H,
-                             Sq_pad, Skv_pad, D, nkv, scale, out, layout, workspace,
+                             Sq_pad, Skv_pad, D, block_size, nkv, scale, out, layout, workspace,
                              workspace_bytes, st);
 }
 
@@ -605,7 +620,7 @@ int build_vsa_metadata(int T, int Hh, int W, int tT, int tH, int tW,
                        int64_t* slot_token, int32_t* n_tiles) {
   if (T <= 0 || Hh <= 0 || W <= 0 || tT <= 0 || tH <= 0 || tW <= 0) return VSA_ERR_INVALID_ARG;
   const int vol = tT * tH * tW;
-  if (vol > 64) return VSA_ERR_INVALID_ARG;
+  if (vol > 128) return VSA_ERR_INVALID_ARG;
   const int nT = (T + tT - 1) / tT, nH = (Hh + tH - 1) / tH, nW = (W + tW - 1) / tW;
   const long long ntiles = (long long)nT * nH * nW;
   if (ntiles > 0x7FFFFFFFLL) return VSA_ERR_UNSUPPORTED;
@@ -683,8 +698,9 @@ int vsa_selftest_exp2(const float* x, float* y, int64_t n, int* mismatch, void* 
 }
 
 int vsa_selftest_umma(int mode, int D, const void* a, const void* b, float* c, void* stream) {
-  if (!a || !b || !c || (mode != 0 && mode != 1)) return VSA_ERR_INVALID_ARG;
+  if (!a || !b || !c || mode < 0 || mode > 3) return VSA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
+  if (mode >= 2) return launch_selftest128(mode, D, a, b, c, static_cast<cudaStream_t>(stream));
   return launch_selftest_umma(mode, D, a, b, c, static_cast<cudaStream_t>(stream));
 }
 

@@ -56,6 +56,7 @@ extern "C" int vsa_forward_noalloc(const void* q, const void* k, const void* v, 
                                    float scale, void* out, int32_t* q2k_idx, int32_t* q2k_num,
                                    int idx_stride, float* out_c, void* stream) {
   ForwardArgs a;
+  a.block = 64;
   a.q = q; a.k = k; a.v = v; a.gate = gate;
   a.q_st = a.out_st = bhsd_strides(H, Sq_pad, D);
   a.k_st = a.v_st = bhsd_strides(H, Skv_pad, D);

@@ -23,13 +23,14 @@
 namespace vsa {
 
 // ---------------------------------------------------------------------------
-// a1: pooling.  One CTA of 256 threads per (tensor, batch*head, block).
+// a1: pooling.  One CTA of 256 threads per (tensor, batch*head, block) of
+// BS slots (64 or 128).
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, int BS>
 __global__ void __launch_bounds__(256, 8) pool_kernel(PoolParams p) {
   constexpr int CPR = D / 8;          // 16-byte chunks per row
   constexpr int RPP = 256 / CPR;      // rows per pass
-  constexpr int PASSES = 64 / RPP;
+  constexpr int PASSES = BS / RPP;
   __shared__ float red[RPP][D + 1];
   __shared__ float wmax[8];
 
@@ -56,25 +57,32 @@ __global__ void __launch_bounds__(256, 8) pool_kernel(PoolParams p) {
   const int group = item / nblocks;
   const int blk = item - group * nblocks;
   const int b = group / p.H, h = group - b * p.H;
-  int m = bs ? bs[blk] : 64;
-  if (m < 1 || m > 64) {
+  int m = bs ? bs[blk] : BS;
+  if (m < 1 || m > BS) {
     if (threadIdx.x == 0) set_status(p.status, VSA_ERR_BLOCK_SIZE);
-    m = m < 1 ? 1 : 64;
+    m = m < 1 ? 1 : BS;
   }
-  const int lim = (nrm && all_rows) ? 64 : m;  // rows read
-  // first slot of the block in the strided view (item = group*nblocks + blk)
-  const __nv_bfloat16* base = src + b * st.b + h * st.h + 64LL * blk * st.s;
+  const int lim = (nrm && all_rows) ? BS : m;  // rows read
   const int chunk = threadIdx.x % CPR;
   const int r0 = threadIdx.x / CPR;
 
   uint4 buf[PASSES];
+  if (st.s == D && st.h == (long long)nblocks * BS * D && st.b == st.h * p.H) {
+    // contiguous [B, H, S, D]: the block is BS consecutive rows
+    const uint4* base = reinterpret_cast<const uint4*>(src) + (long long)item * BS * CPR + chunk;
 #pragma unroll
-  for (int ps = 0; ps < PASSES; ++ps) {
-    const int row = r0 + ps * RPP;
-    if (row < lim) {
-      buf[ps] = __ldcs(reinterpret_cast<const uint4*>(base + (long long)row * st.s) + chunk);
-    } else {
-      buf[ps] = make_uint4(0u, 0u, 0u, 0u);
+    for (int ps = 0; ps < PASSES; ++ps) {
+      const int row = r0 + ps * RPP;
+      buf[ps] = row < lim ? __ldcs(base + row * CPR) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  } else {
+    // first slot of the block in the strided view (item = group*nblocks + blk)
+    const __nv_bfloat16* base = src + b * st.b + h * st.h + (long long)BS * blk * st.s;
+#pragma unroll
+    for (int ps = 0; ps < PASSES; ++ps) {
+      const int row = r0 + ps * RPP;
+      buf[ps] = row < lim ? __ldcs(reinterpret_cast<const uint4*>(base + (long long)row * st.s) + chunk)
+                          : make_uint4(0u, 0u, 0u, 0u);
     }
   }
   // block sums over the real rows and, per pass, this chunk's part of the
@@ -418,8 +426,13 @@ int launch_pool(const PoolParams& p, int D, cudaStream_t stream) {
   const long long items = (long long)p.groups * (p.nq + 2LL * p.nkv);
   if (items <= 0) return VSA_OK;
   if (items > 0x7FFFFFFFLL) return VSA_ERR_UNSUPPORTED;
-  if (D == 128) pool_kernel<128><<<(unsigned)items, 256, 0, stream>>>(p);
-  else pool_kernel<64><<<(unsigned)items, 256, 0, stream>>>(p);
+  if (p.block == 128) {
+    if (D == 128) pool_kernel<128, 128><<<(unsigned)items, 256, 0, stream>>>(p);
+    else pool_kernel<64, 128><<<(unsigned)items, 256, 0, stream>>>(p);
+  } else {
+    if (D == 128) pool_kernel<128, 64><<<(unsigned)items, 256, 0, stream>>>(p);
+    else pool_kernel<64, 64><<<(unsigned)items, 256, 0, stream>>>(p);
+  }
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 

@@ -1000,11 +1000,11 @@ EncodeTiledFn get_encode_fn() {
 // 4-D map of a strided [B, H, S, D] bf16 view: dimension 0 is the head dim,
 // dimensions 1..3 the sequence, head and batch axes in increasing stride
 // order (an axis of extent 1 goes last, with the stride an outer contiguous
-// axis would have); 64 x 1 x 64 x 1 boxes (64 head dims of 64 slots of one
-// head and batch), 128-byte swizzle.  The caller checked that every stride
+// axis would have); boxes of 64 head dims x box_rows slots of one head and
+// batch, 128-byte swizzle.  The caller checked that every stride
 // is a multiple of 8 elements (16 bytes) and the base 16-byte aligned.
-static bool make_view_map(CUtensorMap* map, TmaAxes* ax, const void* base, int D, long long S,
-                          int H, int B, Strides3 st) {
+bool make_view_map_rows(CUtensorMap* map, TmaAxes* ax, const void* base, int D, long long S,
+                        int H, int B, Strides3 st, int box_rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   struct A { int id; long long ext, str; } a[3] = {{0, S, st.s}, {1, H, st.h}, {2, B, st.b}};
@@ -1029,7 +1029,7 @@ static bool make_view_map(CUtensorMap* map, TmaAxes* ax, const void* base, int D
     else ax->b = slot;
   }
   cuuint32_t box[4] = {64, 1, 1, 1};
-  box[ax->s] = 64;
+  box[ax->s] = (cuuint32_t)box_rows;
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1070,6 +1070,11 @@ static int launch_sparse_t(const SparseParams& p, const CUtensorMap& mq, const C
   const long long grid = n_items < sm_count() ? n_items : sm_count();
   kern<<<(unsigned)grid, kThreads, L::kAlloc, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+static bool make_view_map(CUtensorMap* map, TmaAxes* ax, const void* base, int D, long long S,
+                          int H, int B, Strides3 st) {
+  return make_view_map_rows(map, ax, base, D, S, H, B, st, 64);
 }
 
 int launch_sparse(const SparseParams& p_in, const void* q, Strides3 q_st, long long q_seq,

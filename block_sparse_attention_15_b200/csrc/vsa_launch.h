@@ -31,6 +31,7 @@ struct PoolParams {
   const int32_t* kv_bs;  // [nkv] or null
   int groups;            // B * H
   int H;
+  int block;             // slots per block: 64 or 128
   int nq, nkv;
   float* qc;             // [groups, nq, D]
   float* kc;             // [groups, nkv, D]
@@ -98,6 +99,17 @@ int launch_sparse(const SparseParams& p, const void* q, Strides3 q_st, long long
                   int D, bool combine, bool gated, cudaStream_t stream);
 int launch_selftest_umma(int mode, int D, const void* a, const void* b, float* c,
                          cudaStream_t stream);
+// The 128-token block path (sparse128_fwd.cu): same parameters, blocks of
+// 128 slots, no varlen tables.
+int launch_sparse128(const SparseParams& p, const void* q, Strides3 q_st, long long q_seq,
+                     const void* k, Strides3 k_st, const void* v, Strides3 v_st, long long kv_seq,
+                     int D, bool combine, bool gated, cudaStream_t stream);
+int launch_selftest128(int mode, int D, const void* a, const void* b, float* c,
+                       cudaStream_t stream);
+// 4-D tile map of a strided [B, H, S, D] bf16 view with boxes of 64 head
+// dims x box_rows slots (sparse_fwd.cu).
+bool make_view_map_rows(CUtensorMap* map, TmaAxes* ax, const void* base, int D, long long S,
+                        int H, int B, Strides3 st, int box_rows);
 int launch_selftest_exp2(const float* x, float* y, long long n, int* mismatch,
                          cudaStream_t stream);
 
@@ -165,6 +177,7 @@ struct ForwardArgs {
   const int32_t* q_block_sizes;
   const int32_t* kv_block_sizes;
   int B, H, Sq_pad, Skv_pad, D, topk;
+  int block;  // slots per block: 64 or 128
   float scale;
   void* out;
   int32_t* q2k_idx;

@@ -68,29 +68,30 @@ def topk_count(frac: float, n_kv_blocks: int) -> int:
 
 
 def pad_tokens_bhsd(x_tokens: torch.Tensor, block_sizes: list[int],
-                    pad_value: float = 0.0) -> torch.Tensor:
+                    pad_value: float = 0.0, block: int = BLOCK) -> torch.Tensor:
     """Place contiguous tokens ``[B, H, N, D]`` into the padded layout.
 
     Block ``j`` takes the next ``block_sizes[j]`` tokens in order and occupies
-    slots ``64*j .. 64*j + block_sizes[j] - 1``; the rest of its slots hold
-    ``pad_value``.  Returns ``[B, H, 64*len(block_sizes), D]``.
+    slots ``block*j .. block*j + block_sizes[j] - 1``; the rest of its slots
+    hold ``pad_value``.  Returns ``[B, H, block*len(block_sizes), D]``.
     """
     B, H, N, D = x_tokens.shape
     assert sum(block_sizes) == N
-    out = torch.full((B, H, BLOCK * len(block_sizes), D), pad_value, dtype=x_tokens.dtype)
+    out = torch.full((B, H, block * len(block_sizes), D), pad_value, dtype=x_tokens.dtype)
     src = 0
     for j, n in enumerate(block_sizes):
-        out[:, :, BLOCK * j:BLOCK * j + n] = x_tokens[:, :, src:src + n]
+        out[:, :, block * j:block * j + n] = x_tokens[:, :, src:src + n]
         src += n
     return out
 
 
 def padded_normal_bhsd(B: int, H: int, block_sizes: list[int], D: int, seed: int,
-                       stream: int, pad_value: float = 0.0, scale: float = 1.0) -> torch.Tensor:
-    """N(0,1) bf16 activations directly in the padded ``[B, H, 64*n, D]`` layout."""
+                       stream: int, pad_value: float = 0.0, scale: float = 1.0,
+                       block: int = BLOCK) -> torch.Tensor:
+    """N(0,1) bf16 activations directly in the padded ``[B, H, block*n, D]`` layout."""
     n_tok = sum(block_sizes)
     x = normal_bf16((B, H, n_tok, D), seed, stream, scale=scale)
-    return pad_tokens_bhsd(x, block_sizes, pad_value)
+    return pad_tokens_bhsd(x, block_sizes, pad_value, block)
 
 
 @dataclass
@@ -106,6 +107,7 @@ class Workload:
     gated: bool = True
     seed: int = 1000
     extra: dict = field(default_factory=dict)
+    block: int = BLOCK  # slots per block: 64, or 128 for VSA-128 tiles
 
     @property
     def nq(self) -> int:
@@ -121,8 +123,9 @@ class Workload:
 
     @property
     def flops(self) -> float:
-        """Algorithmic FLOPs of the selected 64x64 tiles: 4 * 64 * 64 * D each."""
-        return 4.0 * BLOCK * BLOCK * self.D * self.selected_tiles
+        """Algorithmic FLOPs of the selected tiles: 4 * block * block * D each
+        (QK^T and PV of a block x block tile)."""
+        return 4.0 * self.block * self.block * self.D * self.selected_tiles
 
 
 def workload_tiny() -> Workload:
@@ -144,6 +147,14 @@ def workload_long(frac: float, gated: bool = True) -> Workload:
     k = topk_count(frac, nb)
     return Workload(f"long: B1 H40 D128 S32768 top{k} ({frac:.0%}) {'gated' if gated else 'ungated'}",
                     1, 40, 128, [64] * nb, [64] * nb, k, gated, 1005)
+
+
+def workload_vsa128() -> Workload:
+    """The README's VSA-128 benchmark shape: B=1, H=12, D=128, 39936 tokens
+    in 312 blocks of 128 (128-token video tiles), top 40, gated."""
+    nb = 39936 // 128
+    return Workload("VSA-128: B1 H12 D128 S39936 (312 blocks of 128) top40 gated", 1, 12, 128,
+                    [128] * nb, [128] * nb, 40, True, 1006, block=128)
 
 
 VARLEN_Q_LENS = (3000, 6144, 9216, 15488)

@@ -166,23 +166,32 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * vsa_forward_strided -- vsa_forward on strided views: q, k, v, out and gate
- * are read and written through the strides in `layout` (host pointer), so
- * BSHD tensors, slices of a fused QKV tensor and a transposed gate view need
- * no copy.  Same results as vsa_forward on the same values.
+ * vsa_forward_strided -- vsa_forward on strided views and either block size:
+ * q, k, v, out and gate are read and written through the strides in `layout`
+ * (host pointer), so BSHD tensors, slices of a fused QKV tensor and a
+ * transposed gate view need no copy.  Same results as vsa_forward on the
+ * same values at block_size 64.
+ *
+ * block_size  slots per block, 64 or 128.  With 128 ("VSA-128": 128-token
+ *          video tiles), Sq_pad and Skv_pad are multiples of 128, block
+ *          sizes lie in [1, 128], pooling and the coarse stage work on
+ *          128-slot blocks and the sparse stage attends over 128 x 128
+ *          tiles (a kernel shaped for the tensor core's native 128 rows).
  *
  * Defined by: release 0.3.0, "Block-sparse / VSA attention improvements"
- * (the BSHD-native `video_sparse_attn_bshd` entry, the "skip the bool-mask
- * round-trip" item) and PR #1813's follow-up (the gate passed as a
+ * (the BSHD-native `video_sparse_attn_bshd` entry and the 128/256-token tile
+ * fastpath) and the README's kernel inventory (Blackwell forward kernels for
+ * 64- and 128-token blocks); PR #1813's follow-up (the gate passed as a
  * transposed view of its [B, S, H, D] memory).  All other arguments as in
- * vsa_forward; the workspace is the same size.
+ * vsa_forward with n_q_blocks = Sq_pad / block_size; the workspace size is
+ * vsa_forward_workspace_size(B, H, n_q_blocks, n_kv_blocks, D).
  */
 int vsa_forward_strided(const void* q, const void* k, const void* v, const void* gate,
                         const vsa_layout* layout, const int32_t* q_block_sizes,
                         const int32_t* kv_block_sizes, int B, int H, int Sq_pad, int Skv_pad,
-                        int D, int topk, float scale, void* out, int32_t* q2k_idx,
-                        int32_t* q2k_num, int idx_stride, float* out_c, void* workspace,
-                        size_t workspace_bytes, void* stream);
+                        int D, int block_size, int topk, float scale, void* out,
+                        int32_t* q2k_idx, int32_t* q2k_num, int idx_stride, float* out_c,
+                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * vsa_forward_bshd -- vsa_forward with q, k, v and out contiguous
@@ -296,16 +305,20 @@ int vsa_forward_host(const void* q, const void* k, const void* v, const void* ga
  *          pair's maxima by 2^32, the sparse kernel skips its running-max
  *          check (same results, fewer instructions).  Without it every step
  *          keeps the check.
- * (ABI 2.0 added layout and workspace.)
+ *          (Block size 64 only; at 128 the workspace is not used.)
+ * block_size  64 or 128 (see vsa_forward_strided); n_q_blocks = Sq_pad /
+ *          block_size
+ * (ABI 2.0 added layout, block_size and workspace.)
  */
 size_t block_sparse_attn_from_indices_workspace_size(int B, int H, int n_q_blocks,
                                                      int n_kv_blocks);
 int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
                                    const int32_t* q2k_idx, const int32_t* q2k_num,
                                    const int32_t* q_block_sizes, const int32_t* kv_block_sizes,
-                                   int B, int H, int Sq_pad, int Skv_pad, int D, int idx_stride,
-                                   float scale, void* out, const vsa_layout* layout,
-                                   void* workspace, size_t workspace_bytes, void* stream);
+                                   int B, int H, int Sq_pad, int Skv_pad, int D, int block_size,
+                                   int idx_stride, float scale, void* out,
+                                   const vsa_layout* layout, void* workspace,
+                                   size_t workspace_bytes, void* stream);
 
 /*
  * block_sparse_attn -- block-sparse attention from a bool block map:
@@ -327,9 +340,9 @@ int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
  */
 int block_sparse_attn(const void* q, const void* k, const void* v, const uint8_t* block_map,
                       const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B, int H,
-                      int Sq_pad, int Skv_pad, int D, float scale, void* out, int32_t* q2k_idx,
-                      int32_t* q2k_num, const vsa_layout* layout, void* workspace,
-                      size_t workspace_bytes, void* stream);
+                      int Sq_pad, int Skv_pad, int D, int block_size, float scale, void* out,
+                      int32_t* q2k_idx, int32_t* q2k_num, const vsa_layout* layout,
+                      void* workspace, size_t workspace_bytes, void* stream);
 
 /* ======================================================================== *
  * a6: varlen block-sparse attention
@@ -416,7 +429,7 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
  *                                 each padded slot, -1 for padding
  * n_tiles                         int32 [1]
  * Returns VSA_ERR_INVALID_ARG for non-positive sizes or a tile volume above
- * 64.
+ * 128 (64 for the 64-slot path, 128 for VSA-128 tiles such as 4 x 4 x 8).
  */
 int build_vsa_metadata(int T, int Hh, int W, int tT, int tH, int tW,
                        int64_t* tile_partition_indices, int64_t* reverse_tile_partition_indices,
@@ -458,11 +471,14 @@ int vsa_scatter_tokens(const void* src, void* dst, const int64_t* slot_token, in
 int vsa_set_profile_events(void* const* events);
 
 /*
- * vsa_selftest_umma -- run the two tensor-core products of the sparse kernel
- * once on operands in global memory, to check shared-memory layouts in
- * isolation.  mode 0: c[128][64] = a[128][D] * b[64][D]^T (fp32), the
- * transposed-score product; mode 1: c[D][64] = a[128][D]^T * b[128][64], the
- * transposed-output product.  a, b device bf16; c device fp32.  D 64 or 128.
+ * vsa_selftest_umma -- run the tensor-core products of the sparse kernels
+ * once on operands in global memory, to check shared-memory and TMEM
+ * layouts in isolation.  64-slot kernel: mode 0: c[128][64] = a[128][D] *
+ * b[64][D]^T (fp32), the transposed-score product; mode 1: c[D][64] =
+ * a[128][D]^T * b[128][64], the transposed-output product.  128-slot
+ * kernel: mode 2: c[128][128] = a[128][D] * b[128][D]^T; mode 3: c[128][D] =
+ * a[128][128] * b[128][D] with a staged in TMEM.  a, b device bf16; c device
+ * fp32.  D 64 or 128.
  */
 int vsa_selftest_umma(int mode, int D, const void* a, const void* b, float* c, void* stream);
 

@@ -36,7 +36,9 @@ Readings where the pages leave a step open:
   R11 video tiles are (4,4,4), visited in row-major (t, h, w) tile order, with
       row-major (t, h, w) token order inside a tile and clipped edge tiles;
   R12 varlen inputs are token-packed ``[H, sum(len), D]`` tensors delimited by
-      cu_seqlens, and each sequence's ``q2k_idx`` rows hold local KV indices.
+      cu_seqlens, and each sequence's ``q2k_idx`` rows hold local KV indices;
+  R14 with 128-token tiles every step is the same with blocks of 128 slots
+      (pooling over 128 tokens, selections of 128 x 128 tiles).
 """
 
 from __future__ import annotations
@@ -58,25 +60,26 @@ def default_scale(D: int) -> float:
 # ---------------------------------------------------------------------------
 # a1: block mean-pooling
 # ---------------------------------------------------------------------------
-def block_pool(x, block_sizes) -> np.ndarray:
+def block_pool(x, block_sizes, block: int = BLOCK) -> np.ndarray:
     """Mean of each block's real tokens.
 
     [combine] Problem / Notes: the compression branch works on per-block means
     of q, k and v (the BSHD path takes an fp32 block sum).  Block ``j`` holds
-    its ``block_sizes[j]`` real tokens in slots ``64*j ..``; padded slots are
-    not pooled (R5, R6).
+    its ``block_sizes[j]`` real tokens in slots ``block*j ..``; padded slots
+    are not pooled (R5, R6).  ``block`` is the tile volume: 64, or 128 for the
+    128-token tiles of [readme] / [release] (R14).
 
-    x: [B, H, 64*n, D]  ->  [B, H, n, D] fp64
+    x: [B, H, block*n, D]  ->  [B, H, n, D] fp64
     """
     x = _f64(x)
     B, H, S, D = x.shape
     n = len(block_sizes)
-    assert S == BLOCK * n, "padded sequence must hold 64 slots per block"
+    assert S == block * n, "padded sequence must hold `block` slots per block"
     out = np.zeros((B, H, n, D), dtype=np.float64)
     for j, m in enumerate(block_sizes):
         m = int(m)
-        assert 1 <= m <= BLOCK
-        out[:, :, j, :] = x[:, :, BLOCK * j:BLOCK * j + m, :].sum(axis=2) / m
+        assert 1 <= m <= block
+        out[:, :, j, :] = x[:, :, block * j:block * j + m, :].sum(axis=2) / m
     return out
 
 
@@ -143,7 +146,7 @@ def select_topk(scores, topk: int, width: int | None = None):
 # a4: block-sparse attention over selected tiles
 # ---------------------------------------------------------------------------
 def block_sparse_attention(q, k, v, q2k_idx, q2k_num, q_block_sizes, kv_block_sizes,
-                           scale: float, items=None) -> np.ndarray:
+                           scale: float, items=None, block: int = BLOCK) -> np.ndarray:
     """Softmax attention of each query row over the real keys of the KV blocks
     its query block selected.
 
@@ -153,15 +156,16 @@ def block_sparse_attention(q, k, v, q2k_idx, q2k_num, q_block_sizes, kv_block_si
     contributes twice); padded keys are excluded and padded query rows are 0
     (R6); ``q2k_num == 0`` gives 0 (R9).
 
-    q: [B,H,64*nq,D], k/v: [B,H,64*nkv,D].  ``items`` optionally restricts the
-    work to an iterable of (b, h, query block) triples; other rows stay 0.
-    Returns O_s [B,H,64*nq,D] fp64.
+    q: [B,H,block*nq,D], k/v: [B,H,block*nkv,D] (block = 64, or 128 for the
+    128-token tiles, R14).  ``items`` optionally restricts the work to an
+    iterable of (b, h, query block) triples; other rows stay 0.
+    Returns O_s [B,H,block*nq,D] fp64.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, Sq, D = q.shape
     nq = len(q_block_sizes)
     nkv = len(kv_block_sizes)
-    assert Sq == BLOCK * nq and k.shape[2] == BLOCK * nkv
+    assert Sq == block * nq and k.shape[2] == block * nkv
     out = np.zeros_like(q)
     if items is None:
         items = [(b, h, a) for b in range(B) for h in range(H) for a in range(nq)]
@@ -175,12 +179,12 @@ def block_sparse_attention(q, k, v, q2k_idx, q2k_num, q_block_sizes, kv_block_si
             c = int(q2k_idx[b, h, a, j])
             if not 0 <= c < nkv:
                 raise IndexError(f"q2k_idx entry {c} outside [0, {nkv})")
-            key_rows.append(np.arange(BLOCK * c, BLOCK * c + int(kv_block_sizes[c])))
+            key_rows.append(np.arange(block * c, block * c + int(kv_block_sizes[c])))
         rows = np.concatenate(key_rows)
-        qa = q[b, h, BLOCK * a:BLOCK * a + mq, :]
+        qa = q[b, h, block * a:block * a + mq, :]
         logits = scale * (qa @ k[b, h, rows, :].T)
         p = softmax_rows(logits)
-        out[b, h, BLOCK * a:BLOCK * a + mq, :] = p @ v[b, h, rows, :]
+        out[b, h, block * a:block * a + mq, :] = p @ v[b, h, rows, :]
     return out
 
 
@@ -209,11 +213,11 @@ def block_map_to_indices(block_map):
 # ---------------------------------------------------------------------------
 # a5: coarse/sparse combine
 # ---------------------------------------------------------------------------
-def combine(out_c, o_s, gate, q_block_sizes) -> np.ndarray:
+def combine(out_c, o_s, gate, q_block_sizes, block: int = BLOCK) -> np.ndarray:
     """out = out_c * gate + out_s, with out_c held per block.
 
     [combine] Problem / Change: the coarse output stays at block resolution
-    [B, H, n_blocks, 1, D] and broadcasts over the 64 slots of its block;
+    [B, H, n_blocks, 1, D] and broadcasts over the slots of its block;
     the gate (``compress_attn_weight``) is laid out [B, S, H, D].  Ungated
     (gate None): out_c + out_s.  Padded query rows are 0 (R6).  Returned in
     fp64, i.e. before the single rounding of R10.
@@ -225,7 +229,7 @@ def combine(out_c, o_s, gate, q_block_sizes) -> np.ndarray:
     g = None if gate is None else _f64(gate).transpose(0, 2, 1, 3)  # -> [B,H,S,D]
     for a in range(nq):
         m = int(q_block_sizes[a])
-        sl = slice(BLOCK * a, BLOCK * a + m)
+        sl = slice(block * a, block * a + m)
         oc = out_c[:, :, a:a + 1, :]
         if g is None:
             out[:, :, sl, :] = oc + o_s[:, :, sl, :]
@@ -235,21 +239,22 @@ def combine(out_c, o_s, gate, q_block_sizes) -> np.ndarray:
 
 
 def vsa_forward(q, k, v, gate, q_block_sizes, kv_block_sizes, topk: int,
-                scale: float | None = None, width: int | None = None, items=None) -> dict:
+                scale: float | None = None, width: int | None = None, items=None,
+                block: int = BLOCK) -> dict:
     """The whole VSA forward: pool -> coarse attention -> top-k -> block-sparse
     attention -> combine ([readme] Usage ``video_sparse_attn``; [combine]
-    Problem for the combine)."""
+    Problem for the combine), on blocks of ``block`` slots (R14)."""
     D = np.shape(q)[-1]
     if scale is None:
         scale = default_scale(D)
-    qc = block_pool(q, q_block_sizes)
-    kc = block_pool(k, kv_block_sizes)
-    vc = block_pool(v, kv_block_sizes)
+    qc = block_pool(q, q_block_sizes, block)
+    kc = block_pool(k, kv_block_sizes, block)
+    vc = block_pool(v, kv_block_sizes, block)
     scores, out_c = coarse_attention(qc, kc, vc, scale)
     q2k_idx, q2k_num = select_topk(scores, topk, width)
     o_s = block_sparse_attention(q, k, v, q2k_idx, q2k_num, q_block_sizes, kv_block_sizes,
-                                 scale, items=items)
-    out = combine(out_c, o_s, gate, q_block_sizes)
+                                 scale, items=items, block=block)
+    out = combine(out_c, o_s, gate, q_block_sizes, block)
     return dict(qc=qc, kc=kc, vc=vc, scores=scores, out_c=out_c, q2k_idx=q2k_idx,
                 q2k_num=q2k_num, o_s=o_s, out=out)
 

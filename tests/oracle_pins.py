@@ -537,11 +537,70 @@ def check_block_map_to_indices(O):
     assert np.allclose(got[:, :, qr], want[:, :, qr], atol=1e-12)
 
 
+def check_block128(O):
+    """128-slot blocks (tile volume 128): pooling closed forms, the dense
+    limit against torch SDPA over the real tokens, arbitrary selections
+    against masked SDPA, the ungated combine as broadcast + sparse, and the
+    whole forward with topk = all equal to dense attention plus out_c."""
+    rng = _rng(31)
+    blk = 128
+    B, H, D = 1, 2, 16
+
+    def padded(sizes, pad_value=0.0):
+        x = np.full((B, H, blk * len(sizes), D), pad_value)
+        for j, m in enumerate(sizes):
+            x[:, :, blk * j:blk * j + m] = _bf16_like(rng, (B, H, m, D))
+        return x
+
+    def rows(sizes):
+        return np.concatenate([np.arange(blk * j, blk * j + m) for j, m in enumerate(sizes)])
+
+    # pooling: a ramp over the real slots has the mean of its real values
+    sizes = [128, 70, 1]
+    x = np.zeros((1, 1, blk * 3, 1))
+    for j, m in enumerate(sizes):
+        x[0, 0, blk * j:blk * j + m, 0] = np.arange(m)
+    x[0, 0, blk * 1 + 70:blk * 2, 0] = 1e6   # padding must not count
+    got = O.block_pool(x, sizes, block=blk)
+    assert np.allclose(got[0, 0, :, 0], [(m - 1) / 2 for m in sizes])
+    # dense limit, partial blocks, nq != nkv
+    q_sizes, kv_sizes = [128, 100], [128, 17, 128]
+    q, k, v = padded(q_sizes), padded(kv_sizes, 7.0), padded(kv_sizes, -7.0)
+    nkv = len(kv_sizes)
+    idx = np.broadcast_to(np.arange(nkv, dtype=np.int32), (B, H, 2, nkv)).copy()
+    num = np.full((B, H, 2), nkv, dtype=np.int32)
+    scale = 1 / np.sqrt(D)
+    got = O.block_sparse_attention(q, k, v, idx, num, q_sizes, kv_sizes, scale, block=blk)
+    qr, kr = rows(q_sizes), rows(kv_sizes)
+    want = _sdpa(q[:, :, qr], k[:, :, kr], v[:, :, kr], scale)
+    assert np.allclose(got[:, :, qr], want, atol=1e-12)
+    # arbitrary selections: masked SDPA
+    idx = np.array([[[[2, -1], [0, 1]], [[1, 2], [2, -1]]]], dtype=np.int32)
+    num = np.array([[[1, 2], [2, 1]]], dtype=np.int32)
+    got = O.block_sparse_attention(q, k, v, idx, num, q_sizes, kv_sizes, 0.3, block=blk)
+    mask = np.zeros((B, H, blk * 2, blk * 3), dtype=bool)
+    for b, h, a in np.ndindex(B, H, 2):
+        for j in range(num[b, h, a]):
+            c = idx[b, h, a, j]
+            mask[b, h, blk * a:blk * (a + 1), blk * c:blk * c + kv_sizes[c]] = True
+    want = _sdpa(q, k, v, 0.3, mask)
+    assert np.allclose(got[:, :, qr], want[:, :, qr], atol=1e-12)
+    # whole forward, topk = all: out = out_c (per block) + dense attention
+    res = O.vsa_forward(q, k, v, None, q_sizes, kv_sizes, nkv, block=blk)
+    dense = _sdpa(q[:, :, qr], k[:, :, kr], v[:, :, kr], scale)
+    oc = res["out_c"]
+    bcast = np.concatenate([np.repeat(oc[:, :, a:a + 1], m, axis=2) for a, m in enumerate(q_sizes)],
+                           axis=2)
+    assert np.allclose(res["out"][:, :, qr], bcast + dense, atol=1e-12)
+    pad = np.setdiff1d(np.arange(blk * 2), qr)
+    assert np.all(res["out"][:, :, pad] == 0.0)
+
+
 ALL_CHECKS = [
     check_pool_closed_forms, check_coarse_special_cases, check_coarse_vs_library,
     check_topk_brute_force, check_topk_edge_cases, check_sparse_dense_equivalence,
     check_sparse_vs_masked_library, check_sparse_invariants, check_combine,
     check_forward_dense_limit, check_varlen_pack_indices, check_varlen_equals_per_sequence,
     check_varlen_dense_vs_library, check_metadata, check_page_figures,
-    check_block_map_to_indices,
+    check_block_map_to_indices, check_block128,
 ]

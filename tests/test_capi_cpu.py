@@ -193,8 +193,11 @@ def test_metadata_matches_oracle(shape, tile):
 def test_metadata_rejects_bad_tiles():
     lib = _lib()
     n = ctypes.c_int32(0)
-    assert lib.build_vsa_metadata(4, 4, 4, 8, 4, 4, None, None, None, None, None,
-                                  ctypes.byref(n)) == 1          # tile volume 128 > 64
+    assert lib.build_vsa_metadata(4, 4, 4, 8, 4, 8, None, None, None, None, None,
+                                  ctypes.byref(n)) == 1          # tile volume 256 > 128
+    assert lib.build_vsa_metadata(8, 4, 4, 8, 4, 4, None, None, None, None, None,
+                                  ctypes.byref(n)) == 0          # 128-token tiles (VSA-128)
+    assert n.value == 1
     assert lib.build_vsa_metadata(0, 4, 4, 4, 4, 4, None, None, None, None, None,
                                   ctypes.byref(n)) == 1
 
@@ -218,22 +221,30 @@ def test_layouts_and_strided_argument_checks():
 
     def fwd(layout):
         return lib.vsa_forward_strided(fake, fake, fake, None, layout, None, None, B, H, Sq, Skv, D,
-                                       1, 0.0, fake, fake, fake, 1, None, None, 0, None)
+                                       block, 1, 0.0, fake, fake, fake, 1, None, None, 0, None)
+    block = 64
     assert fwd(None) == 1
     L.q.seq = 68   # 136 bytes: not a TMA stride
     assert fwd(ctypes.byref(L)) == 3
     lib.vsa_make_layout(0, B, H, Sq, Skv, D, ctypes.byref(L))
     assert fwd(ctypes.byref(L)) == 7   # valid layout: next check is the missing workspace
+    block = 96
+    assert fwd(ctypes.byref(L)) == 3   # block size neither 64 nor 128
+    block = 128
+    assert fwd(ctypes.byref(L)) == 2   # Skv = 192 is not a multiple of 128
+
 
 
 def test_bool_mask_entry_argument_checks():
     lib = _lib()
     fake = ctypes.c_void_p(1 << 20)
 
-    def call(bm=fake, idx=fake, num=fake, Sq=128, Skv=128, D=128):
-        return lib.block_sparse_attn(fake, fake, fake, bm, None, None, 1, 1, Sq, Skv, D, 0.0, fake,
-                                     idx, num, None, None, 0, None)
+    def call(bm=fake, idx=fake, num=fake, Sq=128, Skv=128, D=128, block=64):
+        return lib.block_sparse_attn(fake, fake, fake, bm, None, None, 1, 1, Sq, Skv, D, block, 0.0,
+                                     fake, idx, num, None, None, 0, None)
     assert call(bm=None) == 1
     assert call(idx=None) == 1
     assert call(Sq=100) == 2
     assert call(Skv=64 * 4096) == 3
+    assert call(block=96) == 3
+    assert call(Sq=192, block=128) == 2

@@ -17,9 +17,9 @@ MUTATIONS = [
      "idx[pos][:len(chosen)] = chosen[::-1]"),
     ("block map counts all entries", "num = bm.sum(axis=-1).astype(np.int32)",
      "num = np.full(bm.shape[:-1], bm.shape[-1], dtype=np.int32)"),
-    ("pool divides by 64", "sum(axis=2) / m", "sum(axis=2) / BLOCK"),
-    ("pool includes padding", "x[:, :, BLOCK * j:BLOCK * j + m, :].sum(axis=2)",
-     "x[:, :, BLOCK * j:BLOCK * j + BLOCK, :].sum(axis=2)"),
+    ("pool divides by the block", "sum(axis=2) / m", "sum(axis=2) / block"),
+    ("pool includes padding", "x[:, :, block * j:block * j + m, :].sum(axis=2)",
+     "x[:, :, block * j:block * j + block, :].sum(axis=2)"),
     ("coarse drops scale", 'scores = scale * np.einsum("bhqd,bhkd->bhqk", qc, kc)',
      'scores = np.einsum("bhqd,bhkd->bhqk", qc, kc)'),
     ("coarse softmax over q", "    p = softmax_rows(scores)\n",
@@ -32,12 +32,14 @@ MUTATIONS = [
     ("topk picks smallest", "order = np.lexsort((cols, -scores[b, h, a]))",
      "order = np.lexsort((cols, scores[b, h, a]))"),
     ("sparse attends padded keys",
-     "key_rows.append(np.arange(BLOCK * c, BLOCK * c + int(kv_block_sizes[c])))",
-     "key_rows.append(np.arange(BLOCK * c, BLOCK * c + BLOCK))"),
+     "key_rows.append(np.arange(block * c, block * c + int(kv_block_sizes[c])))",
+     "key_rows.append(np.arange(block * c, block * c + block))"),
     ("sparse drops scale", "logits = scale * (qa @ k[b, h, rows, :].T)",
      "logits = (qa @ k[b, h, rows, :].T)"),
     ("sparse uses k as values", "p @ v[b, h, rows, :]", "p @ k[b, h, rows, :]"),
-    ("sparse ignores q block size", "mq = int(q_block_sizes[a])", "mq = BLOCK"),
+    ("sparse ignores q block size", "mq = int(q_block_sizes[a])", "mq = block"),
+    ("sparse keys at 64-slot offsets", "key_rows.append(np.arange(block * c,",
+     "key_rows.append(np.arange(BLOCK * c,"),
     ("combine gate not transposed", "g = None if gate is None else _f64(gate).transpose(0, 2, 1, 3)",
      "g = None if gate is None else _f64(gate).reshape(o_s.shape)"),
     ("combine gates the sparse branch", "out[:, :, sl, :] = oc * g[:, :, sl, :] + o_s[:, :, sl, :]",
