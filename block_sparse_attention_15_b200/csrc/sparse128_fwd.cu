@@ -21,19 +21,21 @@
 // thread execute in issue order.
 //
 // Persistent grid, one CTA per SM walking the work items (query block, head,
-// batch) with stride gridDim.  384 threads, three warpgroups:
+// batch) with stride gridDim.  512 threads, four warpgroups:
 //   warp 0      Q tiles (double-buffered per item) and K tiles (2-stage ring)
 //   warp 1      TMEM owner; issues S(j) and PV(j-1) in that order
 //   warp 2      V tiles (2-stage ring)
-//   warps 4-7   softmax: S(j) -> P(j), row max with a lazy refresh (the
-//               reference max moves only when a logit exceeds it by more
-//               than kRefresh log2 units; then O is rescaled once the PV
-//               product before it is done), row sums
-//   warps 8-11  epilogue: O / l, out = out_c * gate + o (or out_c + o, or o),
+//   warps 4-11  softmax, two warpgroups splitting each row's key columns:
+//               S(j) -> P(j), row max with a lazy refresh (the reference max
+//               moves only when a logit exceeds it by more than kRefresh
+//               log2 units; then O is rescaled once the PV product before it
+//               is done), row sums
+//   warps 12-15 epilogue: O / l, out = out_c * gate + o (or out_c + o, or o),
 //               bf16 stores; double-buffered O lets it overlap the next item
-// Every wait is bounded and reports VSA_ERR_DEVICE_TIMEOUT; no named barrier
-// is used after the role split, so a warp that gives up a wait leaves no
-// other warp behind at a barrier.
+// Every wait is bounded and reports VSA_ERR_DEVICE_TIMEOUT.  The only named
+// barrier after the role split joins the two softmax groups; it also ORs
+// their abort flags, so a warp that gave up a wait never leaves the others
+// behind at it.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -46,10 +48,10 @@
 namespace vsa {
 namespace b128 {
 
-constexpr int kThreads = 384;
-constexpr uint32_t kRegsProducer = 56, kRegsSoftmax = 240, kRegsEpilogue = 112;
-constexpr uint32_t kLaunchRegs = 168;  // 384 x 168 <= 65536
-static_assert(128u * (kRegsProducer + kRegsSoftmax + kRegsEpilogue) <= 384u * kLaunchRegs,
+constexpr int kThreads = 512;
+constexpr uint32_t kRegsProducer = 56, kRegsSoftmax = 176, kRegsEpilogue = 104;
+constexpr uint32_t kLaunchRegs = 128;  // 512 x 128 = 65536
+static_assert(128u * (kRegsProducer + 2u * kRegsSoftmax + kRegsEpilogue) <= 512u * kLaunchRegs,
               "register split exceeds the launch's registers");
 constexpr int NK = 2, NV = 2;
 // Largest excess (log2 units) of a logit over its row's reference max that
@@ -65,7 +67,10 @@ struct Layout {
   static constexpr uint32_t kKOff = kQOff + 2 * kTile;         // [NK]
   static constexpr uint32_t kVOff = kKOff + NK * kTile;        // [NV]
   static constexpr uint32_t kInvLOff = kVOff + NV * kTile;     // [2][128] f32
-  static constexpr uint32_t kKMetaOff = kInvLOff + 2u * 128u * 4u;  // [NK] key counts
+  // exchange slots [4][2 halves][128] f32: tile maxima by tile parity (0, 1),
+  // row sums by item parity (2, 3)
+  static constexpr uint32_t kXchOff = kInvLOff + 2u * 128u * 4u;
+  static constexpr uint32_t kKMetaOff = kXchOff + 4u * 256u * 4u;   // [NK] key counts
   static constexpr uint32_t kSMetaOff = kKMetaOff + 4u * NK;        // [2] key count per S buffer
   static constexpr uint32_t kBarOff = (kSMetaOff + 4u * 2u + 7u) & ~7u;
   static constexpr int kQFull = 0, kQEmpty = 2, kKFull = 4, kKEmpty = kKFull + NK,
@@ -172,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t count = 1;  // a TMA transaction arrival or one tcgen05.commit
       if (i == L::kPFull || i == L::kPFull + 1 || i == L::kLFull || i == L::kLFull + 1 ||
           i == L::kOEmpty || i == L::kOEmpty + 1)
-        count = 4;  // one arrival per warp of the softmax or epilogue warpgroup
+        count = (i == L::kOEmpty || i == L::kOEmpty + 1) ? 4 : 8;  // per epilogue / softmax warp
       if (i == L::kSFull || i == L::kSFull + 1) count = 2;  // commit + key-count record
       mbar_init(bars + i, count);
     }
@@ -325,20 +330,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         g += x.num;
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     regs_inc<kRegsSoftmax>();
-    // ===================== softmax: one thread per query row =====================
-    const int wq = warp - 4;
-    const int row = wq * 32 + lane;  // TMEM lane = query row
+    // ===================== softmax =====================
+    // Two warpgroups split each query row's 128 key columns: a thread owns
+    // one row (TMEM lane) and 64 columns.  The row's tile max is combined
+    // through shared memory once per tile (named barrier 1, both groups), so
+    // both halves move the reference max at the same tile; each half keeps a
+    // partial row sum, added up at the end of the item.
+    const int half = (warp - 4) >> 2;           // key columns 64*half .. 64*half + 63
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;             // TMEM lane = query row
     const uint32_t t_lane = tmem_base + (uint32_t(wq * 32) << 16);
+    const uint32_t col0 = 64u * half;
+    float* xch = reinterpret_cast<float*>(smem + L::kXchOff);  // [slot][half][row]
     const float c = p.scale_log2;
     const uint64_t cc = pk2(c, c);
     uint32_t g = 0, n = 0;
-    bool aborted = false;
+    // A wait that gives up sets `aborted`; the groups' next barrier ORs it and
+    // every softmax warp leaves the loop there together.
+    bool aborted = false, stop = false;
     auto wwait = [&](uint64_t* bar, uint32_t parity) {
       if (!aborted && !warp_wait(bar, parity, abort_flag, p.status)) aborted = true;
     };
-    for (long long it = it0; !aborted && it < n_items; it += it_step, ++n) {
+    for (long long it = it0; !stop && it < n_items; it += it_step, ++n) {
       const Item x = load_item(p, it);
       const int o = (int)(n & 1);
       float m = -INFINITY;  // reference max of the row (log2 units)
@@ -348,23 +363,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         wwait(bars + L::kSFull + sb, (g >> 1) & 1);
         const int len = smeta[sb];
         tc_fence_after_sync();
-        uint32_t s[128];
+        uint32_t s[64];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) VSA_TMEM_LD16(t_lane + 128u * sb + 16u * q, s, 16 * q);
+        for (int q = 0; q < 4; ++q) VSA_TMEM_LD16(t_lane + 128u * sb + col0 + 16u * q, s, 16 * q);
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        // masked key columns become -inf
-        if (len < 128) {
+        const bool full = len >= 128;
+        if (!full) {
+          // masked key columns become -inf
 #pragma unroll
-          for (int q = 0; q < 128; ++q)
-            if (q >= len) s[q] = __float_as_uint(-INFINITY);
+          for (int q = 0; q < 64; ++q)
+            if ((int)col0 + q >= len) s[q] = __float_as_uint(-INFINITY);
         }
         float mx = -INFINITY;
 #pragma unroll
-        for (int q = 0; q < 128; q += 2) mx = fmax3(mx, __uint_as_float(s[q]), __uint_as_float(s[q + 1]));
-        mx *= c;
+        for (int q = 0; q < 64; q += 2) mx = fmax3(mx, __uint_as_float(s[q]), __uint_as_float(s[q + 1]));
+        // the row's tile max over both halves
+        float* xs = xch + (g & 1) * 256;
+        xs[half * 128 + row] = mx;
+        if (bar_red_or(1, 256, aborted)) { stop = true; break; }
+        mx = fmaxf(mx, xs[(half ^ 1) * 128 + row]) * c;
         // move the reference only when this tile's max exceeds it by more
-        // than kRefresh; then O (if any product has accumulated) and the
-        // partial sums are rescaled
+        // than kRefresh; then the partial sums and O (if any product has
+        // accumulated; each half scales half of O's columns) are rescaled
         const bool move = mx > m + kRefresh;
         if (__any_sync(0xffffffffu, move)) {
           const float nm = move ? mx : m;
@@ -376,62 +396,77 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t t = g - 1;
             wwait(bars + L::kPVDone + (int)(t & 1), (t >> 1) & 1);
             tc_fence_after_sync();
-            const uint32_t to = t_lane + kTmemO + D * o;
+            const uint32_t to = t_lane + kTmemO + D * o + (D / 2) * half;
 #pragma unroll
-            for (int q0 = 0; q0 < D; q0 += 32) {
-              uint32_t ov[32];
+            for (int q0 = 0; q0 < D / 2; q0 += 16) {
+              uint32_t ov[16];
               VSA_TMEM_LD16(to + q0, ov, 0);
-              VSA_TMEM_LD16(to + q0 + 16u, ov, 16);
               asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-              for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * alpha);
+              for (int q = 0; q < 16; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * alpha);
               VSA_TMEM_ST16(to + q0, ov, 0);
-              VSA_TMEM_ST16(to + q0 + 16u, ov, 16);
             }
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
           }
           m = nm;
         }
-        // probabilities 2^(s*c - m) as bf16 pairs, sums in fp32; a row that
-        // has seen no valid key yet (m = -inf) gets zeros
-        const float mref = (m == -INFINITY) ? 0.f : m;
-        const uint64_t nm2 = pk2(-mref, -mref);
-        uint32_t pk[64];
+        // probabilities 2^(s*c - m) as bf16 pairs, sums in fp32
+        uint32_t pk[32];
+        if (full) {
+          // every key real (the common case): no per-element tests
+          const uint64_t nm2 = pk2(-m, -m);
 #pragma unroll
-        for (int q = 0; q < 64; ++q) {
-          float a, b;
-          upk2(ffma2(pk2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), cc, nm2), a, b);
-          const uint64_t pp = ((q & 7) < 3) ? exp2_fma2(a, b) : pk2(fast_exp2(a), fast_exp2(b));
-          float p0, p1;
-          upk2(pp, p0, p1);
-          // masked columns: s = -inf gives 2^-inf = 0 on MUFU; the FMA-pipe
-          // routine clamps at -120, so zero those explicitly
-          if (2 * q >= len) p0 = 0.f;
-          if (2 * q + 1 >= len) p1 = 0.f;
-          if (m == -INFINITY) { p0 = 0.f; p1 = 0.f; }
-          upk2(fadd2(pk2(l0, l1), pk2(p0, p1)), l0, l1);
-          pk[q] = pack_bf16x2(p0, p1);
+          for (int q = 0; q < 32; ++q) {
+            float a, b;
+            upk2(ffma2(pk2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), cc, nm2), a, b);
+            const uint64_t pp = ((q & 7) < 3) ? exp2_fma2(a, b) : pk2(fast_exp2(a), fast_exp2(b));
+            upk2(fadd2(pk2(l0, l1), pp), l0, l1);
+            float p0, p1;
+            upk2(pp, p0, p1);
+            pk[q] = pack_bf16x2(p0, p1);
+          }
+        } else {
+          // masked columns (s = -inf) give exactly 0; a row that has seen no
+          // real key yet (m = -inf) too
+          const bool none = (m == -INFINITY);
+          const uint64_t nm2 = pk2(none ? 0.f : -m, none ? 0.f : -m);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            float a, b;
+            upk2(ffma2(pk2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), cc, nm2), a, b);
+            float p0 = fast_exp2(a), p1 = fast_exp2(b);
+            if (none || (int)col0 + 2 * q >= len) p0 = 0.f;
+            if (none || (int)col0 + 2 * q + 1 >= len) p1 = 0.f;
+            upk2(fadd2(pk2(l0, l1), pk2(p0, p1)), l0, l1);
+            pk[q] = pack_bf16x2(p0, p1);
+          }
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) VSA_TMEM_ST16(t_lane + 128u * sb + 16u * q, pk, 16 * q);
+        // P (bf16 pairs) into this half's 32 columns of the S buffer
+        VSA_TMEM_ST16(t_lane + 128u * sb + (col0 >> 1), pk, 0);
+        VSA_TMEM_ST16(t_lane + 128u * sb + (col0 >> 1) + 16u, pk, 16);
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(bars + L::kPFull + sb);
       }
-      // end of item: 1 / row sum for the epilogue (the epilogue of item n - 2
-      // has read this buffer's previous values: it released O buffer o, and
-      // the MMA warp waited for that before this item's first product)
-      const float lsum = l0 + l1;
-      if (n >= 2) wwait(bars + L::kOEmpty + o, ((n - 2) >> 1) & 1);
-      inv_l[o * 128 + row] = lsum > 0.f ? 1.f / lsum : 0.f;
+      if (stop) break;
+      // end of item: the row sum of both halves, then 1 / l for the epilogue
+      // (after the epilogue of item n - 2 released this buffer)
+      float* xs = xch + (2 + (n & 1)) * 256;
+      xs[half * 128 + row] = l0 + l1;
+      if (n >= 2 && half == 0) wwait(bars + L::kOEmpty + o, ((n - 2) >> 1) & 1);
+      if (bar_red_or(1, 256, aborted)) break;
+      if (half == 0) {
+        const float lsum = xs[row] + xs[128 + row];
+        inv_l[o * 128 + row] = lsum > 0.f ? 1.f / lsum : 0.f;
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + L::kLFull + o);
     }
   } else {
     regs_dec<kRegsEpilogue>();
     // ===================== epilogue: one thread per query row =====================
-    const int wq = warp - 8;
+    const int wq = warp - 12;
     const int row = wq * 32 + lane;
     const uint32_t t_lane = tmem_base + (uint32_t(wq * 32) << 16);
     uint32_t n = 0;
