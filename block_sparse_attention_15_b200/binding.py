@@ -74,7 +74,7 @@ SIGNATURES = {
                           _c_void_p, _c_size_t, _c_void_p]),
     "block_sparse_attn_from_indices_workspace_size": (_c_size_t, [_c_int] * 4),
     "block_sparse_attn_from_indices": (_c_int, [_c_void_p] * 7 + [_c_int] * 7 +
-                                       [_c_float, _c_void_p, _PL, _c_void_p, _c_size_t,
+                                       [_c_float, _c_void_p, _c_void_p, _PL, _c_void_p, _c_size_t,
                                         _c_void_p]),
     "block_sparse_attn": (_c_int, [_c_void_p] * 6 + [_c_int] * 6 +
                           [_c_float, _c_void_p, _c_void_p, _c_void_p, _PL, _c_void_p, _c_size_t,
@@ -82,7 +82,7 @@ SIGNATURES = {
     "block_sparse_attn_varlen_workspace_size": (_c_size_t, [_c_int] * 4),
     "block_sparse_attn_varlen": (_c_int, [_c_void_p] * 3 + [_P32, _P32, _P32, _P32, _P32, _P32] +
                                  [_c_int] * 3 + [_c_void_p, _c_void_p, _c_int, _c_float,
-                                                 _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                                 _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                                                  _c_void_p, _c_size_t, _c_void_p]),
     "build_vsa_metadata": (_c_int, [_c_int] * 6 + [_P64, _P64, _P32, _P64, _P64, _P32]),
     "vsa_gather_tokens": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int64, _c_int64, _c_int64,
@@ -91,6 +91,7 @@ SIGNATURES = {
                                     _c_int64, _c_int, _c_void_p]),
     "vsa_selftest_umma": (_c_int, [_c_int, _c_int, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "vsa_selftest_exp2": (_c_int, [_c_void_p, _c_void_p, _c_int64, _c_void_p, _c_void_p]),
+    "vsa_permute_rows": (_c_int, [_c_void_p, _c_void_p, _P64, _P64, _c_int, _c_void_p]),
     "vsa_set_profile_events": (_c_int, [ctypes.POINTER(_c_void_p)]),
 }
 
@@ -345,13 +346,16 @@ def _sparse_common(q, k, v, out):
 
 def block_sparse_attn_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes=None,
                                    kv_block_sizes=None, *, scale: float | None = None, out=None,
-                                   logit_bound: bool = True, block: int = 64, stream=None):
+                                   logit_bound: bool = True, block: int = 64,
+                                   return_lse: bool = False, stream=None):
     """Block-sparse attention over the listed tiles (``block_sparse_attn_from_indices``).
 
     q, k, v, out: [B, H, S, D] views (see :func:`vsa_forward`).  With
     ``logit_bound`` (default) a workspace is passed, so the library bounds
     each query block's logits first and the kernel skips its running-max
-    check where the bound allows (same results)."""
+    check where the bound allows (same results).  With ``return_lse`` also
+    returns the fp32 [B, H, Sq] natural-log log-sum-exp per query row (the
+    normaliser :func:`block_sparse_attn_backward` takes)."""
     B, H, Sq, Skv, D, out = _sparse_common(q, k, v, out)
     _require(q2k_idx, torch.int32, "q2k_idx")
     _require(q2k_num, torch.int32, "q2k_num")
@@ -367,11 +371,12 @@ def block_sparse_attn_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes=None
         ws = torch.empty(max(L.block_sparse_attn_from_indices_workspace_size(B, H, nq, nkv), 256),
                          dtype=torch.uint8, device=dev)
     lay = _layout(q, k, v, out)
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev) if return_lse else None
     _check("block_sparse_attn_from_indices", L.block_sparse_attn_from_indices(
         _ptr(q), _ptr(k), _ptr(v), _ptr(q2k_idx), _ptr(q2k_num), _ptr(qbs), _ptr(kbs), B, H, Sq,
         Skv, D, int(block), q2k_idx.shape[3], float(scale) if scale is not None else 0.0, _ptr(out),
-        ctypes.byref(lay), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
-    return out
+        _ptr(lse), ctypes.byref(lay), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return (out, lse) if return_lse else out
 
 
 def block_sparse_attn(q, k, v, block_map, q_block_sizes=None, kv_block_sizes=None, *,
@@ -429,7 +434,7 @@ def _host_i32(xs):
 def block_sparse_attn_varlen(q, k, v, cu_seqlens_q, cu_seqlens_kv, q2k_idx, q2k_num, *,
                              scale: float | None = None, q_block_sizes_list=None,
                              kv_block_sizes_list=None, return_aux: bool = False, out=None,
-                             stream=None):
+                             lse=None, stream=None):
     """Varlen block-sparse attention (``block_sparse_attn_varlen``).
 
     q: [H, total_q, D]; k, v: [H, total_kv, D]; cu_seqlens_*: host sequences
@@ -479,7 +484,7 @@ def block_sparse_attn_varlen(q, k, v, cu_seqlens_q, cu_seqlens_kv, q2k_idx, q2k_
     stride = q2k_idx.shape[-1]
     _check("block_sparse_attn_varlen", L.block_sparse_attn_varlen(
         _ptr(q), _ptr(k), _ptr(v), cq_p, ck_p, qs_p, qcb_p, ks_p, kcb_p, n, H, D, _ptr(q2k_idx),
-        _ptr(q2k_num), stride, float(scale) if scale is not None else 0.0, _ptr(out),
+        _ptr(q2k_num), stride, float(scale) if scale is not None else 0.0, _ptr(out), _ptr(lse),
         _ptr(aux[0]) if aux else None, _ptr(aux[1]) if aux else None,
         _ptr(aux[2]) if aux else None, _ptr(ws), ws.numel(), _stream(stream)))
     del keep
@@ -542,6 +547,29 @@ def selftest_umma(mode: int, a, b, *, stream=None):
     _check("vsa_selftest_umma", lib().vsa_selftest_umma(mode, D, _ptr(a), _ptr(b), _ptr(c),
                                                         _stream(stream)))
     return c
+
+
+def permute_rows(src, extents, src_strides, *, out=None, stream=None):
+    """``vsa_permute_rows``: rows of the last axis of ``src`` (a contiguous
+    bf16 CUDA tensor, D = src.shape[-1]) gathered into a new tensor of shape
+    (*extents, D): out[a0, a1, a2, a3] = src row a0*S0 + a1*S1 + a2*S2 + a3*S3."""
+    _require(src, torch.bfloat16, "src")
+    D = src.shape[-1]
+    ext = [int(e) for e in extents]
+    st = [int(x) for x in src_strides]
+    if len(ext) != 4 or len(st) != 4:
+        raise ValueError("extents and src_strides take four entries")
+    rows = src.numel() // D
+    if any(e > 0 for e in ext) and sum((e - 1) * s_ for e, s_ in zip(ext, st) if e > 0) >= rows:
+        raise ValueError("the strides reach past the end of src")
+    if out is None:
+        out = torch.empty((*ext, D), dtype=src.dtype, device=src.device)
+    _require(out, torch.bfloat16, "out")
+    e64 = (ctypes.c_int64 * 4)(*ext)
+    s64 = (ctypes.c_int64 * 4)(*st)
+    _check("vsa_permute_rows", lib().vsa_permute_rows(_ptr(src), _ptr(out), e64, s64, D,
+                                                      _stream(stream)))
+    return out
 
 
 def selftest_exp2(x, *, stream=None):

@@ -338,8 +338,8 @@ static int sparse_from_indices(const void* q, const void* k, const void* v,
                                const int32_t* q2k_idx, const int32_t* q2k_num,
                                const int32_t* q_block_sizes, const int32_t* kv_block_sizes, int B,
                                int H, int Sq_pad, int Skv_pad, int D, int block, int idx_stride,
-                               float scale, void* out, const vsa_layout* layout, void* workspace,
-                               size_t workspace_bytes, cudaStream_t st) {
+                               float scale, void* out, float* lse, const vsa_layout* layout,
+                               void* workspace, size_t workspace_bytes, cudaStream_t st) {
   if (!q || !k || !v || !out || !q2k_idx || !q2k_num) return VSA_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || idx_stride < 1 || !(scale == scale))
     return VSA_ERR_INVALID_ARG;
@@ -349,6 +349,7 @@ static int sparse_from_indices(const void* q, const void* k, const void* v,
   const int nq = Sq_pad / block, nkv = Skv_pad / block;
   if (idx_stride > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return VSA_ERR_INVALID_ARG;
+  if (lse && block != 64) return VSA_ERR_UNSUPPORTED;
   vsa_layout L;
   if (layout) L = *layout;
   else fill_layout(VSA_LAYOUT_BHSD, B, H, Sq_pad, Skv_pad, D, &L);
@@ -403,6 +404,8 @@ static int sparse_from_indices(const void* q, const void* k, const void* v,
   sp.nkv = nkv;
   sp.scale_log2 = sc * kLog2e;
   sp.qk_bound = qk_bound;
+  sp.lse = lse;
+  sp.lse_seq = Sq_pad;
   sp.status = status;
   if (block == 128)
     return launch_sparse128(sp, q, to_strides(L.q), Sq_pad, k, to_strides(L.k), v, to_strides(L.v),
@@ -415,11 +418,11 @@ int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
                                    const int32_t* q2k_idx, const int32_t* q2k_num,
                                    const int32_t* q_block_sizes, const int32_t* kv_block_sizes,
                                    int B, int H, int Sq_pad, int Skv_pad, int D, int block_size,
-                                   int idx_stride, float scale, void* out,
+                                   int idx_stride, float scale, void* out, float* lse,
                                    const vsa_layout* layout, void* workspace,
                                    size_t workspace_bytes, void* stream) {
   return sparse_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes, kv_block_sizes, B, H,
-                             Sq_pad, Skv_pad, D, block_size, idx_stride, scale, out, layout,
+                             Sq_pad, Skv_pad, D, block_size, idx_stride, scale, out, lse, layout,
                              workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
@@ -441,8 +444,8 @@ int block_sparse_attn(const void* q, const void* k, const void* v, const uint8_t
   int rc = launch_mask_to_indices(block_map, (long long)B * H * nq, nkv, q2k_idx, q2k_num, st);
   if (rc != VSA_OK) return rc;
   return sparse_from_indices(q, k, v, q2k_idx, q2k_num, q_block_sizes, kv_block_sizes, B, H,
-                             Sq_pad, Skv_pad, D, block_size, nkv, scale, out, layout, workspace,
-                             workspace_bytes, st);
+                             Sq_pad, Skv_pad, D, block_size, nkv, scale, out, nullptr, layout,
+                             workspace, workspace_bytes, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -494,7 +497,7 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
                              const int32_t* kv_block_sizes, const int32_t* cu_kv_blocks,
                              int n_seqs, int H, int D, const int32_t* q2k_idx,
                              const int32_t* q2k_num, int idx_stride, float scale, void* out,
-                             int64_t* pack_index_q, int64_t* pack_index_kv,
+                             float* lse, int64_t* pack_index_q, int64_t* pack_index_kv,
                              int32_t* q2k_idx_rebased, void* workspace, size_t workspace_bytes,
                              void* stream) {
   if (!q || !k || !v || !out || !q2k_idx || !q2k_num || !cu_seqlens_q || !cu_seqlens_kv)
@@ -606,6 +609,8 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
   sp.nkv = nkvb;
   sp.scale_log2 = sc * kLog2e;
   sp.qk_bound = bp.qk_bound;
+  sp.lse = lse;
+  sp.lse_seq = total_q;
   sp.varlen = 1;
   sp.status = status;
   return launch_sparse(sp, q, q_st, total_q, k, kv_st, v, kv_st, total_kv, D, false, false, st);

@@ -106,7 +106,8 @@ struct Layout {
   static constexpr uint32_t kAlphaOff = kFinOff + 64u * 4u;     // [64] rescale factors
   static constexpr uint32_t kMnOff = kAlphaOff + 64u * 4u;      // [64] minus the running max per column
   static constexpr uint32_t kInvLOff = kMnOff + 64u * 4u;       // [2][64] 1 / row sum per O buffer
-  static constexpr uint32_t kKMetaOff = kInvLOff + 2u * 64u * 4u;  // [NK] int2: key counts
+  static constexpr uint32_t kLseOff = kInvLOff + 2u * 64u * 4u;   // [2][64] log-sum-exp (log2 units)
+  static constexpr uint32_t kKMetaOff = kLseOff + 2u * 64u * 4u;  // [NK] int2: key counts
   static constexpr uint32_t kSMetaOff = kKMetaOff + 8u * NK;       // [kNS] int2: key counts per S^T buffer
   static constexpr uint32_t kVIssuedOff = kSMetaOff + 8u * kNS;   // V pairs requested so far
   static constexpr uint32_t kBarOff = kVIssuedOff + 16u;
@@ -396,6 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* red_all = reinterpret_cast<float*>(smem + L::kRedOff);
   float* fin_all = reinterpret_cast<float*>(smem + L::kFinOff);
   float* inv_l = reinterpret_cast<float*>(smem + L::kInvLOff);
+  float* lse_s = reinterpret_cast<float*>(smem + L::kLseOff);
   int2* kmeta = reinterpret_cast<int2*>(smem + L::kKMetaOff);
   int2* smeta = reinterpret_cast<int2*>(smem + L::kSMetaOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
@@ -789,7 +791,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // end of item: 1 / row sums for the epilogue
       if (n >= 2) wwait(bars + L::kOEmpty + o, (uint32_t)(((n - 2) >> 1) & 1));
       if (col_reduce32<false>(lp, red, fin, wq, lane, t128, bar_red, aborted)) { ok = false; break; }
-      if (t128 < 32) inv_l[o * 64 + col0 + t128] = fin[t128] > 0.f ? 1.f / fin[t128] : 0.f;
+      if (t128 < 32) {
+        const float l = fin[t128];
+        inv_l[o * 64 + col0 + t128] = l > 0.f ? 1.f / l : 0.f;
+        // log2 of the column's sum of 2^(s*c) = running max + log2(sum)
+        lse_s[o * 64 + col0 + t128] = l > 0.f ? __log2f(l) - mns[t128] : -INFINITY;
+      }
       named_barrier_sync(bar_red, 128);
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + L::kLFull + o);
@@ -824,6 +831,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool bad = !warp_wait(bars + L::kOFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status);
       if (!bad) bad = !warp_wait(bars + L::kLFull + o, (uint32_t)((n >> 1) & 1), abort_flag, p.status);
       if (bar_red_or(5, 128, bad)) break;
+      if (p.lse && t128 < 64) {
+        // natural-log log-sum-exp of each real query row (0 on padding rows)
+        const int q = t128;
+        if (q < x.q_len)
+          p.lse[x.group * p.lse_seq + x.q_tok + q] = lse_s[o * 64 + q] * 0.69314718055994531f;
+        else if (!p.varlen)
+          p.lse[x.group * p.lse_seq + x.q_tok + q] = 0.f;
+      }
       float4 oc = make_float4(0.f, 0.f, 0.f, 0.f);
       if (COMBINE) oc = *reinterpret_cast<const float4*>(p.out_c + (x.group * p.nq + x.a) * (long long)D + d0);
       // element offsets of the block's first token in out and gate

@@ -86,6 +86,8 @@ struct SparseParams {
   int B, H, nq, nkv;
   float scale_log2;           // softmax scale * log2(e)
   const float* qk_bound;      // [groups, nq] bound on scale_log2 * q.k (CoarseParams), or null
+  float* lse;                 // [groups, lse_seq] natural-log log-sum-exp per query row, or null
+  long long lse_seq;
   int varlen;                 // write only real rows
   int* status;
 };

@@ -295,6 +295,11 @@ int vsa_forward_host(const void* q, const void* k, const void* v, const void* ga
  * q2k_num  device int32 [B, H, n_q_blocks], each in [0, idx_stride]
  * idx_stride  1 .. VSA_MAX_BLOCKS
  * out      device bf16 [B, H, Sq_pad, D]
+ * lse      device fp32 [B, H, Sq_pad] or NULL: the natural-log
+ *          log-sum-exp of each real query row's scaled logits over its
+ *          selected keys (-inf where nothing is selected, 0 on padded rows),
+ *          the softmax normaliser block_sparse_attn_backward takes.  Block
+ *          size 64 only.
  * layout   host, strides of q, k, v and out (gate unused), or NULL for
  *          contiguous BHSD
  * workspace  device, >= block_sparse_attn_from_indices_workspace_size(...)
@@ -316,7 +321,7 @@ int block_sparse_attn_from_indices(const void* q, const void* k, const void* v,
                                    const int32_t* q2k_idx, const int32_t* q2k_num,
                                    const int32_t* q_block_sizes, const int32_t* kv_block_sizes,
                                    int B, int H, int Sq_pad, int Skv_pad, int D, int block_size,
-                                   int idx_stride, float scale, void* out,
+                                   int idx_stride, float scale, void* out, float* lse,
                                    const vsa_layout* layout, void* workspace,
                                    size_t workspace_bytes, void* stream);
 
@@ -381,6 +386,9 @@ size_t block_sparse_attn_varlen_workspace_size(int n_seqs, int total_q_blocks,
  *          hold indices local to sequence i's KV blocks
  * q2k_num  device int32 [H, total_q_blocks]
  * out      device bf16 [H, total_q, D]; only real token rows are written
+ * lse      device fp32 [H, total_q] or NULL: per real token row the
+ *          natural-log log-sum-exp of its scaled logits (see
+ *          block_sparse_attn_from_indices)
  * pack_index_q   device int64 [64 * total_q_blocks] or NULL: for each packed
  *          slot the token row of q it holds, -1 for padding
  * pack_index_kv  device int64 [64 * total_kv_blocks] or NULL: same for k/v
@@ -398,7 +406,7 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
                              const int32_t* kv_block_sizes, const int32_t* cu_kv_blocks,
                              int n_seqs, int H, int D, const int32_t* q2k_idx,
                              const int32_t* q2k_num, int idx_stride, float scale, void* out,
-                             int64_t* pack_index_q, int64_t* pack_index_kv,
+                             float* lse, int64_t* pack_index_q, int64_t* pack_index_kv,
                              int32_t* q2k_idx_rebased, void* workspace, size_t workspace_bytes,
                              void* stream);
 
@@ -454,6 +462,33 @@ int vsa_gather_tokens(const void* src, void* dst, const int64_t* slot_token, int
  */
 int vsa_scatter_tokens(const void* src, void* dst, const int64_t* slot_token, int64_t n_tokens,
                        int64_t n_slots, int64_t groups, int D, void* stream);
+
+/* ======================================================================== *
+ * head-sharded multi-GPU path: resharding around the all-to-all exchanges
+ * ======================================================================== */
+
+/*
+ * vsa_permute_rows -- copy rows of D bf16 elements: destination row
+ * ((a0 * E1 + a1) * E2 + a2) * E3 + a3 (a_i < E_i, extents[i] = E_i) takes
+ * source row a0 * S0 + a1 * S1 + a2 * S2 + a3 * S3 (src_strides[i] = S_i,
+ * in rows).  Every reshard of the sequence-parallel ("Ulysses") wrapper is
+ * one such call: a rank's sequence shard [B, S_local, H, D] packed into
+ * per-destination head groups [N, B, S_local, H/N, D] before the first
+ * all-to-all, the received shards gathered into [B, S, H/N, D], and the
+ * reverse two after the forward.
+ *
+ * Defined by: README "Compiled CUDA extensions" (the fused NVLink Ulysses
+ * all-to-all that reshards between sequence and head parallelism) and the
+ * 4-GPU sequence-parallel recipe it serves; the exchange itself is NCCL's.
+ *
+ * src, dst   device bf16; src must hold every row the strides reach, dst
+ *            E0 * E1 * E2 * E3 rows; both 16-byte aligned, not overlapping
+ * extents    host int64 [4]; E0, E1 <= 65535
+ * src_strides host int64 [4], >= 0
+ * D          a multiple of 8
+ */
+int vsa_permute_rows(const void* src, void* dst, const int64_t* extents,
+                     const int64_t* src_strides, int D, void* stream);
 
 /* ======================================================================== *
  * diagnostics

@@ -210,6 +210,103 @@ def block_map_to_indices(block_map):
     return idx, num
 
 
+def block_sparse_lse(q, k, q2k_idx, q2k_num, q_block_sizes, kv_block_sizes, scale: float,
+                     block: int = BLOCK) -> np.ndarray:
+    """Natural-log log-sum-exp of each real query row's scaled logits over
+    the keys its block selected (the softmax normaliser the backward pass
+    reuses); -inf where nothing is selected, 0 on padded rows.
+
+    Returns [B, H, block*nq] fp64.
+    """
+    q, k = _f64(q), _f64(k)
+    B, H, Sq, D = q.shape
+    lse = np.zeros((B, H, Sq), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            for a in range(len(q_block_sizes)):
+                mq = int(q_block_sizes[a])
+                n_sel = int(q2k_num[b, h, a])
+                if n_sel <= 0:
+                    lse[b, h, block * a:block * a + mq] = -np.inf
+                    continue
+                rows = np.concatenate([np.arange(block * int(c), block * int(c) + int(kv_block_sizes[int(c)]))
+                                       for c in q2k_idx[b, h, a, :n_sel]])
+                logits = scale * (q[b, h, block * a:block * a + mq] @ k[b, h, rows].T)
+                m = logits.max(axis=1)
+                lse[b, h, block * a:block * a + mq] = m + np.log(np.exp(logits - m[:, None]).sum(axis=1))
+    return lse
+
+
+def block_sparse_attention_backward(q, k, v, dout, q2k_idx, q2k_num, q_block_sizes,
+                                    kv_block_sizes, scale: float, block: int = BLOCK):
+    """Gradients of the block-sparse attention output with respect to q, k
+    and v, given the output gradient ``dout``.
+
+    "[kernel] Add varlen support for block-sparse attention", Backward
+    correctness / Test plan: dQ/dK/dV of the block-sparse attention, the
+    varlen backward equal to per-sequence gradients.  Per query block a with
+    selected key rows J (a block listed twice contributes its keys twice) and
+    P = softmax(scale * q_a k_J^T):
+      dV_J += P^T dout_a;  dP = dout_a v_J^T;
+      dS = P * (dP - rowsum(dP * P));
+      dq_a = scale * dS k_J;  dK_J += scale * dS^T q_a.
+    Padded rows (query or key) get 0.
+
+    Returns (dq, dk, dv) fp64, shaped like q, k, v.
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, H, Sq, D = q.shape
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        for h in range(H):
+            for a in range(len(q_block_sizes)):
+                mq = int(q_block_sizes[a])
+                n_sel = int(q2k_num[b, h, a])
+                if n_sel <= 0:
+                    continue
+                rows = np.concatenate([np.arange(block * int(c), block * int(c) + int(kv_block_sizes[int(c)]))
+                                       for c in q2k_idx[b, h, a, :n_sel]])
+                qa = q[b, h, block * a:block * a + mq]
+                da = do[b, h, block * a:block * a + mq]
+                p = softmax_rows(scale * (qa @ k[b, h, rows].T))
+                np.add.at(dv[b, h], rows, p.T @ da)
+                dp = da @ v[b, h, rows].T
+                ds = p * (dp - (dp * p).sum(axis=1, keepdims=True))
+                dq[b, h, block * a:block * a + mq] = scale * (ds @ k[b, h, rows])
+                np.add.at(dk[b, h], rows, scale * (ds.T @ qa))
+    return dq, dk, dv
+
+
+def build_k2q(q2k_idx, q2k_num, n_kv_blocks: int):
+    """The transposed selection: for every KV block c, the query blocks that
+    selected it, ascending, each with the number of times it lists c.
+
+    "[kernel] Add varlen support for block-sparse attention", Backward: the
+    varlen backward runs on a k2q index (KV block -> query blocks).
+    Returns (k2q_idx int32 [..., n_kv, nq] with -1 tails, k2q_cnt int32
+    [..., n_kv, nq] multiplicities, k2q_num int32 [..., n_kv]).
+    """
+    idx = np.asarray(q2k_idx)
+    num = np.asarray(q2k_num)
+    lead = idx.shape[:-2]
+    nq = idx.shape[-2]
+    k2q = np.full(lead + (n_kv_blocks, nq), -1, dtype=np.int32)
+    cnt = np.zeros(lead + (n_kv_blocks, nq), dtype=np.int32)
+    k2n = np.zeros(lead + (n_kv_blocks,), dtype=np.int32)
+    for pos in np.ndindex(*lead):
+        for c in range(n_kv_blocks):
+            blocks = []
+            for a in range(nq):
+                m = int(np.sum(idx[pos][a, :int(num[pos][a])] == c))
+                if m:
+                    blocks.append((a, m))
+            k2n[pos][c] = len(blocks)
+            for t, (a, m) in enumerate(blocks):
+                k2q[pos][c, t] = a
+                cnt[pos][c, t] = m
+    return k2q, cnt, k2n
+
+
 # ---------------------------------------------------------------------------
 # a5: coarse/sparse combine
 # ---------------------------------------------------------------------------

@@ -596,11 +596,90 @@ def check_block128(O):
     assert np.all(res["out"][:, :, pad] == 0.0)
 
 
+def _torch_sparse_forward(q, k, v, idx, num, q_sizes, kv_sizes, scale, block=BLOCK):
+    """Block-sparse attention written in torch ops (row gathers with
+    repeats, masked softmax) so that autograd differentiates it: a second,
+    independent route to the gradients."""
+    B, H, Sq, D = q.shape
+    out = torch.zeros_like(q)
+    outs = []
+    for b in range(B):
+        for h in range(H):
+            for a in range(len(q_sizes)):
+                mq = q_sizes[a]
+                n = int(num[b, h, a])
+                if n <= 0:
+                    continue
+                rows = torch.cat([torch.arange(block * int(c), block * int(c) + kv_sizes[int(c)])
+                                  for c in idx[b, h, a, :n]])
+                qa = q[b, h, block * a:block * a + mq]
+                p = torch.softmax(scale * qa @ k[b, h, rows].T, dim=-1)
+                outs.append(((b, h, a, mq), p @ v[b, h, rows]))
+    for (b, h, a, mq), o in outs:
+        out = out.index_put((torch.tensor([b]), torch.tensor([h]),
+                             torch.arange(block * a, block * a + mq)), o)
+    return out
+
+
+def check_backward(O):
+    """dq, dk, dv against torch autograd (fp64) of an independently written
+    forward, with duplicates, partial blocks, an empty selection and
+    nq != nkv; against central finite differences on a tiny case; lse
+    against torch's logsumexp; and the k2q index against a brute-force
+    count."""
+    rng = _rng(41)
+    B, H, D = 1, 2, 8
+    q_sizes, kv_sizes = [64, 37, 64], [64, 64, 20, 64]
+    q = _padded(rng, B, H, q_sizes, D)
+    k = _padded(rng, B, H, kv_sizes, D, pad_value=2.0)
+    v = _padded(rng, B, H, kv_sizes, D, pad_value=-2.0)
+    do = _padded(rng, B, H, q_sizes, D)
+    idx = np.array([[[[1, 2, 2, -1], [0, 3, -1, -1], [3, 1, 0, 2]],
+                     [[0, -1, -1, -1], [0, 0, 0, 0], [2, 3, -1, -1]]]], dtype=np.int32)
+    num = np.array([[[3, 2, 4], [0, 4, 2]]], dtype=np.int32)
+    scale = 0.37
+    dq, dk, dv = O.block_sparse_attention_backward(q, k, v, do, idx, num, q_sizes, kv_sizes, scale)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    out = _torch_sparse_forward(tq, tk, tv, idx, num, q_sizes, kv_sizes, scale)
+    out.backward(torch.tensor(do))
+    for got, want in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.allclose(got, want.numpy(), atol=1e-12)
+    assert np.all(dq[0, 1, 0:64] == 0.0)           # empty selection: no gradient
+    # finite differences on a few coordinates of a tiny case
+    f = lambda qq, kk, vv: float((O.block_sparse_attention(qq, kk, vv, idx, num, q_sizes, kv_sizes,
+                                                            scale) * do).sum())
+    eps = 1e-6
+    for arr, grad, where in ((q, dq, (0, 0, 70, 3)), (k, dk, (0, 1, 130, 5)), (v, dv, (0, 0, 140, 1)),
+                             (k, dk, (0, 0, 200, 0))):
+        plus, minus = arr.copy(), arr.copy()
+        plus[where] += eps
+        minus[where] -= eps
+        args_p = [plus if x is arr else x for x in (q, k, v)]
+        args_m = [minus if x is arr else x for x in (q, k, v)]
+        fd = (f(*args_p) - f(*args_m)) / (2 * eps)
+        assert abs(fd - grad[where]) < 1e-6, (where, fd, grad[where])
+    # lse against logsumexp over the selected real keys
+    lse = O.block_sparse_lse(q, k, idx, num, q_sizes, kv_sizes, scale)
+    rows = np.concatenate([np.arange(64 * c, 64 * c + kv_sizes[c]) for c in [3, 1, 0, 2]])
+    want = torch.logsumexp(scale * torch.tensor(q[0, 0, 128:192]) @ torch.tensor(k[0, 0, rows]).T, dim=-1)
+    assert np.allclose(lse[0, 0, 128:192], want.numpy(), atol=1e-12)
+    assert np.all(np.isneginf(lse[0, 1, 0:64]))
+    # k2q: brute-force multiplicities
+    k2q, cnt, k2n = O.build_k2q(idx, num, len(kv_sizes))
+    for h in range(H):
+        for c in range(len(kv_sizes)):
+            want = [(a, int(np.sum(idx[0, h, a, :num[0, h, a]] == c))) for a in range(len(q_sizes))]
+            want = [(a, m) for a, m in want if m]
+            assert k2n[0, h, c] == len(want)
+            assert [(int(k2q[0, h, c, t]), int(cnt[0, h, c, t])) for t in range(k2n[0, h, c])] == want
+            assert np.all(k2q[0, h, c, len(want):] == -1)
+
+
 ALL_CHECKS = [
     check_pool_closed_forms, check_coarse_special_cases, check_coarse_vs_library,
     check_topk_brute_force, check_topk_edge_cases, check_sparse_dense_equivalence,
     check_sparse_vs_masked_library, check_sparse_invariants, check_combine,
     check_forward_dense_limit, check_varlen_pack_indices, check_varlen_equals_per_sequence,
     check_varlen_dense_vs_library, check_metadata, check_page_figures,
-    check_block_map_to_indices, check_block128,
+    check_block_map_to_indices, check_block128, check_backward,
 ]

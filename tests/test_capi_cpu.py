@@ -161,7 +161,7 @@ def test_varlen_host_argument_checks():
         p = lambda x: None if x is None else x.ctypes.data_as(_P32)
         return lib.block_sparse_attn_varlen(fake, fake, fake, p(a), p(b), p(qs_a), p(qcb_a), None,
                                             None, n, 2, 128, fake, fake, 4, 0.0, fake, None, None,
-                                            None, None, 0, None)
+                                            None, None, None, 0, None)
 
     assert call([0], [0], 0) == 2                                 # empty batch
     assert call([0, 64, 64], [0, 64, 128], 2) == 2                # zero-token sequence

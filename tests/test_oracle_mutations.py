@@ -13,6 +13,14 @@ ORACLE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))
 
 # (name, exact source fragment, replacement)
 MUTATIONS = [
+    ("backward drops the softmax's rowsum term",
+     "ds = p * (dp - (dp * p).sum(axis=1, keepdims=True))", "ds = p * dp"),
+    ("backward dk without the scale", "np.add.at(dk[b, h], rows, scale * (ds.T @ qa))",
+     "np.add.at(dk[b, h], rows, ds.T @ qa)"),
+    ("backward dv ignores duplicates", "np.add.at(dv[b, h], rows, p.T @ da)",
+     "dv[b, h][rows] += p.T @ da"),
+    ("k2q drops multiplicities", "m = int(np.sum(idx[pos][a, :int(num[pos][a])] == c))",
+     "m = int(np.any(idx[pos][a, :int(num[pos][a])] == c))"),
     ("block map rows not ascending", "idx[pos][:len(chosen)] = chosen",
      "idx[pos][:len(chosen)] = chosen[::-1]"),
     ("block map counts all entries", "num = bm.sum(axis=-1).astype(np.int32)",
@@ -37,7 +45,9 @@ MUTATIONS = [
     ("sparse drops scale", "logits = scale * (qa @ k[b, h, rows, :].T)",
      "logits = (qa @ k[b, h, rows, :].T)"),
     ("sparse uses k as values", "p @ v[b, h, rows, :]", "p @ k[b, h, rows, :]"),
-    ("sparse ignores q block size", "mq = int(q_block_sizes[a])", "mq = block"),
+    ("sparse ignores q block size",
+     "        n_sel = int(q2k_num[b, h, a])\n        mq = int(q_block_sizes[a])\n",
+     "        n_sel = int(q2k_num[b, h, a])\n        mq = block\n"),
     ("sparse keys at 64-slot offsets", "key_rows.append(np.arange(block * c,",
      "key_rows.append(np.arange(BLOCK * c,"),
     ("combine gate not transposed", "g = None if gate is None else _f64(gate).transpose(0, 2, 1, 3)",
