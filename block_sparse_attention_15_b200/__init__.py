@@ -8,8 +8,10 @@ package is its Python binding plus the seeded input generator
 from .binding import (  # noqa: F401
     VSAError,
     block_sparse_attn,
+    block_sparse_attn_backward,
     block_sparse_attn_from_indices,
     block_sparse_attn_varlen,
+    block_sparse_attn_varlen_backward,
     build_vsa_metadata,
     check_device_status,
     gather_tokens,
@@ -22,7 +24,8 @@ from .binding import (  # noqa: F401
 )
 
 __all__ = [
-    "VSAError", "block_sparse_attn", "block_sparse_attn_from_indices", "block_sparse_attn_varlen", "build_vsa_metadata",
+    "VSAError", "block_sparse_attn", "block_sparse_attn_backward",
+    "block_sparse_attn_from_indices", "block_sparse_attn_varlen_backward", "block_sparse_attn_varlen", "build_vsa_metadata",
     "check_device_status", "gather_tokens", "get_device_status", "lib", "scatter_tokens",
     "vsa_forward", "vsa_forward_host", "video_sparse_attn_bshd",
 ]

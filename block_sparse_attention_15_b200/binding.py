@@ -80,6 +80,15 @@ SIGNATURES = {
                           [_c_float, _c_void_p, _c_void_p, _c_void_p, _PL, _c_void_p, _c_size_t,
                            _c_void_p]),
     "block_sparse_attn_varlen_workspace_size": (_c_size_t, [_c_int] * 4),
+    "block_sparse_attn_backward_workspace_size": (_c_size_t, [_c_int] * 4),
+    "block_sparse_attn_backward": (_c_int, [_c_void_p] * 10 + [_c_int] * 6 +
+                                   [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                    _c_size_t, _c_void_p]),
+    "block_sparse_attn_varlen_backward_workspace_size": (_c_size_t, [_c_int] * 5),
+    "block_sparse_attn_varlen_backward": (_c_int, [_c_void_p] * 6 + [_P32] * 6 + [_c_int] * 3 +
+                                          [_c_void_p, _c_void_p, _c_int, _c_float, _c_void_p,
+                                           _c_void_p, _c_void_p, _c_void_p, _c_size_t,
+                                           _c_void_p]),
     "block_sparse_attn_varlen": (_c_int, [_c_void_p] * 3 + [_P32, _P32, _P32, _P32, _P32, _P32] +
                                  [_c_int] * 3 + [_c_void_p, _c_void_p, _c_int, _c_float,
                                                  _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
@@ -426,6 +435,36 @@ def video_sparse_attn_bshd(q, k, v, gate=None, q_block_sizes=None, kv_block_size
     return (out,) + tuple(res[1:])
 
 
+def block_sparse_attn_backward(q, k, v, out, dout, lse, q2k_idx, q2k_num, q_block_sizes=None,
+                               kv_block_sizes=None, *, scale: float | None = None, stream=None):
+    """dq, dk, dv of :func:`block_sparse_attn_from_indices` (64-slot blocks,
+    contiguous BHSD) for the output gradient ``dout``; ``out`` and ``lse``
+    come from that forward call (``return_lse=True``)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _require(t, torch.bfloat16, n)
+    _require(lse, torch.float32, "lse")
+    _require(q2k_idx, torch.int32, "q2k_idx")
+    _require(q2k_num, torch.int32, "q2k_num")
+    B, H, Sq, D = q.shape
+    Skv = k.shape[2]
+    nq, nkv = Sq // 64, Skv // 64
+    if out.shape != q.shape or dout.shape != q.shape or lse.shape != (B, H, Sq):
+        raise ValueError("out and dout must be shaped like q, lse [B, H, Sq_pad]")
+    dev = q.device
+    qbs = _block_sizes_tensor(q_block_sizes, nq, dev)
+    kbs = _block_sizes_tensor(kv_block_sizes, nkv, dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    L = lib()
+    ws = torch.empty(max(L.block_sparse_attn_backward_workspace_size(B, H, Sq, nkv), 256),
+                     dtype=torch.uint8, device=dev)
+    _check("block_sparse_attn_backward", L.block_sparse_attn_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(q2k_idx), _ptr(q2k_num),
+        _ptr(qbs), _ptr(kbs), B, H, Sq, Skv, D, q2k_idx.shape[3],
+        float(scale) if scale is not None else 0.0, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
 def _host_i32(xs):
     arr = np.ascontiguousarray(np.asarray(xs, dtype=np.int32))
     return arr, arr.ctypes.data_as(_P32)
@@ -489,6 +528,36 @@ def block_sparse_attn_varlen(q, k, v, cu_seqlens_q, cu_seqlens_kv, q2k_idx, q2k_
         _ptr(aux[2]) if aux else None, _ptr(ws), ws.numel(), _stream(stream)))
     del keep
     return (out, *aux) if return_aux else out
+
+
+def block_sparse_attn_varlen_backward(q, k, v, out, dout, lse, cu_seqlens_q, cu_seqlens_kv,
+                                      q2k_idx, q2k_num, *, scale: float | None = None,
+                                      stream=None):
+    """dq, dk, dv of :func:`block_sparse_attn_varlen` (64-token blocks with a
+    partial last block per sequence); ``out`` and ``lse`` [H, total_q] come
+    from that forward call."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _require(t, torch.bfloat16, n)
+    _require(lse, torch.float32, "lse")
+    _require(q2k_idx, torch.int32, "q2k_idx")
+    _require(q2k_num, torch.int32, "q2k_num")
+    H, total_q, D = q.shape
+    cq, cq_p = _host_i32(cu_seqlens_q)
+    ck, ck_p = _host_i32(cu_seqlens_kv)
+    n = len(cq) - 1
+    nqb = sum(-(-(int(cq[i + 1]) - int(cq[i])) // 64) for i in range(n))
+    nkb = sum(-(-(int(ck[i + 1]) - int(ck[i])) // 64) for i in range(n))
+    dq, dk, dv = torch.zeros_like(q), torch.zeros_like(k), torch.zeros_like(v)
+    L = lib()
+    ws = torch.empty(max(L.block_sparse_attn_varlen_backward_workspace_size(n, nqb, nkb, H, total_q), 256),
+                     dtype=torch.uint8, device=q.device)
+    _check("block_sparse_attn_varlen_backward", L.block_sparse_attn_varlen_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), cq_p, ck_p, None, None, None,
+        None, n, H, D, _ptr(q2k_idx), _ptr(q2k_num), q2k_idx.shape[-1],
+        float(scale) if scale is not None else 0.0, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    del cq, ck
+    return dq, dk, dv
 
 
 def build_vsa_metadata(T: int, Hh: int, W: int, tile=(4, 4, 4)) -> dict:

@@ -491,6 +491,46 @@ static int resolve_blocks(const int32_t* cu, const int32_t* sizes, const int32_t
   return VSA_OK;
 }
 
+// Host-resolved varlen block tables: per packed query block its first token
+// row, size, first KV block of its sequence and that sequence's KV block
+// count; per packed KV block its first token row and size.
+struct VarlenTables {
+  std::vector<int32_t> table;  // qtok | qlen | kvbase | kvcount (nqb each), ktok | klen (nkvb each)
+  int nqb = 0, nkvb = 0;
+};
+
+static int varlen_tables(const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv,
+                         const int32_t* q_block_sizes, const int32_t* cu_q_blocks,
+                         const int32_t* kv_block_sizes, const int32_t* cu_kv_blocks, int n_seqs,
+                         VarlenTables& t) {
+  std::vector<int32_t> qtok, qlen, qfirst, ktok, klen, kfirst;
+  int rc = resolve_blocks(cu_seqlens_q, q_block_sizes, cu_q_blocks, n_seqs, qtok, qlen, qfirst);
+  if (rc != VSA_OK) return rc;
+  rc = resolve_blocks(cu_seqlens_kv, kv_block_sizes, cu_kv_blocks, n_seqs, ktok, klen, kfirst);
+  if (rc != VSA_OK) return rc;
+  const int nqb = (int)qtok.size(), nkvb = (int)ktok.size();
+  t.nqb = nqb;
+  t.nkvb = nkvb;
+  t.table.assign(4 * (size_t)nqb + 2 * (size_t)nkvb, 0);
+  int32_t* t_qtok = t.table.data();
+  int32_t* t_qlen = t_qtok + nqb;
+  int32_t* t_kvbase = t_qlen + nqb;
+  int32_t* t_kvcount = t_kvbase + nqb;
+  int32_t* t_ktok = t_kvcount + nqb;
+  int32_t* t_klen = t_ktok + nkvb;
+  for (int i = 0; i < n_seqs; ++i) {
+    for (int a = qfirst[i]; a < qfirst[i + 1]; ++a) {
+      t_qtok[a] = qtok[a];
+      t_qlen[a] = qlen[a];
+      t_kvbase[a] = kfirst[i];
+      t_kvcount[a] = kfirst[i + 1] - kfirst[i];
+    }
+  }
+  memcpy(t_ktok, ktok.data(), sizeof(int32_t) * nkvb);
+  memcpy(t_klen, klen.data(), sizeof(int32_t) * nkvb);
+  return VSA_OK;
+}
+
 int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
                              const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv,
                              const int32_t* q_block_sizes, const int32_t* cu_q_blocks,
@@ -507,29 +547,12 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
   if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
   if (idx_stride > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return VSA_ERR_INVALID_ARG;
-  std::vector<int32_t> qtok, qlen, qfirst, ktok, klen, kfirst;
-  int rc = resolve_blocks(cu_seqlens_q, q_block_sizes, cu_q_blocks, n_seqs, qtok, qlen, qfirst);
+  VarlenTables vt;
+  int rc = varlen_tables(cu_seqlens_q, cu_seqlens_kv, q_block_sizes, cu_q_blocks, kv_block_sizes,
+                         cu_kv_blocks, n_seqs, vt);
   if (rc != VSA_OK) return rc;
-  rc = resolve_blocks(cu_seqlens_kv, kv_block_sizes, cu_kv_blocks, n_seqs, ktok, klen, kfirst);
-  if (rc != VSA_OK) return rc;
-  const int nqb = (int)qtok.size(), nkvb = (int)ktok.size();
-  std::vector<int32_t> table(4 * (size_t)nqb + 2 * (size_t)nkvb);
-  int32_t* t_qtok = table.data();
-  int32_t* t_qlen = t_qtok + nqb;
-  int32_t* t_kvbase = t_qlen + nqb;
-  int32_t* t_kvcount = t_kvbase + nqb;
-  int32_t* t_ktok = t_kvcount + nqb;
-  int32_t* t_klen = t_ktok + nkvb;
-  for (int i = 0; i < n_seqs; ++i) {
-    for (int a = qfirst[i]; a < qfirst[i + 1]; ++a) {
-      t_qtok[a] = qtok[a];
-      t_qlen[a] = qlen[a];
-      t_kvbase[a] = kfirst[i];
-      t_kvcount[a] = kfirst[i + 1] - kfirst[i];
-    }
-  }
-  memcpy(t_ktok, ktok.data(), sizeof(int32_t) * nkvb);
-  memcpy(t_klen, klen.data(), sizeof(int32_t) * nkvb);
+  const int nqb = vt.nqb, nkvb = vt.nkvb;
+  const std::vector<int32_t>& table = vt.table;
   const size_t need = block_sparse_attn_varlen_workspace_size(n_seqs, nqb, nkvb, H);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return VSA_ERR_WORKSPACE;
@@ -614,6 +637,164 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
   sp.varlen = 1;
   sp.status = status;
   return launch_sparse(sp, q, q_st, total_q, k, kv_st, v, kv_st, total_kv, D, false, false, st);
+}
+
+// ---------------------------------------------------------------------------
+// backward of block_sparse_attn_from_indices and of the varlen entry
+// ---------------------------------------------------------------------------
+static size_t bwd_scratch_bytes(long long groups, long long q_rows_per_group, int nqb, int nkvb) {
+  return align256(sizeof(float) * (size_t)(groups * q_rows_per_group)) +
+         align256(sizeof(int32_t) * (size_t)groups * nkvb * nqb) +
+         align256(sizeof(int32_t) * (size_t)groups * nkvb);
+}
+
+size_t block_sparse_attn_backward_workspace_size(int B, int H, int Sq_pad, int n_kv_blocks) {
+  if (B <= 0 || H <= 0 || Sq_pad <= 0 || Sq_pad % 64 || n_kv_blocks <= 0) return 0;
+  return bwd_scratch_bytes((long long)B * H, Sq_pad, Sq_pad / 64, n_kv_blocks);
+}
+
+static void carve_bwd(BwdParams& bp, void* workspace, long long groups, long long q_rows, int nqb,
+                      int nkvb) {
+  char* ws = static_cast<char*>(workspace);
+  bp.delta = reinterpret_cast<float*>(ws);
+  ws += align256(sizeof(float) * (size_t)(groups * q_rows));
+  bp.k2q = reinterpret_cast<int32_t*>(ws);
+  ws += align256(sizeof(int32_t) * (size_t)groups * nkvb * nqb);
+  bp.k2q_num = reinterpret_cast<int32_t*>(ws);
+}
+
+int block_sparse_attn_backward(const void* q, const void* k, const void* v, const void* out,
+                               const void* dout, const float* lse, const int32_t* q2k_idx,
+                               const int32_t* q2k_num, const int32_t* q_block_sizes,
+                               const int32_t* kv_block_sizes, int B, int H, int Sq_pad,
+                               int Skv_pad, int D, int idx_stride, float scale, void* dq,
+                               void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (!q || !k || !v || !out || !dout || !lse || !q2k_idx || !q2k_num || !dq || !dk || !dv)
+    return VSA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || idx_stride < 1 || !(scale == scale))
+    return VSA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
+  if (Sq_pad % 64 || Skv_pad % 64) return VSA_ERR_SHAPE;
+  const int nq = Sq_pad / 64, nkv = Skv_pad / 64;
+  if (idx_stride > VSA_MAX_BLOCKS || nq > VSA_MAX_BLOCKS || nkv > VSA_MAX_BLOCKS)
+    return VSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return VSA_ERR_INVALID_ARG;
+  const size_t need = block_sparse_attn_backward_workspace_size(B, H, Sq_pad, nkv);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return VSA_ERR_WORKSPACE;
+  int* status = device_status_ptr();
+  if (!status) return VSA_ERR_CUDA;
+  const float sc = resolve_scale(scale, D);
+  BwdParams bp;
+  memset(&bp, 0, sizeof(bp));
+  bp.q = static_cast<const __nv_bfloat16*>(q);
+  bp.k = static_cast<const __nv_bfloat16*>(k);
+  bp.v = static_cast<const __nv_bfloat16*>(v);
+  bp.dout = static_cast<const __nv_bfloat16*>(dout);
+  bp.q_st = bp.do_st = bp.dq_st = bhsd_strides(H, Sq_pad, D);
+  bp.k_st = bp.v_st = bp.dk_st = bp.dv_st = bhsd_strides(H, Skv_pad, D);
+  bp.lse = lse;
+  bp.q_seq = Sq_pad;
+  bp.kv_seq = Skv_pad;
+  bp.q2k_idx = q2k_idx;
+  bp.q2k_num = q2k_num;
+  bp.idx_stride = idx_stride;
+  bp.q_bs = q_block_sizes;
+  bp.kv_bs = kv_block_sizes;
+  bp.dq = static_cast<__nv_bfloat16*>(dq);
+  bp.dk = static_cast<__nv_bfloat16*>(dk);
+  bp.dv = static_cast<__nv_bfloat16*>(dv);
+  bp.B = B;
+  bp.H = H;
+  bp.nq = nq;
+  bp.nkv = nkv;
+  bp.scale = sc;
+  bp.scale_log2 = sc * kLog2e;
+  bp.status = status;
+  carve_bwd(bp, workspace, (long long)B * H, Sq_pad, nq, nkv);
+  return launch_backward(bp, out, bhsd_strides(H, Sq_pad, D), D, static_cast<cudaStream_t>(stream));
+}
+
+size_t block_sparse_attn_varlen_backward_workspace_size(int n_seqs, int total_q_blocks,
+                                                        int total_kv_blocks, int H, int total_q) {
+  if (n_seqs <= 0 || total_q_blocks <= 0 || total_kv_blocks <= 0 || H <= 0 || total_q <= 0) return 0;
+  return align256(sizeof(int32_t) * (4 * (size_t)total_q_blocks + 2 * (size_t)total_kv_blocks)) +
+         bwd_scratch_bytes(H, total_q, total_q_blocks, total_kv_blocks);
+}
+
+int block_sparse_attn_varlen_backward(
+    const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv, const int32_t* q_block_sizes,
+    const int32_t* cu_q_blocks, const int32_t* kv_block_sizes, const int32_t* cu_kv_blocks,
+    int n_seqs, int H, int D, const int32_t* q2k_idx, const int32_t* q2k_num, int idx_stride,
+    float scale, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+    void* stream) {
+  if (!q || !k || !v || !out || !dout || !lse || !q2k_idx || !q2k_num || !dq || !dk || !dv ||
+      !cu_seqlens_q || !cu_seqlens_kv)
+    return VSA_ERR_INVALID_ARG;
+  if (n_seqs <= 0) return VSA_ERR_SHAPE;
+  if (H <= 0 || idx_stride < 1 || !(scale == scale)) return VSA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
+  if (idx_stride > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return VSA_ERR_INVALID_ARG;
+  VarlenTables vt;
+  int rc = varlen_tables(cu_seqlens_q, cu_seqlens_kv, q_block_sizes, cu_q_blocks, kv_block_sizes,
+                         cu_kv_blocks, n_seqs, vt);
+  if (rc != VSA_OK) return rc;
+  const int nqb = vt.nqb, nkvb = vt.nkvb;
+  if (nqb > 0xFFFF) return VSA_ERR_UNSUPPORTED;  // k2q packs query block numbers in 16 bits
+  const long long total_q = cu_seqlens_q[n_seqs], total_kv = cu_seqlens_kv[n_seqs];
+  const size_t need = block_sparse_attn_varlen_backward_workspace_size(n_seqs, nqb, nkvb, H, (int)total_q);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return VSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* dtab = static_cast<int32_t*>(workspace);
+  if (cudaMemcpyAsync(dtab, vt.table.data(), sizeof(int32_t) * vt.table.size(),
+                      cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  int* status = device_status_ptr();
+  if (!status) return VSA_ERR_CUDA;
+  const float sc = resolve_scale(scale, D);
+  const Strides3 q_st{0, total_q * D, D}, kv_st{0, total_kv * D, D};
+  BwdParams bp;
+  memset(&bp, 0, sizeof(bp));
+  bp.q = static_cast<const __nv_bfloat16*>(q);
+  bp.k = static_cast<const __nv_bfloat16*>(k);
+  bp.v = static_cast<const __nv_bfloat16*>(v);
+  bp.dout = static_cast<const __nv_bfloat16*>(dout);
+  bp.q_st = bp.do_st = bp.dq_st = q_st;
+  bp.k_st = bp.v_st = bp.dk_st = bp.dv_st = kv_st;
+  bp.lse = lse;
+  bp.q_seq = total_q;
+  bp.kv_seq = total_kv;
+  bp.q2k_idx = q2k_idx;
+  bp.q2k_num = q2k_num;
+  bp.idx_stride = idx_stride;
+  bp.q_tok = dtab;
+  bp.q_bs = dtab + nqb;
+  bp.q_kv_base = dtab + 2 * nqb;
+  bp.q_kv_count = dtab + 3 * nqb;
+  bp.kv_tok = dtab + 4 * nqb;
+  bp.kv_bs = dtab + 4 * nqb + nkvb;
+  bp.dq = static_cast<__nv_bfloat16*>(dq);
+  bp.dk = static_cast<__nv_bfloat16*>(dk);
+  bp.dv = static_cast<__nv_bfloat16*>(dv);
+  bp.B = 1;
+  bp.H = H;
+  bp.nq = nqb;
+  bp.nkv = nkvb;
+  bp.scale = sc;
+  bp.scale_log2 = sc * kLog2e;
+  bp.varlen = 1;
+  bp.status = status;
+  carve_bwd(bp, static_cast<char*>(workspace) + align256(sizeof(int32_t) * vt.table.size()), H,
+            total_q, nqb, nkvb);
+  return launch_backward(bp, out, q_st, D, st);
 }
 
 // ---------------------------------------------------------------------------

@@ -115,6 +115,43 @@ bool make_view_map_rows(CUtensorMap* map, TmaAxes* ax, const void* base, int D, 
 int launch_selftest_exp2(const float* x, float* y, long long n, int* mismatch,
                          cudaStream_t stream);
 
+// Backward of the 64-slot block-sparse attention (sparse_bwd.cu).  Work of
+// the dq pass: (query block, head, batch); of the dk/dv pass: (KV block,
+// head, batch).  Tables as in SparseParams (null: regular layout).
+struct BwdParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const __nv_bfloat16* dout;
+  Strides3 q_st, k_st, v_st, do_st;
+  TmaAxes q_ax, k_ax, v_ax, do_ax;  // filled by launch_backward
+  const float* lse;           // [groups, q_seq] natural-log log-sum-exp
+  float* delta;               // [groups, q_seq] scratch: sum_d dout * out
+  long long q_seq, kv_seq;
+  const int32_t* q2k_idx;     // [groups, nq, idx_stride]
+  const int32_t* q2k_num;
+  int idx_stride;
+  const int32_t* q_bs;
+  const int32_t* kv_bs;
+  const int32_t* q_tok;
+  const int32_t* kv_tok;
+  const int32_t* q_kv_base;
+  const int32_t* q_kv_count;
+  int32_t* k2q;               // [groups, nkv, nq] scratch: query block | multiplicity << 16
+  int32_t* k2q_num;           // [groups, nkv]
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  Strides3 dq_st, dk_st, dv_st;
+  int B, H, nq, nkv;
+  float scale, scale_log2;
+  int varlen;
+  int* status;
+};
+// delta, k2q, then the dq and dk/dv kernels, on `stream`.
+int launch_backward(const BwdParams& p, const void* out, Strides3 out_st, int D,
+                    cudaStream_t stream);
+
 // varlen / metadata helpers (vsa_varlen.cu)
 // Logit bound for the entries that take indices (same meaning as
 // CoarseParams::qk_bound): block row norms of q and k, then per (group,

@@ -411,6 +411,71 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
                              void* stream);
 
 /* ======================================================================== *
+ * backward of the block-sparse attention (64-slot blocks)
+ * ======================================================================== */
+
+/*
+ * Workspace bytes block_sparse_attn_backward needs: fp32 delta (sum over
+ * the head dim of dout * out) per query row [B, H, Sq_pad], then the k2q
+ * index (for every KV block the query blocks that selected it, with their
+ * multiplicities) [B, H, n_kv_blocks, Sq_pad / 64] and its counts.
+ */
+size_t block_sparse_attn_backward_workspace_size(int B, int H, int Sq_pad, int n_kv_blocks);
+
+/*
+ * block_sparse_attn_backward -- dq, dk, dv of block_sparse_attn_from_indices
+ * (block size 64) for the output gradient dout.
+ *
+ * Defined by: PR #1319 "Summary" / "Backward correctness" (dQ/dK/dV of the
+ * block-sparse attention; the backward goes through a k2q index, KV block
+ * -> query blocks) and release 0.3.0 ("Supports forward and backward").
+ * With P = softmax(scale * q k^T) over each query block's selected keys (a
+ * block listed twice counts twice): dv = P^T dout, dS = P * (dout v^T -
+ * rowsum(dout * out)), dq = scale * dS k, dk = scale * dS^T q.  Padded rows
+ * of dq, dk, dv are written as 0; keys no query block selected get 0.
+ *
+ * q, k, v, q2k_idx, q2k_num, block sizes, sizes, scale: as in the forward
+ *          call (contiguous BHSD)
+ * out      device bf16 [B, H, Sq_pad, D]: that call's output
+ * dout     device bf16 [B, H, Sq_pad, D]
+ * lse      device fp32 [B, H, Sq_pad]: that call's log-sum-exp output
+ * dq       device bf16 [B, H, Sq_pad, D], written
+ * dk, dv   device bf16 [B, H, Skv_pad, D], written
+ * workspace  device, >= block_sparse_attn_backward_workspace_size(...),
+ *          256-aligned
+ * Four launches on `stream`: delta, k2q, the dq pass and the dk/dv pass.
+ */
+int block_sparse_attn_backward(const void* q, const void* k, const void* v, const void* out,
+                               const void* dout, const float* lse, const int32_t* q2k_idx,
+                               const int32_t* q2k_num, const int32_t* q_block_sizes,
+                               const int32_t* kv_block_sizes, int B, int H, int Sq_pad,
+                               int Skv_pad, int D, int idx_stride, float scale, void* dq,
+                               void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* Workspace bytes block_sparse_attn_varlen_backward needs: the block tables,
+ * delta per packed query row [H, total_q] and the k2q index over the packed
+ * blocks. */
+size_t block_sparse_attn_varlen_backward_workspace_size(int n_seqs, int total_q_blocks,
+                                                        int total_kv_blocks, int H, int total_q);
+
+/*
+ * block_sparse_attn_varlen_backward -- dq, dk, dv of block_sparse_attn_varlen
+ * (PR #1319: the varlen backward through a k2q index; "dQ/dK/dV match
+ * per-sequence reference exactly").  Arguments as in the forward varlen call
+ * plus out and lse from it (lse [H, total_q]), dout [H, total_q, D] and the
+ * outputs dq [H, total_q, D], dk, dv [H, total_kv, D] (real token rows
+ * written).
+ */
+int block_sparse_attn_varlen_backward(
+    const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv, const int32_t* q_block_sizes,
+    const int32_t* cu_q_blocks, const int32_t* kv_block_sizes, const int32_t* cu_kv_blocks,
+    int n_seqs, int H, int D, const int32_t* q2k_idx, const int32_t* q2k_num, int idx_stride,
+    float scale, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+    void* stream);
+
+/* ======================================================================== *
  * a7: video tile metadata (host) and token gather / scatter (device)
  * ======================================================================== */
 
