@@ -681,20 +681,65 @@ def run_entry(args, wl):
     """Other entry points on the same workload, one call per step, the whole
     call timed: ``indices`` = block_sparse_attn_from_indices (with its
     logit-bound pass) on the selection the forward makes; ``bshd`` = the
-    whole forward on BSHD tensors (video_sparse_attn_bshd)."""
+    whole forward on BSHD tensors (video_sparse_attn_bshd); ``backward`` =
+    block_sparse_attn_backward on that selection (TFLOP/s over 2.5 x the
+    forward's tile FLOPs: S recomputed, dP, dV, dK and dQ); ``ulysses`` = the
+    sequence-parallel wrapper over the job's ranks (strong scaling: the
+    sequence is split, the total work is fixed)."""
     from block_sparse_attention_15_b200 import binding as vsa
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
-        raise SystemExit("--entry other than forward runs on one GPU")
+    world_env = int(os.environ.get("WORLD_SIZE", "1"))
+    if world_env > 1 and args.entry != "ulysses":
+        raise SystemExit("--entry other than forward and ulysses runs on one GPU")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.entry == "ulysses":
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev,
+                                init_method="env://" if world_env > 1 else
+                                f"tcp://127.0.0.1:{29500 + (os.getpid() % 1000)}",
+                                rank=int(os.environ.get("RANK", "0")), world_size=world_env)
     q_h, k_h, v_h, g_h = host_inputs(wl)
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     gate = None if g_h is None else g_h.to(dev)
     qbs = None if all(s == 64 for s in wl.q_block_sizes) else wl.q_block_sizes
     kbs = None if all(s == 64 for s in wl.kv_block_sizes) else wl.kv_block_sizes
-    out, idx, num = vsa.vsa_forward(q, k, v, gate, qbs, kbs, topk=wl.topk)
-    if args.entry == "indices":
+    out, idx, num = vsa.vsa_forward(q, k, v, gate, qbs, kbs, topk=wl.topk, block=wl.block)
+    flops = wl.flops
+    kernels = None
+    if args.entry == "backward":
+        # the backward of the sparse attention on the forward's selection:
+        # algorithmic work 5 tile products (S recomputed, dP, dV, dK, dQ)
+        # = 2.5 x the forward's per tile
+        if wl.block != 64:
+            raise SystemExit("the backward covers 64-slot blocks")
+        o_s, lse = vsa.block_sparse_attn_from_indices(q, k, v, idx, num, qbs, kbs, return_lse=True)
+        dout = I.normal_bf16(tuple(q.shape), wl.seed, 7).to(dev)
+
+        def step():
+            vsa.block_sparse_attn_backward(q, k, v, o_s, dout, lse, idx, num, qbs, kbs)
+        what = "block_sparse_attn_backward (delta, k2q, dq pass, dk/dv pass) on the forward's selection"
+        launches = 4
+        flops = 2.5 * wl.flops
+    elif args.entry == "ulysses":
+        # the sequence-parallel wrapper over the ranks of the job (one rank:
+        # the exchanges are the identity; the reshards and the forward run)
+        from block_sparse_attention_15_b200 import ulysses as U
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        qb, kb, vb = (x.transpose(1, 2).contiguous() for x in (q, k, v))
+        del q, k, v
+        rank = int(os.environ.get("RANK", "0"))
+        Sl, Skl = qb.shape[1] // world, kb.shape[1] // world
+        sh = lambda x, s_: x[:, rank * s_:(rank + 1) * s_].contiguous()
+        qs_, ks_, vs_ = sh(qb, Sl), sh(kb, Skl), sh(vb, Skl)
+        gs_ = None if gate is None else sh(gate, Sl)
+
+        def step():
+            U.vsa_forward_ulysses(qs_, ks_, vs_, gs_, qbs, kbs, topk=wl.topk, block=wl.block)
+        what = "sequence-parallel forward (row reshards + all-to-all + BSHD forward)"
+        launches = 11
+    elif args.entry == "indices":
         def step():
             vsa.block_sparse_attn_from_indices(q, k, v, idx, num, qbs, kbs, out=out)
         what = "block_sparse_attn_from_indices with its logit-bound pass, on the forward's selection"
@@ -726,7 +771,7 @@ def run_entry(args, wl):
     ms = e0.elapsed_time(e1) / args.steps
     peaks, peak_kind = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    tflops = wl.flops / (ms * 1e-3) / 1e12
+    tflops = flops / (ms * 1e-3) / 1e12
     line = {"metric": METRIC + f" [{args.entry} entry]", "value": tflops, "unit": "TFLOP/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -735,7 +780,16 @@ def run_entry(args, wl):
                          "frac": tflops / peak, "traffic": None, "kernel": f"whole call: {what}",
                          "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS)"},
             "gpu_launches": launches * args.steps, "clocks": clocks}
-    print(json.dumps(line), flush=True)
+    if args.entry == "ulysses":
+        import torch.distributed as dist
+        line["n_gpus"] = dist.get_world_size()
+        line["scaling"] = "strong"
+        if dist.get_rank() != 0:
+            line = None
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
     return 0
 
 
@@ -751,7 +805,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-items", type=int, default=24,
                     help="query blocks per reference-arm step (bounded CPU sample)")
-    ap.add_argument("--entry", choices=["forward", "indices", "bshd"], default="forward",
+    ap.add_argument("--entry", choices=["forward", "indices", "bshd", "backward", "ulysses"],
+                    default="forward",
                     help="entry point timed on the workload (forward: the headline line)")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (smaller cases for profiler captures)")

@@ -108,6 +108,9 @@ def vsa_forward_ulysses(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=N
     if (N * Sq) % block or (N * Skv) % block:
         raise ValueError("the gathered sequences must be multiples of the block size")
     Hn = H // N
+    if N == 1:
+        # one rank: both exchanges and all four reshards are the identity
+        return ops.forward(q, k, v, gate, q_block_sizes, kv_block_sizes, topk, scale, block)
 
     def to_heads(x, S):
         sent = ops.permute(x.contiguous().view(-1, D), *pack_heads_spec(B, S, H, N))

@@ -1,7 +1,7 @@
 """The sequence-parallel wrapper's kernels on the GPU: the library's row
 permutation (vsa_permute_rows) against the reference gather on the four
-reshard specs, bit for bit; and the whole wrapper on a one-rank NCCL group,
-where both exchanges are the identity, equal to the single-GPU BSHD forward
+reshard specs, bit for bit; and the whole wrapper on a one-rank NCCL group
+(where it calls the forward directly) equal to the single-GPU BSHD forward
 bit for bit.  (The exchange order across several ranks is covered on the CPU
 with two gloo ranks in test_ulysses_multirank.py; this run has one GPU.)"""
 import os
