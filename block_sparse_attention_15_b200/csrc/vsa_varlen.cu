@@ -47,28 +47,48 @@ __global__ void rebase_kernel(const int32_t* q2k_idx, const int32_t* q2k_num,
   out[i] = v;
 }
 
-// One CTA per (16 slots, group): thread t moves 16-byte chunk t % (D / 8) of
-// slot t / (D / 8); 32-bit index arithmetic only (every tensor here holds
-// fewer than 2^31 16-byte chunks per group).
+// One CTA per (SPB * kSlotsPerThread slots, group): thread t moves 16-byte
+// chunk t % (D / 8) of kSlotsPerThread slots spaced SPB apart.  The slot
+// indices are loaded first, then every data load, then every store, so a
+// gather's two dependent loads (index, then token row) overlap across slots.
+// 32-bit index arithmetic (every tensor here holds fewer than 2^31 16-byte
+// chunks per group).
+constexpr int kSlotsPerThread = 4;
+
 template <bool SCATTER, int D>
 __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint4* src, uint4* dst,
                                                             const int64_t* slot_token,
                                                             int n_tokens, int n_slots) {
   constexpr int CH = D / 8;             // 16-byte chunks per row
-  constexpr int SPB = 256 / CH;         // slots per CTA
-  const int s = blockIdx.x * SPB + (int)threadIdx.x / CH;
+  constexpr int SPB = 256 / CH;         // slots per pass
   const int ch = (int)threadIdx.x % CH;
-  if (s >= n_slots) return;
+  const int s0 = blockIdx.x * SPB * kSlotsPerThread + (int)threadIdx.x / CH;
   const long long g = blockIdx.y;
-  const int64_t tok = slot_token[s];
-  const bool real = tok >= 0 && tok < n_tokens;
-  const long long slot_i = (g * n_slots + s) * CH + ch;
-  if (!SCATTER) {
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (real) v = __ldcs(src + ((g * n_tokens + tok) * CH + ch));
-    __stcs(dst + slot_i, v);
-  } else if (real) {
-    __stcs(dst + ((g * n_tokens + tok) * CH + ch), __ldcs(src + slot_i));
+  int64_t tok[kSlotsPerThread];
+#pragma unroll
+  for (int i = 0; i < kSlotsPerThread; ++i) {
+    const int s = s0 + i * SPB;
+    tok[i] = s < n_slots ? slot_token[s] : -1;
+  }
+  uint4 v[kSlotsPerThread];
+#pragma unroll
+  for (int i = 0; i < kSlotsPerThread; ++i) {
+    const int s = s0 + i * SPB;
+    const bool real = tok[i] >= 0 && tok[i] < n_tokens;
+    v[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (s < n_slots && real)
+      v[i] = SCATTER ? __ldcs(src + (g * n_slots + s) * CH + ch)
+                     : __ldcs(src + (g * n_tokens + tok[i]) * CH + ch);
+  }
+#pragma unroll
+  for (int i = 0; i < kSlotsPerThread; ++i) {
+    const int s = s0 + i * SPB;
+    if (s >= n_slots) continue;
+    if (!SCATTER) {
+      __stcs(dst + (g * n_slots + s) * CH + ch, v[i]);
+    } else if (tok[i] >= 0 && tok[i] < n_tokens) {
+      __stcs(dst + (g * n_tokens + tok[i]) * CH + ch, v[i]);
+    }
   }
 }
 
@@ -264,7 +284,7 @@ int launch_gather_tokens(const void* src, void* dst, const int64_t* slot_token, 
                          cudaStream_t stream) {
   if (groups <= 0 || n_slots <= 0) return VSA_OK;
   if (n_tokens > 0x7FFFFFFFLL || n_slots > 0x7FFFFFFFLL || groups > 65535) return VSA_ERR_UNSUPPORTED;
-  const int spb = D <= 2048 ? 256 / (D / 8) : 1;
+  const int spb = D <= 2048 ? 256 / (D / 8) * kSlotsPerThread : 1;
   const dim3 grid((unsigned)((n_slots + spb - 1) / spb), (unsigned)groups);
   const uint4* s4 = static_cast<const uint4*>(src);
   uint4* d4 = static_cast<uint4*>(dst);
