@@ -122,9 +122,9 @@ int check_forward_args(const ForwardArgs& a) {
 int launch_forward(const ForwardArgs& a, void* scratch, bool profile, cudaStream_t st) {
   const int B = a.B, H = a.H, D = a.D;
   const int nq = a.Sq_pad / a.block, nkv = a.Skv_pad / a.block;
-  // the logit bound serves the 64-slot kernel's vote-free step; the 128-slot
-  // kernel keeps its row maxima in-thread and needs none
-  const bool bound = a.block == 64;
+  // the logit bound lets both sparse kernels skip their running-max checks
+  // where it proves them unneeded
+  const bool bound = true;
   const int k_eff = a.topk < nkv ? a.topk : nkv;
   int* status = device_status_ptr();
   if (!status) return VSA_ERR_CUDA;

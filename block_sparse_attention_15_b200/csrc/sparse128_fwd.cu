@@ -58,6 +58,13 @@ constexpr int NK = 2, NV = 2;
 // is exponentiated without moving the reference: probabilities stay below
 // 2^8, well inside bf16 and fp32 range.
 constexpr float kRefresh = 8.f;
+// Largest excess (log2 units) of a logit over its row's first-tile max that
+// the logit bound must rule out before an item's later tiles skip the max
+// exchange: probabilities then stay below 2^32 (bf16 and fp32 hold them).
+constexpr float kBoundLimit = 32.f;
+#ifndef VSA128_POLY8
+#define VSA128_POLY8 3  // column pairs in eight whose exponential runs on the FMA pipe
+#endif
 
 template <int D>
 struct Layout {
@@ -358,6 +365,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int o = (int)(n & 1);
       float m = -INFINITY;  // reference max of the row (log2 units)
       float l0 = 0.f, l1 = 0.f;
+      // bound on every logit of the item (log2 units), from block row norms;
+      // once the first tile has fixed the row maxima and the bound keeps
+      // every later logit within kBoundLimit of them, later tiles skip the
+      // max exchange (same results: the reference max would not move)
+      const float qk_bound = p.qk_bound ? p.qk_bound[x.group * p.nq + x.a] : INFINITY;
+      bool novote = false;
       for (int j = 0; j < x.num; ++j, ++g) {
         const int sb = (int)(g & 1);
         wwait(bars + L::kSFull + sb, (g >> 1) & 1);
@@ -374,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int q = 0; q < 64; ++q)
             if ((int)col0 + q >= len) s[q] = __float_as_uint(-INFINITY);
         }
+        if (!novote) {
         float mx = -INFINITY;
 #pragma unroll
         for (int q = 0; q < 64; q += 2) mx = fmax3(mx, __uint_as_float(s[q]), __uint_as_float(s[q + 1]));
@@ -410,6 +424,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           m = nm;
         }
+        if (j == 0) {
+          // the first tile fixed the row maxima: can the bound rule out a move
+          // for every row of the item?  (m = -inf fails the test)
+          novote = bar_red_and(1, 256, qk_bound - m <= kBoundLimit);
+        }
+        }
         // probabilities 2^(s*c - m) as bf16 pairs, sums in fp32
         uint32_t pk[32];
         if (full) {
@@ -419,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int q = 0; q < 32; ++q) {
             float a, b;
             upk2(ffma2(pk2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), cc, nm2), a, b);
-            const uint64_t pp = ((q & 7) < 3) ? exp2_fma2(a, b) : pk2(fast_exp2(a), fast_exp2(b));
+            const uint64_t pp = ((q & 7) < VSA128_POLY8) ? exp2_fma2(a, b) : pk2(fast_exp2(a), fast_exp2(b));
             upk2(fadd2(pk2(l0, l1), pp), l0, l1);
             float p0, p1;
             upk2(pp, p0, p1);
