@@ -55,6 +55,8 @@ def make_workload(name: str) -> I.Workload:
         return I.workload_h3()
     if name == "vsa128":
         return I.workload_vsa128()
+    if name == "vsa256":
+        return I.workload_vsa256()
     m = re.fullmatch(r"long(\d+)(-ungated)?", name)
     if m:
         return I.workload_long(int(m.group(1)) / 100.0, gated=m.group(2) is None)

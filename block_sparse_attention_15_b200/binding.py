@@ -217,8 +217,8 @@ def vsa_forward(q, k, v, gate=None, q_block_sizes=None, kv_block_sizes=None, *, 
     or None.  Any of them may be a strided view (head dim contiguous, other
     strides multiples of 8): a BSHD tensor transposed to [B, H, S, D], a
     slice of a fused QKV tensor.  ``out`` (allocated like q if None) may be a
-    view too.  ``block``: slots per block, 64 or 128 (VSA-128 tiles; S is then
-    padded to multiples of 128).  Returns ``(out, q2k_idx, q2k_num)`` plus
+    view too.  ``block``: slots per block, 64, 128 or 256 (VSA-128 / VSA-256
+    tiles; S is then padded to multiples of the block).  Returns ``(out, q2k_idx, q2k_num)`` plus
     ``out_c`` and the pooled (qc, kc, vc) when asked.
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):

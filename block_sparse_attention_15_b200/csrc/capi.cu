@@ -99,7 +99,7 @@ int check_forward_args(const ForwardArgs& a) {
   if (a.B <= 0 || a.H <= 0 || a.Sq_pad <= 0 || a.Skv_pad <= 0 || a.topk < 1 || !(a.scale == a.scale))
     return VSA_ERR_INVALID_ARG;
   if (a.D != 64 && a.D != 128) return VSA_ERR_UNSUPPORTED;
-  if (a.block != 64 && a.block != 128) return VSA_ERR_UNSUPPORTED;
+  if (a.block != 64 && a.block != 128 && a.block != 256) return VSA_ERR_UNSUPPORTED;
   if (a.Sq_pad % a.block || a.Skv_pad % a.block) return VSA_ERR_SHAPE;
   const int nq = a.Sq_pad / a.block, nkv = a.Skv_pad / a.block;
   if (nq > VSA_MAX_BLOCKS || nkv > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
@@ -213,8 +213,9 @@ int launch_forward(const ForwardArgs& a, void* scratch, bool profile, cudaStream
   sp.scale_log2 = sc * kLog2e;
   sp.qk_bound = bound ? qk_bound : nullptr;
   sp.varlen = 0;
+  sp.sub = a.block == 256 ? 1 : 0;  // 256-slot blocks: two 128-row halves
   sp.status = status;
-  rc = a.block == 128
+  rc = a.block != 64
            ? launch_sparse128(sp, a.q, a.q_st, a.Sq_pad, a.k, a.k_st, a.v, a.v_st, a.Skv_pad, D,
                               /*combine=*/true, /*gated=*/a.gate != nullptr, st)
            : launch_sparse(sp, a.q, a.q_st, a.Sq_pad, a.k, a.k_st, a.v, a.v_st, a.Skv_pad, D,
@@ -344,7 +345,7 @@ static int sparse_from_indices(const void* q, const void* k, const void* v,
   if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || idx_stride < 1 || !(scale == scale))
     return VSA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
-  if (block != 64 && block != 128) return VSA_ERR_UNSUPPORTED;
+  if (block != 64 && block != 128 && block != 256) return VSA_ERR_UNSUPPORTED;
   if (Sq_pad % block || Skv_pad % block) return VSA_ERR_SHAPE;
   const int nq = Sq_pad / block, nkv = Skv_pad / block;
   if (idx_stride > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
@@ -363,7 +364,7 @@ static int sparse_from_indices(const void* q, const void* k, const void* v,
   if (!status) return VSA_ERR_CUDA;
   const float sc = resolve_scale(scale, D);
   const float* qk_bound = nullptr;
-  if (workspace && block == 64) {
+  if (workspace) {
     // logit bound of every item from block row norms and its selection
     BoundParams bp;
     memset(&bp, 0, sizeof(bp));
@@ -381,6 +382,7 @@ static int sparse_from_indices(const void* q, const void* k, const void* v,
     bp.H = H;
     bp.nqb = nq;
     bp.nkvb = nkv;
+    bp.block = block;
     bp.bound_scale = sc * kLog2e * (1.f + 0x1p-8f);
     bp.qn = static_cast<float*>(workspace);
     bp.kn = bp.qn + (size_t)B * H * nq;
@@ -407,7 +409,8 @@ static int sparse_from_indices(const void* q, const void* k, const void* v,
   sp.lse = lse;
   sp.lse_seq = Sq_pad;
   sp.status = status;
-  if (block == 128)
+  sp.sub = block == 256 ? 1 : 0;
+  if (block != 64)
     return launch_sparse128(sp, q, to_strides(L.q), Sq_pad, k, to_strides(L.k), v, to_strides(L.v),
                             Skv_pad, D, false, false, st);
   return launch_sparse(sp, q, to_strides(L.q), Sq_pad, k, to_strides(L.k), v, to_strides(L.v),
@@ -436,7 +439,7 @@ int block_sparse_attn(const void* q, const void* k, const void* v, const uint8_t
                       void* workspace, size_t workspace_bytes, void* stream) {
   if (!block_map || !q2k_idx || !q2k_num) return VSA_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0) return VSA_ERR_INVALID_ARG;
-  if (block_size != 64 && block_size != 128) return VSA_ERR_UNSUPPORTED;
+  if (block_size != 64 && block_size != 128 && block_size != 256) return VSA_ERR_UNSUPPORTED;
   if (Sq_pad % block_size || Skv_pad % block_size) return VSA_ERR_SHAPE;
   const int nq = Sq_pad / block_size, nkv = Skv_pad / block_size;
   if (nkv > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;

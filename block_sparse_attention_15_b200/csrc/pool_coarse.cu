@@ -24,13 +24,15 @@ namespace vsa {
 
 // ---------------------------------------------------------------------------
 // a1: pooling.  One CTA of 256 threads per (tensor, batch*head, block) of
-// BS slots (64 or 128).
+// BS slots (64, 128 or 256).
 // ---------------------------------------------------------------------------
 template <int D, int BS>
-__global__ void __launch_bounds__(256, 8) pool_kernel(PoolParams p) {
+__global__ void __launch_bounds__(256, BS == 64 ? 8 : 6) pool_kernel(PoolParams p) {
   constexpr int CPR = D / 8;          // 16-byte chunks per row
   constexpr int RPP = 256 / CPR;      // rows per pass
-  constexpr int PASSES = BS / RPP;
+  constexpr int CHUNK = 64;           // rows held in registers at a time
+  constexpr int PASSES = CHUNK / RPP;
+  static_assert(BS % CHUNK == 0, "block must be a multiple of 64 slots");
   __shared__ float red[RPP][D + 1];
   __shared__ float wmax[8];
 
@@ -65,57 +67,54 @@ __global__ void __launch_bounds__(256, 8) pool_kernel(PoolParams p) {
   const int lim = (nrm && all_rows) ? BS : m;  // rows read
   const int chunk = threadIdx.x % CPR;
   const int r0 = threadIdx.x / CPR;
+  // contiguous [B, H, S, D]: the block is BS consecutive rows; else the
+  // block's first slot in the strided view (item = group*nblocks + blk)
+  const bool contiguous = st.s == D && st.h == (long long)nblocks * BS * D && st.b == st.h * p.H;
+  const __nv_bfloat16* base = contiguous ? src + (long long)item * BS * D
+                                         : src + b * st.b + h * st.h + (long long)BS * blk * st.s;
+  const long long rstride = contiguous ? (long long)D : st.s;
 
-  uint4 buf[PASSES];
-  if (st.s == D && st.h == (long long)nblocks * BS * D && st.b == st.h * p.H) {
-    // contiguous [B, H, S, D]: the block is BS consecutive rows
-    const uint4* base = reinterpret_cast<const uint4*>(src) + (long long)item * BS * CPR + chunk;
-#pragma unroll
-    for (int ps = 0; ps < PASSES; ++ps) {
-      const int row = r0 + ps * RPP;
-      buf[ps] = row < lim ? __ldcs(base + row * CPR) : make_uint4(0u, 0u, 0u, 0u);
-    }
-  } else {
-    // first slot of the block in the strided view (item = group*nblocks + blk)
-    const __nv_bfloat16* base = src + b * st.b + h * st.h + (long long)BS * blk * st.s;
-#pragma unroll
-    for (int ps = 0; ps < PASSES; ++ps) {
-      const int row = r0 + ps * RPP;
-      buf[ps] = row < lim ? __ldcs(reinterpret_cast<const uint4*>(base + (long long)row * st.s) + chunk)
-                          : make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-  // block sums over the real rows and, per pass, this chunk's part of the
-  // row's squared norm (over every row read)
-  float acc[8], sq[PASSES];
+  // block sums over the real rows and the largest squared row norm (over
+  // every row read), 64 rows at a time with every load of a chunk issued
+  // before any use
+  float acc[8], mx = 0.f;
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  const uint4* rp = reinterpret_cast<const uint4*>(base + r0 * rstride) + chunk;
+  const long long pstride = rstride * RPP / 8;  // uint4 units between passes
+#pragma unroll 1
+  for (int c0 = 0; c0 < BS; c0 += CHUNK, rp += pstride * PASSES) {
+    if (c0 >= lim) break;
+    uint4 buf[PASSES];
 #pragma unroll
-  for (int ps = 0; ps < PASSES; ++ps) {
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&buf[ps]);
-    const bool real = r0 + ps * RPP < m;
-    sq[ps] = 0.f;
+    for (int ps = 0; ps < PASSES; ++ps) {
+      const int row = c0 + r0 + ps * RPP;
+      buf[ps] = row < lim ? __ldcs(rp + ps * pstride) : make_uint4(0u, 0u, 0u, 0u);
+    }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(h2[e]);
-      sq[ps] = fmaf(f.x, f.x, sq[ps]);
-      sq[ps] = fmaf(f.y, f.y, sq[ps]);
-      if (real) {
-        acc[2 * e] += f.x;
-        acc[2 * e + 1] += f.y;
+    for (int ps = 0; ps < PASSES; ++ps) {
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&buf[ps]);
+      const bool real = c0 + r0 + ps * RPP < m;
+      float sq = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        sq = fmaf(f.x, f.x, sq);
+        sq = fmaf(f.y, f.y, sq);
+        if (real) {
+          acc[2 * e] += f.x;
+          acc[2 * e + 1] += f.y;
+        }
+      }
+      if (nrm) {
+        // a row's CPR chunks sit in CPR consecutive lanes
+#pragma unroll
+        for (int o = CPR / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        mx = fmaxf(mx, sq);
       }
     }
   }
   if (nrm) {
-    // a row's CPR chunks sit in CPR consecutive lanes
-    float mx = 0.f;
-#pragma unroll
-    for (int ps = 0; ps < PASSES; ++ps) {
-      float t = sq[ps];
-#pragma unroll
-      for (int o = CPR / 2; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-      mx = fmaxf(mx, t);
-    }
 #pragma unroll
     for (int o = CPR; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = mx;
@@ -426,7 +425,10 @@ int launch_pool(const PoolParams& p, int D, cudaStream_t stream) {
   const long long items = (long long)p.groups * (p.nq + 2LL * p.nkv);
   if (items <= 0) return VSA_OK;
   if (items > 0x7FFFFFFFLL) return VSA_ERR_UNSUPPORTED;
-  if (p.block == 128) {
+  if (p.block == 256) {
+    if (D == 128) pool_kernel<128, 256><<<(unsigned)items, 256, 0, stream>>>(p);
+    else pool_kernel<64, 256><<<(unsigned)items, 256, 0, stream>>>(p);
+  } else if (p.block == 128) {
     if (D == 128) pool_kernel<128, 128><<<(unsigned)items, 256, 0, stream>>>(p);
     else pool_kernel<64, 128><<<(unsigned)items, 256, 0, stream>>>(p);
   } else {

@@ -127,24 +127,41 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
   }
 }
 
+// A work item: 128 query rows.  With blocks of 128 slots (p.sub = 0) it is
+// one query block and its selection, one tile per selected block.  With
+// blocks of 256 slots (p.sub = 1) it is one half of a query block: the tile
+// rows of the block's 256 slots split in two, each selected KV block read as
+// two 128-key sub-tiles (the second empty when the block holds at most 128
+// real keys), so both halves see exactly the block's selected keys.
 struct Item {
-  int a, h, b;
+  int a;        // 128-row tile index in the sequence
+  int ab;       // the caller's block index (a >> p.sub)
+  int h, b;
   long long group;
-  int num;
-  int q_len;
+  int num;      // 128-key tiles to process
+  int q_len;    // real query rows of the tile (0 .. 128)
 };
+
+__device__ __forceinline__ long long num_items(const SparseParams& p) {
+  return ((long long)p.B * p.H * p.nq) << p.sub;
+}
 
 __device__ __forceinline__ Item load_item(const SparseParams& p, long long it) {
   Item x;
-  x.a = (int)(it % p.nq);
-  const long long t = it / p.nq;
+  const long long per_group = (long long)p.nq << p.sub;
+  x.a = (int)(it % per_group);
+  x.ab = x.a >> p.sub;
+  const long long t = it / per_group;
   x.h = (int)(t % p.H);
   x.b = (int)(t / p.H);
   x.group = t;
-  const int num = p.q2k_num[t * p.nq + x.a];
-  x.num = num < 0 ? 0 : (num > p.idx_stride ? p.idx_stride : num);
-  const int ql = p.q_bs ? p.q_bs[x.a] : 128;
-  x.q_len = ql < 1 ? 0 : (ql > 128 ? 128 : ql);
+  const int num = p.q2k_num[t * p.nq + x.ab];
+  x.num = (num < 0 ? 0 : (num > p.idx_stride ? p.idx_stride : num)) << p.sub;
+  const int blk = 128 << p.sub;
+  int ql = p.q_bs ? p.q_bs[x.ab] : blk;
+  ql = ql < 1 ? 0 : (ql > blk ? blk : ql);
+  ql -= 128 * (x.a & ((1 << p.sub) - 1));
+  x.q_len = ql < 0 ? 0 : (ql > 128 ? 128 : ql);
   return x;
 }
 
@@ -176,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x;
   const int warp = tid / 32, lane = tid % 32;
-  const long long n_items = (long long)p.B * p.H * p.nq;
+  const long long n_items = num_items(p);
   const long long it0 = blockIdx.x, it_step = gridDim.x;
 
   if (tid == 0) {
@@ -218,10 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int qb = (int)(n & 1);
           if (n >= 2) ok = mbar_wait(bars + L::kQEmpty + qb, ((n - 2) >> 1) & 1, abort_flag, p.status);
           if (ok) {
-            const int raw = p.q2k_num[x.group * p.nq + x.a];
+            const int raw = p.q2k_num[x.group * p.nq + x.ab];
             if (raw < 0 || raw > p.idx_stride) set_status(p.status, VSA_ERR_INDEX_RANGE);
-            const int ql = p.q_bs ? p.q_bs[x.a] : 128;
-            if (ql < 1 || ql > 128) set_status(p.status, VSA_ERR_BLOCK_SIZE);
+            const int ql = p.q_bs ? p.q_bs[x.ab] : (128 << p.sub);
+            if (ql < 1 || ql > (128 << p.sub)) set_status(p.status, VSA_ERR_BLOCK_SIZE);
             mbar_arrive_expect_tx(bars + L::kQFull + qb, L::kTile);
 #pragma unroll
             for (int dh = 0; dh < L::DH; ++dh)
@@ -230,7 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        const int32_t* idx_row = p.q2k_idx + (x.group * p.nq + x.a) * (long long)p.idx_stride;
+        const int32_t* idx_row = p.q2k_idx + (x.group * p.nq + x.ab) * (long long)p.idx_stride;
+        const int smask = (1 << p.sub) - 1;
         for (int j = 0; ok && j < x.num; ++j, ++g) {
           if (lane == 0) {
             const int N = is_k ? NK : NV;
@@ -240,16 +258,22 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = mbar_wait(bars + (is_k ? L::kKEmpty : L::kVEmpty) + st, (u - 1) & 1, abort_flag,
                              p.status);
             if (ok) {
-              int c = idx_row[j], len = 0, row = 0;
+              // tile j: sub-tile (j & smask) of selected block j >> sub
+              const int part = j & smask;
+              int c = idx_row[j >> p.sub], len = 0, row = 0;
               if (c < 0 || c >= p.nkv) {
-                if (is_k) set_status(p.status, VSA_ERR_INDEX_RANGE);
+                if (is_k && part == 0) set_status(p.status, VSA_ERR_INDEX_RANGE);
               } else {
-                row = 128 * c;
-                len = p.kv_bs ? p.kv_bs[c] : 128;
-                if (len < 1 || len > 128) {
-                  if (is_k) set_status(p.status, VSA_ERR_BLOCK_SIZE);
+                row = 128 * ((c << p.sub) + part);
+                const int blk = 128 << p.sub;
+                len = p.kv_bs ? p.kv_bs[c] : blk;
+                if (len < 1 || len > blk) {
+                  if (is_k && part == 0) set_status(p.status, VSA_ERR_BLOCK_SIZE);
                   len = 0;
                 }
+                // the sub-tile's real keys (none in a second half past the block's end)
+                len -= 128 * part;
+                len = len < 0 ? 0 : (len > 128 ? 128 : len);
               }
               uint64_t* full = bars + (is_k ? L::kKFull : L::kVFull) + st;
               if (is_k) kmeta[st] = len;
@@ -369,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // once the first tile has fixed the row maxima and the bound keeps
       // every later logit within kBoundLimit of them, later tiles skip the
       // max exchange (same results: the reference max would not move)
-      const float qk_bound = p.qk_bound ? p.qk_bound[x.group * p.nq + x.a] : INFINITY;
+      const float qk_bound = p.qk_bound ? p.qk_bound[x.group * p.nq + x.ab] : INFINITY;
       bool novote = false;
       for (int j = 0; j < x.num; ++j, ++g) {
         const int sb = (int)(g & 1);
@@ -501,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __nv_bfloat16* orow = p.out + x.b * p.out_st.b + x.h * p.out_st.h + s * p.out_st.s;
       const __nv_bfloat16* grow =
           GATED ? p.gate + x.b * p.gate_st.b + x.h * p.gate_st.h + s * p.gate_st.s : nullptr;
-      const float* oc = COMBINE ? p.out_c + (x.group * p.nq + x.a) * (long long)D : nullptr;
+      const float* oc = COMBINE ? p.out_c + (x.group * p.nq + x.ab) * (long long)D : nullptr;
       const bool real = row < x.q_len;
 #pragma unroll
       for (int q0 = 0; q0 < D; q0 += 32) {
@@ -666,7 +690,7 @@ static int launch128_t(const SparseParams& p, const CUtensorMap& mq, const CUten
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long n_items = (long long)p.B * p.H * p.nq;
+  const long long n_items = ((long long)p.B * p.H * p.nq) << p.sub;
   const long long grid = n_items < sms ? n_items : sms;
   kern<<<(unsigned)grid, b128::kThreads, L::kAlloc, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
@@ -677,6 +701,7 @@ int launch_sparse128(const SparseParams& p_in, const void* q, Strides3 q_st, lon
                      int D, bool combine, bool gated, cudaStream_t stream) {
   if (p_in.nq <= 0 || p_in.H <= 0 || p_in.B <= 0) return VSA_OK;
   if (p_in.q_tok || p_in.kv_tok || p_in.varlen) return VSA_ERR_UNSUPPORTED;
+  if (p_in.sub < 0 || p_in.sub > 1) return VSA_ERR_UNSUPPORTED;
   if (q_seq + 128 > 0x7FFFFFFFLL || kv_seq + 128 > 0x7FFFFFFFLL) return VSA_ERR_UNSUPPORTED;
   SparseParams p = p_in;
   CUtensorMap mq, mk, mv;

@@ -89,6 +89,10 @@ struct SparseParams {
   float* lse;                 // [groups, lse_seq] natural-log log-sum-exp per query row, or null
   long long lse_seq;
   int varlen;                 // write only real rows
+  // 128-slot kernel only: log2 of the 128-slot sub-blocks per caller block
+  // (0: blocks of 128; 1: blocks of 256 walked as two 128-row halves, each
+  // selected block read as two 128-key sub-tiles)
+  int sub;
   int* status;
 };
 
@@ -171,6 +175,7 @@ struct BoundParams {
   const int32_t* q2k_num;     // [groups, nqb]
   int idx_stride;
   int B, H, nqb, nkvb;
+  int block;                  // slots per block (0: 64)
   float bound_scale;
   float* qn;                  // [groups, nqb]
   float* kn;                  // [groups, nkvb]

@@ -93,13 +93,14 @@ __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint4* src, ui
 }
 
 // Largest row L2 norm of one block per (group, block): query blocks over the
-// 64 slots from the block's first token (the rows the sparse kernel's query
-// tile holds, clipped at the end of the sequence), key blocks over their real
-// rows.  One CTA of 256 threads per (group, block); the squared norms of a
-// row's D/8 16-byte chunks add up across consecutive lanes.
+// block's slots from its first token (the rows the sparse kernel's query
+// tiles hold, clipped at the end of the sequence), key blocks over their real
+// rows.  One CTA of 256 threads per (group, block), 64 rows at a time; the
+// squared norms of a row's D/8 16-byte chunks add up across consecutive lanes.
 template <int D>
 __global__ void __launch_bounds__(256, 8) block_norm_kernel(BoundParams p) {
   constexpr int CPR = D / 8, RPP = 256 / CPR, PASSES = 64 / RPP;
+  const int bsz = p.block > 0 ? p.block : 64;
   __shared__ float wmax[8];
   const long long item = blockIdx.x;  // group * (nqb + nkvb) + block
   const int per_group = p.nqb + p.nkvb;
@@ -114,30 +115,32 @@ __global__ void __launch_bounds__(256, 8) block_norm_kernel(BoundParams p) {
   if (is_q) {
     base = p.q + b * p.q_st.b + h * p.q_st.h;
     st = p.q_st.s;
-    s0 = p.q_tok ? p.q_tok[blk] : 64LL * blk;
+    s0 = p.q_tok ? p.q_tok[blk] : (long long)bsz * blk;
     s_end = p.q_seq;
-    rows = 64;
+    rows = bsz;
     dst = p.qn + group * p.nqb + blk;
   } else {
     const int c = blk - p.nqb;
     base = p.k + b * p.k_st.b + h * p.k_st.h;
     st = p.k_st.s;
-    s0 = p.kv_tok ? p.kv_tok[c] : 64LL * c;
+    s0 = p.kv_tok ? p.kv_tok[c] : (long long)bsz * c;
     s_end = p.kv_seq;
-    rows = p.kv_len ? p.kv_len[c] : 64;
-    rows = rows < 0 ? 0 : (rows > 64 ? 64 : rows);
+    rows = p.kv_len ? p.kv_len[c] : bsz;
+    rows = rows < 0 ? 0 : (rows > bsz ? bsz : rows);
     dst = p.kn + group * p.nkvb + c;
   }
   const int chunk = threadIdx.x % CPR, r0 = threadIdx.x / CPR;
-  uint4 buf[PASSES];  // every load issued before any use
+  float mx = 0.f;
+#pragma unroll 1
+  for (int c0 = 0; c0 < rows; c0 += 64) {
+  uint4 buf[PASSES];  // every load of the chunk issued before any use
 #pragma unroll
   for (int ps = 0; ps < PASSES; ++ps) {
-    const int r = r0 + ps * RPP;
+    const int r = c0 + r0 + ps * RPP;
     buf[ps] = (r < rows && s0 + r < s_end)
                   ? __ldcs(reinterpret_cast<const uint4*>(base + (s0 + r) * st) + chunk)
                   : make_uint4(0u, 0u, 0u, 0u);
   }
-  float mx = 0.f;
 #pragma unroll
   for (int ps = 0; ps < PASSES; ++ps) {
     const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&buf[ps]);
@@ -151,6 +154,7 @@ __global__ void __launch_bounds__(256, 8) block_norm_kernel(BoundParams p) {
 #pragma unroll
     for (int o = CPR / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
     mx = fmaxf(mx, sq);
+  }
   }
 #pragma unroll
   for (int o = CPR; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));

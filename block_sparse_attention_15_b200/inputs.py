@@ -107,7 +107,7 @@ class Workload:
     gated: bool = True
     seed: int = 1000
     extra: dict = field(default_factory=dict)
-    block: int = BLOCK  # slots per block: 64, or 128 for VSA-128 tiles
+    block: int = BLOCK  # slots per block: 64, or 128 / 256 for VSA-128 / VSA-256 tiles
 
     @property
     def nq(self) -> int:
@@ -155,6 +155,14 @@ def workload_vsa128() -> Workload:
     nb = 39936 // 128
     return Workload("VSA-128: B1 H12 D128 S39936 (312 blocks of 128) top40 gated", 1, 12, 128,
                     [128] * nb, [128] * nb, 40, True, 1006, block=128)
+
+
+def workload_vsa256() -> Workload:
+    """The README's VSA-256 benchmark shape: B=1, H=12, D=128, 39936 tokens
+    in 156 blocks of 256 (256-token video tiles), top 20, gated."""
+    nb = 39936 // 256
+    return Workload("VSA-256: B1 H12 D128 S39936 (156 blocks of 256) top20 gated", 1, 12, 128,
+                    [256] * nb, [256] * nb, 20, True, 1007, block=256)
 
 
 VARLEN_Q_LENS = (3000, 6144, 9216, 15488)

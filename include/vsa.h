@@ -172,11 +172,15 @@ int vsa_forward(const void* q, const void* k, const void* v, const void* gate,
  * transposed gate view need no copy.  Same results as vsa_forward on the
  * same values at block_size 64.
  *
- * block_size  slots per block, 64 or 128.  With 128 ("VSA-128": 128-token
- *          video tiles), Sq_pad and Skv_pad are multiples of 128, block
- *          sizes lie in [1, 128], pooling and the coarse stage work on
+ * block_size  slots per block, 64, 128 or 256.  With 128 ("VSA-128":
+ *          128-token video tiles), Sq_pad and Skv_pad are multiples of 128,
+ *          block sizes lie in [1, 128], pooling and the coarse stage work on
  *          128-slot blocks and the sparse stage attends over 128 x 128
  *          tiles (a kernel shaped for the tensor core's native 128 rows).
+ *          With 256 ("VSA-256"), the same on 256-slot blocks (sizes in
+ *          [1, 256]); the sparse stage runs the 128-row kernel on each half
+ *          of a query block, reading every selected KV block as two 128-key
+ *          sub-tiles.
  *
  * Defined by: release 0.3.0, "Block-sparse / VSA attention improvements"
  * (the BSHD-native `video_sparse_attn_bshd` entry and the 128/256-token tile
@@ -308,11 +312,12 @@ int vsa_forward_host(const void* q, const void* k, const void* v, const void* ga
  *          its query norm times the largest key norm among the blocks it
  *          lists; where the bound shows no logit can exceed the first tile
  *          pair's maxima by 2^32, the sparse kernel skips its running-max
- *          check (same results, fewer instructions).  Without it every step
- *          keeps the check.
- *          (Block size 64 only; at 128 the workspace is not used.)
- * block_size  64 or 128 (see vsa_forward_strided); n_q_blocks = Sq_pad /
- *          block_size
+ *          check (fewer instructions; the same results at block size 64,
+ *          and at 128 / 256 equal up to rounding where a later tile would
+ *          have moved the running max).  Without it every step keeps the
+ *          check.
+ * block_size  64, 128 or 256 (see vsa_forward_strided); n_q_blocks =
+ *          Sq_pad / block_size
  * (ABI 2.0 added layout, block_size and workspace.)
  */
 size_t block_sparse_attn_from_indices_workspace_size(int B, int H, int n_q_blocks,

@@ -37,8 +37,9 @@ Readings where the pages leave a step open:
       row-major (t, h, w) token order inside a tile and clipped edge tiles;
   R12 varlen inputs are token-packed ``[H, sum(len), D]`` tensors delimited by
       cu_seqlens, and each sequence's ``q2k_idx`` rows hold local KV indices;
-  R14 with 128-token tiles every step is the same with blocks of 128 slots
-      (pooling over 128 tokens, selections of 128 x 128 tiles).
+  R14 with 128- or 256-token tiles every step is the same with blocks of 128
+      or 256 slots (pooling over the block's tokens, selections of block x
+      block tiles).
 """
 
 from __future__ import annotations
@@ -66,8 +67,8 @@ def block_pool(x, block_sizes, block: int = BLOCK) -> np.ndarray:
     [combine] Problem / Notes: the compression branch works on per-block means
     of q, k and v (the BSHD path takes an fp32 block sum).  Block ``j`` holds
     its ``block_sizes[j]`` real tokens in slots ``block*j ..``; padded slots
-    are not pooled (R5, R6).  ``block`` is the tile volume: 64, or 128 for the
-    128-token tiles of [readme] / [release] (R14).
+    are not pooled (R5, R6).  ``block`` is the tile volume: 64, or 128 / 256 for
+    the 128- and 256-token tiles of [readme] / [release] (R14).
 
     x: [B, H, block*n, D]  ->  [B, H, n, D] fp64
     """
@@ -156,8 +157,8 @@ def block_sparse_attention(q, k, v, q2k_idx, q2k_num, q_block_sizes, kv_block_si
     contributes twice); padded keys are excluded and padded query rows are 0
     (R6); ``q2k_num == 0`` gives 0 (R9).
 
-    q: [B,H,block*nq,D], k/v: [B,H,block*nkv,D] (block = 64, or 128 for the
-    128-token tiles, R14).  ``items`` optionally restricts the work to an
+    q: [B,H,block*nq,D], k/v: [B,H,block*nkv,D] (block = 64, or 128 / 256
+    for the larger tiles, R14).  ``items`` optionally restricts the work to an
     iterable of (b, h, query block) triples; other rows stay 0.
     Returns O_s [B,H,block*nq,D] fp64.
     """

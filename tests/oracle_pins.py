@@ -537,13 +537,13 @@ def check_block_map_to_indices(O):
     assert np.allclose(got[:, :, qr], want[:, :, qr], atol=1e-12)
 
 
-def check_block128(O):
-    """128-slot blocks (tile volume 128): pooling closed forms, the dense
-    limit against torch SDPA over the real tokens, arbitrary selections
-    against masked SDPA, the ungated combine as broadcast + sparse, and the
-    whole forward with topk = all equal to dense attention plus out_c."""
-    rng = _rng(31)
-    blk = 128
+def _check_large_block(O, blk, seed):
+    """Blocks of ``blk`` slots (tile volume 128 or 256): pooling closed forms,
+    the dense limit against torch SDPA over the real tokens, arbitrary
+    selections against masked SDPA, the ungated combine as broadcast +
+    sparse, and the whole forward with topk = all equal to dense attention
+    plus out_c."""
+    rng = _rng(seed)
     B, H, D = 1, 2, 16
 
     def padded(sizes, pad_value=0.0):
@@ -556,15 +556,16 @@ def check_block128(O):
         return np.concatenate([np.arange(blk * j, blk * j + m) for j, m in enumerate(sizes)])
 
     # pooling: a ramp over the real slots has the mean of its real values
-    sizes = [128, 70, 1]
+    part = blk // 2 + 6   # a partial block past the half (two sub-tiles at 256)
+    sizes = [blk, part, 1]
     x = np.zeros((1, 1, blk * 3, 1))
     for j, m in enumerate(sizes):
         x[0, 0, blk * j:blk * j + m, 0] = np.arange(m)
-    x[0, 0, blk * 1 + 70:blk * 2, 0] = 1e6   # padding must not count
+    x[0, 0, blk * 1 + part:blk * 2, 0] = 1e6   # padding must not count
     got = O.block_pool(x, sizes, block=blk)
     assert np.allclose(got[0, 0, :, 0], [(m - 1) / 2 for m in sizes])
     # dense limit, partial blocks, nq != nkv
-    q_sizes, kv_sizes = [128, 100], [128, 17, 128]
+    q_sizes, kv_sizes = [blk, blk - 28], [blk, 17, blk]
     q, k, v = padded(q_sizes), padded(kv_sizes, 7.0), padded(kv_sizes, -7.0)
     nkv = len(kv_sizes)
     idx = np.broadcast_to(np.arange(nkv, dtype=np.int32), (B, H, 2, nkv)).copy()
@@ -594,6 +595,16 @@ def check_block128(O):
     assert np.allclose(res["out"][:, :, qr], bcast + dense, atol=1e-12)
     pad = np.setdiff1d(np.arange(blk * 2), qr)
     assert np.all(res["out"][:, :, pad] == 0.0)
+
+
+def check_block128(O):
+    """128-slot blocks (VSA-128 tiles)."""
+    _check_large_block(O, 128, 31)
+
+
+def check_block256(O):
+    """256-slot blocks (VSA-256 tiles)."""
+    _check_large_block(O, 256, 37)
 
 
 def _torch_sparse_forward(q, k, v, idx, num, q_sizes, kv_sizes, scale, block=BLOCK):
@@ -681,5 +692,5 @@ ALL_CHECKS = [
     check_sparse_vs_masked_library, check_sparse_invariants, check_combine,
     check_forward_dense_limit, check_varlen_pack_indices, check_varlen_equals_per_sequence,
     check_varlen_dense_vs_library, check_metadata, check_page_figures,
-    check_block_map_to_indices, check_block128, check_backward,
+    check_block_map_to_indices, check_block128, check_block256, check_backward,
 ]

@@ -1,0 +1,197 @@
+"""256-token blocks (VSA-256 tiles) on the GPU, through the C ABI, against
+the fp64 oracle at block size 256.  The sparse stage runs the 128-row
+kernel on each half of a query block and reads every selected KV block as
+two 128-key sub-tiles, so the cases cover the halves' edges: query blocks
+with at most 128 real rows (an all-padding second half), KV blocks with at
+most 128 real keys (an empty second sub-tile), sizes just past the half,
+duplicates, empty selections, more work items than SMs, peaked logits that
+move the reference max, the whole forward stage by stage, the bool-mask and
+BSHD entries, and the README's VSA-256 shape (B1 H12 D128, 39936 tokens =
+156 blocks, top 20) on every query block."""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_15_b200 import binding as vsa
+from block_sparse_attention_15_b200 import inputs as I
+from oracle import vsa_oracle as O
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+BLK = 256
+
+
+def _padded(B, H, sizes, D, seed, stream, scale=1.0, pad_value=0.0):
+    x = I.normal_bf16((B, H, sum(sizes), D), seed, stream, scale=scale)
+    out = torch.full((B, H, BLK * len(sizes), D), pad_value, dtype=torch.bfloat16)
+    src = 0
+    for j, m in enumerate(sizes):
+        out[:, :, BLK * j:BLK * j + m] = x[:, :, src:src + m]
+        src += m
+    return out
+
+
+def _rows(sizes):
+    return np.concatenate([np.arange(BLK * j, BLK * j + m) for j, m in enumerate(sizes)])
+
+
+def _selection(rng, B, H, nq, nkv, width, allow_dup=False, empty=()):
+    idx = np.full((B, H, nq, width), -1, dtype=np.int32)
+    num = np.zeros((B, H, nq), dtype=np.int32)
+    for b, h, a in np.ndindex(B, H, nq):
+        if (b, h, a) in empty:
+            continue
+        n = int(rng.integers(1, width + 1))
+        sel = rng.integers(0, nkv, size=n) if allow_dup else rng.choice(nkv, size=min(n, nkv), replace=False)
+        idx[b, h, a, :len(sel)] = sel
+        num[b, h, a] = len(sel)
+    return idx, num
+
+
+CASES = [
+    # (D, B, H, q_sizes, kv_sizes, width, dup, seed)
+    (128, 1, 2, [256] * 4, [256] * 5, 3, False, 1),
+    (64, 2, 2, [256, 128, 129, 256], [256, 128, 129, 1, 256, 200], 4, False, 2),
+    (128, 1, 3, [256, 7], [256] * 2 + [100], 4, True, 3),
+    (128, 1, 1, [256] * 100, [256] * 6, 3, False, 4),   # 200 half-block items
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"D{c[0]}-B{c[1]}H{c[2]}-nq{len(c[3])}-nkv{len(c[4])}")
+def test_sparse256_from_indices(case):
+    D, B, H, qs, ks, width, dup, seed = case
+    rng = np.random.default_rng(seed)
+    q = _padded(B, H, qs, D, 700 + seed, 0, pad_value=3.0)
+    k = _padded(B, H, ks, D, 700 + seed, 1, pad_value=5.0)
+    v = _padded(B, H, ks, D, 700 + seed, 2, pad_value=-5.0)
+    idx, num = _selection(rng, B, H, len(qs), len(ks), width, dup, empty={(0, 0, 1)})
+    out = vsa.block_sparse_attn_from_indices(q.to(DEV), k.to(DEV), v.to(DEV), torch.from_numpy(idx).to(DEV),
+                                             torch.from_numpy(num).to(DEV), qs, ks, block=BLK)
+    vsa.check_device_status()
+    want = O.block_sparse_attention(P.to_np(q), P.to_np(k), P.to_np(v), idx, num, qs, ks,
+                                    O.default_scale(D), block=BLK)
+    got = P.to_np(out)
+    rr = _rows(qs)
+    P.assert_outputs_close(got[:, :, rr], want[:, :, rr], "sparse256")
+    pad = np.setdiff1d(np.arange(got.shape[2]), rr)
+    assert np.all(got[:, :, pad] == 0.0)
+    assert np.all(got[0, 0, BLK:BLK + qs[1]] == 0.0)   # the empty selection
+
+
+def test_sparse256_without_bound_pass_is_identical():
+    """The logit-bound pass only lets the kernel skip its max checks.  On
+    these N(0, 1) inputs no later sub-tile exceeds the first one's row maxima
+    by the refresh margin, so both runs take the same steps: the same bits."""
+    B, H, D = 1, 2, 128
+    qs, ks = [256, 256, 130], [256, 90, 256, 256]
+    q, k, v = (_padded(B, H, s, D, 760, i) for i, s in enumerate((qs, ks, ks)))
+    rng = np.random.default_rng(5)
+    idx, num = _selection(rng, B, H, 3, 4, 3)
+    args = (q.to(DEV), k.to(DEV), v.to(DEV), torch.from_numpy(idx).to(DEV), torch.from_numpy(num).to(DEV),
+            qs, ks)
+    o1 = vsa.block_sparse_attn_from_indices(*args, block=BLK)
+    o2 = vsa.block_sparse_attn_from_indices(*args, block=BLK, logit_bound=False)
+    vsa.check_device_status()
+    assert torch.equal(o1, o2)
+
+
+def test_sparse256_peaked_logits_move_the_reference():
+    """q x 6 and the keys of later blocks x 4: later sub-tiles exceed the
+    first sub-tile's maxima by far more than the refresh threshold."""
+    B, H, D = 1, 2, 128
+    qs, ks = [256] * 2, [256] * 5
+    q = _padded(B, H, qs, D, 801, 0, scale=6.0)
+    k = _padded(B, H, ks, D, 801, 1)
+    k[:, :, 2 * BLK + 128:] *= 4
+    v = _padded(B, H, ks, D, 801, 2)
+    idx = np.broadcast_to(np.arange(5, dtype=np.int32), (B, H, 2, 5)).copy()
+    num = np.full((B, H, 2), 5, dtype=np.int32)
+    out = vsa.block_sparse_attn_from_indices(q.to(DEV), k.to(DEV), v.to(DEV), torch.from_numpy(idx).to(DEV),
+                                             torch.from_numpy(num).to(DEV), block=BLK)
+    vsa.check_device_status()
+    want = O.block_sparse_attention(P.to_np(q), P.to_np(k), P.to_np(v), idx, num, qs, ks,
+                                    O.default_scale(D), block=BLK)
+    P.assert_outputs_close(P.to_np(out), want, "sparse256 peaked")
+
+
+FWD_CASES = [
+    (128, True, [256] * 5, [256] * 7, 3, 21),
+    (128, False, [256, 256, 256, 50], [256, 60, 256, 256, 140], 2, 22),
+    (64, True, [256] * 3 + [1], [256] * 4, 4, 23),
+]
+
+
+@pytest.mark.parametrize("case", FWD_CASES, ids=lambda c: f"D{c[0]}-{'gated' if c[1] else 'ungated'}-nq{len(c[2])}")
+def test_forward256(case):
+    D, gated, qs, ks, topk, seed = case
+    B, H = 1, 3
+    q, k, v = (_padded(B, H, s, D, 960 + seed, i) for i, s in enumerate((qs, ks, ks)))
+    gate = I.gate_bf16((B, BLK * len(qs), H, D), 960 + seed) if gated else None
+    out, idx, num, out_c, pooled = vsa.vsa_forward(
+        q.to(DEV), k.to(DEV), v.to(DEV), None if gate is None else gate.to(DEV), qs, ks, topk=topk,
+        return_out_c=True, return_pooled=True, block=BLK)
+    vsa.check_device_status()
+    qn, kn, vn = P.to_np(q), P.to_np(k), P.to_np(v)
+    scale = O.default_scale(D)
+    for got_p, x, sizes in zip(pooled, (qn, kn, vn), (qs, ks, ks)):
+        np.testing.assert_allclose(P.to_np(got_p), O.block_pool(x, sizes, block=BLK), rtol=1e-5, atol=1e-6)
+    qc, kc, vc = (O.block_pool(x, s, block=BLK) for x, s in ((qn, qs), (kn, ks), (vn, ks)))
+    scores, oc = O.coarse_attention(qc, kc, vc, scale)
+    np.testing.assert_allclose(P.to_np(out_c), oc, rtol=1e-4, atol=1e-6)
+    P.check_topk(P.to_np(idx), P.to_np(num), scores, topk)
+    o_s = O.block_sparse_attention(qn, kn, vn, P.to_np(idx), P.to_np(num), qs, ks, scale, block=BLK)
+    want = O.combine(oc, o_s, None if gate is None else P.to_np(gate), qs, block=BLK)
+    got = P.to_np(out)
+    rr = _rows(qs)
+    P.assert_outputs_close(got[:, :, rr], want[:, :, rr], "forward256")
+    pad = np.setdiff1d(np.arange(got.shape[2]), rr)
+    assert np.all(got[:, :, pad] == 0.0)
+
+
+def test_block256_bool_mask_and_bshd():
+    B, H, D = 1, 2, 128
+    qs, ks = [256] * 3, [256] * 5
+    q, k, v = (_padded(B, H, s, D, 995, i) for i, s in enumerate((qs, ks, ks)))
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    rng = np.random.default_rng(19)
+    bm = rng.random((B, H, 3, 5)) < 0.4
+    bm[0, 1, 2] = False
+    out, idx, num = vsa.block_sparse_attn(qd, kd, vd, torch.from_numpy(bm).to(DEV), block=BLK,
+                                          return_indices=True)
+    ref = vsa.block_sparse_attn_from_indices(qd, kd, vd, idx, num, block=BLK)
+    vsa.check_device_status()
+    wi, wn = O.block_map_to_indices(bm)
+    assert np.array_equal(P.to_np(idx), wi) and np.array_equal(P.to_np(num), wn)
+    assert torch.equal(out, ref)
+    gate = I.gate_bf16((B, BLK * 3, H, D), 996).to(DEV)
+    o1, i1, n1 = vsa.vsa_forward(qd, kd, vd, gate, topk=2, block=BLK)
+    qb, kb, vb = (x.transpose(1, 2).contiguous() for x in (qd, kd, vd))
+    o2, i2, n2 = vsa.video_sparse_attn_bshd(qb, kb, vb, gate, topk=2, block=BLK)
+    vsa.check_device_status()
+    assert torch.equal(i1, i2) and torch.equal(n1, n2)
+    assert torch.equal(o2.transpose(1, 2), o1)
+
+
+def test_vsa256_readme_shape_full():
+    """The README's VSA-256 benchmark shape: B1 H12 D128, 39936 tokens
+    (156 blocks of 256), top 20, gated; every query block against the
+    oracle."""
+    wl = I.workload_vsa256()
+    B, H, D, nb, topk, seed = wl.B, wl.H, wl.D, wl.nq, wl.topk, wl.seed
+    sizes = wl.q_block_sizes
+    q, k, v = (_padded(B, H, sizes, D, seed, i) for i in range(3))
+    gate = I.gate_bf16((B, BLK * nb, H, D), seed)
+    out, idx, num, out_c = vsa.vsa_forward(q.to(DEV), k.to(DEV), v.to(DEV), gate.to(DEV), topk=topk,
+                                           return_out_c=True, block=BLK)
+    vsa.check_device_status()
+    qn, kn, vn = P.to_np(q), P.to_np(k), P.to_np(v)
+    scale = O.default_scale(D)
+    qc, kc, vc = (O.block_pool(x, sizes, block=BLK) for x in (qn, kn, vn))
+    scores, oc = O.coarse_attention(qc, kc, vc, scale)
+    np.testing.assert_allclose(P.to_np(out_c), oc, rtol=1e-4, atol=1e-6)
+    idx_np, num_np = P.to_np(idx), P.to_np(num)
+    P.check_topk(idx_np, num_np, scores, topk)
+    o_s = O.block_sparse_attention(qn, kn, vn, idx_np, num_np, sizes, sizes, scale, block=BLK)
+    want = O.combine(oc, o_s, P.to_np(gate), sizes, block=BLK)
+    P.assert_outputs_close(P.to_np(out), want, "VSA-256 README shape")
