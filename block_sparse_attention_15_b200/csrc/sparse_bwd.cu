@@ -173,27 +173,57 @@ __global__ void __launch_bounds__(256) k2q_kernel(const int32_t* q2k_idx, const 
 // --------------------------------------------------------------------------
 // dq kernel
 // --------------------------------------------------------------------------
+// K pairs stay in shared memory until the dQ product of their pair (late);
+// V pairs only until the dP product (early).  So the K ring is one stage
+// deeper than the V ring, and each ring has its own barriers.
+constexpr int kDqNK = 3, kDqNV = 2;
+
 template <int D>
 struct DqLayout {
   static constexpr uint32_t kTile = 64u * D * 2u;   // one 64-row tile
   static constexpr uint32_t kPair = 2u * kTile;
   static constexpr uint32_t kQOff = 0;              // Q tile
   static constexpr uint32_t kDOOff = kQOff + kTile; // dO tile
-  static constexpr uint32_t kKOff = kDOOff + kTile; // [2] K pairs
-  static constexpr uint32_t kVOff = kKOff + 2 * kPair;  // [2] V pairs
-  static constexpr uint32_t kSOff = kVOff + 2 * kPair;  // [2] dS^T [128][64] bf16
-  static constexpr uint32_t kStageOff = kSOff + 2u * 16384u;   // epilogue tile [16][D] f32
-  static constexpr uint32_t kMetaOff = kStageOff + 16u * D * 4u;  // [2] int2 key counts per stage
-  static constexpr uint32_t kSMetaOff = kMetaOff + 16u;            // [2] int2 per TMEM buffer
+  static constexpr uint32_t kKOff = kDOOff + kTile; // [kDqNK] K pairs
+  static constexpr uint32_t kVOff = kKOff + kDqNK * kPair;  // [kDqNV] V pairs
+  static constexpr uint32_t kSOff = kVOff + kDqNV * kPair;  // [2] dS^T [128][64] bf16
+  static constexpr uint32_t kMetaOff = kSOff + 2u * 16384u;  // [kDqNK] int2 key counts per K stage
+  static constexpr uint32_t kSMetaOff = kMetaOff + 32u;      // [2] int2 per TMEM buffer
   static constexpr uint32_t kBarOff = kSMetaOff + 16u;
-  static constexpr int kQFull = 0, kQEmpty = 1, kKVFull = 2, kKVEmpty = 4, kSPFull = 6,
-                       kSPEmpty = 8, kDSFull = 10, kDSEmpty = 12, kOFull = 14, kOEmpty = 16,
-                       kNumBars = 18;
+  static constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + kDqNK,
+                       kVFull = kKEmpty + kDqNK, kVEmpty = kVFull + kDqNV,
+                       kSPFull = kVEmpty + kDqNV, kSPEmpty = kSPFull + 2, kDSFull = kSPEmpty + 2,
+                       kDSEmpty = kDSFull + 2, kOFull = kDSEmpty + 2, kOEmpty = kOFull + 2,
+                       kNumBars = kOEmpty + 2;
   static constexpr uint32_t kMiscOff = kBarOff + 8u * kNumBars;
   static constexpr uint32_t kAlloc = kMiscOff + 16u + 1024u;
   static_assert(kKOff % 1024 == 0 && kSOff % 1024 == 0, "1 KB atoms");
   static_assert(kAlloc <= 227u * 1024u, "shared memory");
 };
+
+// Epilogue helper: this thread holds column d of a transposed accumulator
+// (TMEM lane d, 16 consecutive rows q0 .. q0+15 of the output in v[]).  Lane
+// pairs swap values so that each lane writes one 4-byte word (two adjacent
+// head dims of one row) per two rows: a warp's stores of one row cover 64
+// consecutive bytes.  Rows at or past `len` are written as 0 unless `skip_pad`.
+__device__ __forceinline__ void store_cols_t(__nv_bfloat16* col_d_row0, long long row_stride,
+                                             const float (&v)[16], int q0, int len, bool skip_pad,
+                                             int lane) {
+  const bool odd = lane & 1;
+#pragma unroll
+  for (int j = 0; j < 16; j += 2) {
+    const float send = odd ? v[j] : v[j + 1];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+    // even lane: row j, head dims (d, d + 1); odd lane: row j + 1, (d - 1, d)
+    const int q = q0 + j + (odd ? 1 : 0);
+    const uint32_t word = odd ? pack_bf16x2(recv, v[j + 1]) : pack_bf16x2(v[j], recv);
+    __nv_bfloat16* dst = col_d_row0 + (long long)q * row_stride - (odd ? 1 : 0);
+    if (q < len)
+      *reinterpret_cast<uint32_t*>(dst) = word;
+    else if (!skip_pad)
+      *reinterpret_cast<uint32_t*>(dst) = 0u;
+  }
+}
 
 struct BwdItem {
   int a, h, b;
@@ -304,24 +334,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int np = (x.num + 1) / 2;
         for (int i = 0; ok && i < np; ++i, ++g) {
           if (lane == 0) {
-            const int st = (int)(g & 1);
-            if (g >= 2) ok = mbar_wait(bars + L::kKVEmpty + st, ((g - 2) >> 1) & 1, abort_flag, p.status);
+            const int ks = (int)(g % kDqNK), vs = (int)(g % kDqNV);
+            const uint32_t ku = g / kDqNK, vu = g / kDqNV;
+            if (ku >= 1) ok = mbar_wait(bars + L::kKEmpty + ks, (ku - 1) & 1, abort_flag, p.status);
+            if (ok && vu >= 1) ok = mbar_wait(bars + L::kVEmpty + vs, (vu - 1) & 1, abort_flag, p.status);
             if (ok) {
               int r0, l0, r1, l1;
               resolve_kv(p, x, 2 * i, r0, l0);
               resolve_kv(p, x, 2 * i + 1, r1, l1);
               if (2 * i + 1 >= x.num) { r1 = r0; l1 = 0; }
-              meta[st] = make_int2(l0, l1);
-              uint64_t* full = bars + L::kKVFull + st;
-              mbar_arrive_expect_tx(full, 2 * L::kPair);
+              meta[ks] = make_int2(l0, l1);
+              uint64_t* kfull = bars + L::kKFull + ks;
+              uint64_t* vfull = bars + L::kVFull + vs;
+              mbar_arrive_expect_tx(kfull, L::kPair);
+              mbar_arrive_expect_tx(vfull, L::kPair);
+              uint8_t* kd = smem + L::kKOff + ks * L::kPair;
+              uint8_t* vd = smem + L::kVOff + vs * L::kPair;
 #pragma unroll
               for (int dh = 0; dh < D / 64; ++dh) {
-                uint8_t* kd = smem + L::kKOff + st * L::kPair;
-                uint8_t* vd = smem + L::kVOff + st * L::kPair;
-                load_tile64(kd + pair_off(dh, 0), &tm_k, p.k_ax, full, dh * 64, r0, x.h, x.b);
-                load_tile64(kd + pair_off(dh, 1), &tm_k, p.k_ax, full, dh * 64, r1, x.h, x.b);
-                load_tile64(vd + pair_off(dh, 0), &tm_v, p.v_ax, full, dh * 64, r0, x.h, x.b);
-                load_tile64(vd + pair_off(dh, 1), &tm_v, p.v_ax, full, dh * 64, r1, x.h, x.b);
+                load_tile64(kd + pair_off(dh, 0), &tm_k, p.k_ax, kfull, dh * 64, r0, x.h, x.b);
+                load_tile64(kd + pair_off(dh, 1), &tm_k, p.k_ax, kfull, dh * 64, r1, x.h, x.b);
+              }
+#pragma unroll
+              for (int dh = 0; dh < D / 64; ++dh) {
+                load_tile64(vd + pair_off(dh, 0), &tm_v, p.v_ax, vfull, dh * 64, r0, x.h, x.b);
+                load_tile64(vd + pair_off(dh, 1), &tm_v, p.v_ax, vfull, dh * 64, r1, x.h, x.b);
               }
             }
           }
@@ -329,8 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (ok && lane == 0) {
-        for (uint32_t t = (g > 2u ? g - 2u : 0u); t < g; ++t)
-          if (!mbar_wait(bars + L::kKVEmpty + (int)(t & 1), (t >> 1) & 1, abort_flag, p.status)) break;
+        // drain: every stage's release (a tcgen05 commit) lands before exit
+        for (uint32_t t = (g > (uint32_t)kDqNK ? g - kDqNK : 0u); t < g; ++t)
+          if (!mbar_wait(bars + L::kKEmpty + (int)(t % kDqNK), (t / kDqNK) & 1, abort_flag, p.status)) break;
+        for (uint32_t t = (g > (uint32_t)kDqNV ? g - kDqNV : 0u); t < g; ++t)
+          if (!mbar_wait(bars + L::kVEmpty + (int)(t % kDqNV), (t / kDqNV) & 1, abort_flag, p.status)) break;
         if (n >= 1) mbar_wait(bars + L::kQEmpty, (n - 1) & 1, abort_flag, p.status);
       }
       __syncwarp();
@@ -348,15 +388,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (i < np) {
             const uint32_t t = g0 + i;
             const int st = (int)(t & 1);
-            if (!warp_wait(bars + L::kKVFull + st, (t >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            const int ks = (int)(t % kDqNK), vs = (int)(t % kDqNV);
+            if (!warp_wait(bars + L::kKFull + ks, (t / kDqNK) & 1, abort_flag, p.status)) { ok = false; break; }
+            if (!warp_wait(bars + L::kVFull + vs, (t / kDqNV) & 1, abort_flag, p.status)) { ok = false; break; }
             if (t >= 2 && !warp_wait(bars + L::kSPEmpty + st, ((t - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-            if (lane == 0) smeta[st] = meta[st];
+            if (lane == 0) smeta[st] = meta[ks];
             __syncwarp();
             tc_fence_after_sync();
             if (elect_one()) {
-              mma_pair_single<D>(tmem + 64u * st, sbase + L::kKOff + st * L::kPair, sbase + L::kQOff);
-              mma_pair_single<D>(tmem + 128u + 64u * st, sbase + L::kVOff + st * L::kPair, sbase + L::kDOOff);
+              mma_pair_single<D>(tmem + 64u * st, sbase + L::kKOff + ks * L::kPair, sbase + L::kQOff);
+              mma_pair_single<D>(tmem + 128u + 64u * st, sbase + L::kVOff + vs * L::kPair, sbase + L::kDOOff);
               umma_commit(bars + L::kSPFull + st);
+              umma_commit(bars + L::kVEmpty + vs);   // V is read by dP only
               if (i == np - 1) umma_commit(bars + L::kQEmpty);
             }
             __syncwarp();
@@ -365,14 +408,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (i >= 1) {
             const uint32_t t = g0 + i - 1;
             const int st = (int)(t & 1);
+            const int ks = (int)(t % kDqNK);
             if (i == 1 && n >= 2 && !warp_wait(bars + L::kOEmpty + o, ((n - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
             if (!warp_wait(bars + L::kDSFull + st, (t >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after_sync();
             if (elect_one()) {
-              mma_pairT_mn<D>(tmem + 256u + 64u * o, sbase + L::kKOff + st * L::kPair,
+              mma_pairT_mn<D>(tmem + 256u + 64u * o, sbase + L::kKOff + ks * L::kPair,
                               sbase + L::kSOff + st * 16384u, i > 1);
               umma_commit(bars + L::kDSEmpty + st);
-              umma_commit(bars + L::kKVEmpty + st);
+              umma_commit(bars + L::kKEmpty + ks);
               if (i == np) umma_commit(bars + L::kOFull + o);
             }
             __syncwarp();
@@ -461,14 +505,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     regs_dec<kRegsEpilogue>();
     // ===================== epilogue: scale * dQ^T -> dq rows =====================
+    // thread = head dim d (TMEM lane of dQ^T); rows straight from registers
     const int wq = warp & 3;
     const int d = wq * 32 + lane;
-    const int t128 = (warp - 12) * 32 + lane;
     const uint32_t t_lane = tmem + (uint32_t(wq * 32) << 16);
     const bool active = wq * 32 < D;
-    float* stage = reinterpret_cast<float*>(smem + L::kStageOff);   // [16][D]
-    constexpr int kPerThread = 16 * D / 4 / 128;
-    const int d0 = (t128 % (D / 4)) * 4;
     uint32_t n = 0;
     for (long long it = it0; it < n_items; it += it_step, ++n) {
       const BwdItem x = load_q_item(p, it);
@@ -476,39 +517,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool bad = !warp_wait(bars + L::kOFull + o, (n >> 1) & 1, abort_flag, p.status);
       if (bar_red_or(5, 128, bad)) break;
       tc_fence_after_sync();
-      __nv_bfloat16* orow0 = p.dq + x.b * p.dq_st.b + x.h * p.dq_st.h + x.q_tok * p.dq_st.s + d0;
+      __nv_bfloat16* col = p.dq + x.b * p.dq_st.b + x.h * p.dq_st.h + x.q_tok * p.dq_st.s + d;
       for (int rnd = 0; rnd < 4; ++rnd) {
-        if (active) {
-          uint32_t ov[16];
-          if (x.num > 0) {
-            VSA_TMEM_LD16(t_lane + 256u + 64u * o + 16u * rnd, ov, 0);
-            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-          } else {
+        uint32_t ov[16];
 #pragma unroll
-            for (int q = 0; q < 16; ++q) ov[q] = 0u;
-          }
-#pragma unroll
-          for (int q = 0; q < 16; ++q) stage[q * D + d] = __uint_as_float(ov[q]) * p.scale;
+        for (int q = 0; q < 16; ++q) ov[q] = 0u;
+        if (active && x.num > 0) {
+          VSA_TMEM_LD16(t_lane + 256u + 64u * o + 16u * rnd, ov, 0);
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
         }
         if (rnd == 3) {
+          // the last read of this dQ^T buffer: hand it back before the stores
           tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(bars + L::kOEmpty + o);
         }
-        named_barrier_sync(5, 128);
+        if (active) {
+          float v[16];
 #pragma unroll
-        for (int k = 0; k < kPerThread; ++k) {
-          const int cidx = t128 + 128 * k;
-          const int rowi = cidx / (D / 4);
-          const int q = 16 * rnd + rowi;
-          const float4 v4 = *reinterpret_cast<const float4*>(stage + rowi * D + d0);
-          if (q < x.q_len)
-            *reinterpret_cast<uint2*>(orow0 + q * p.dq_st.s) =
-                make_uint2(pack_bf16x2(v4.x, v4.y), pack_bf16x2(v4.z, v4.w));
-          else if (!p.varlen)
-            *reinterpret_cast<uint2*>(orow0 + q * p.dq_st.s) = make_uint2(0u, 0u);
+          for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(ov[q]) * p.scale;
+          store_cols_t(col, p.dq_st.s, v, 16 * rnd, x.q_len, p.varlen != 0, lane);
         }
-        named_barrier_sync(5, 128);
       }
     }
   }
@@ -531,15 +560,14 @@ struct DkvLayout {
   static constexpr uint32_t kVOff = kKOff + kTile;       // V tile
   static constexpr uint32_t kQOff = kVOff + kTile;       // [2] Q pairs (two query blocks)
   static constexpr uint32_t kDOOff = kQOff + 2 * kPair;  // [2] dO pairs
-  static constexpr uint32_t kPOff = kDOOff + 2 * kPair;  // P [128][64] bf16
-  static constexpr uint32_t kSOff = kPOff + 16384u;      // dS [128][64] bf16
-  static constexpr uint32_t kStageOff = kSOff + 16384u;  // epilogue tile [16][D] f32
-  static constexpr uint32_t kMetaOff = kStageOff + 16u * D * 4u;  // [2] int4: blocks, multiplicities
-  static constexpr uint32_t kSMetaOff = kMetaOff + 32u;           // [2] int4 per TMEM buffer
+  static constexpr uint32_t kPOff = kDOOff + 2 * kPair;  // [2] P [128][64] bf16
+  static constexpr uint32_t kSOff = kPOff + 2u * 16384u; // [2] dS [128][64] bf16
+  static constexpr uint32_t kMetaOff = kSOff + 2u * 16384u;  // [2] int4: blocks, multiplicities
+  static constexpr uint32_t kSMetaOff = kMetaOff + 32u;      // [2] int4 per TMEM buffer
   static constexpr uint32_t kBarOff = kSMetaOff + 32u;
   static constexpr int kKVFull = 0, kKVEmpty = 1, kQFull = 2, kQEmpty = 4, kSPFull = 6,
-                       kSPEmpty = 8, kPSFull = 10, kPSEmpty = 11, kOFull = 12, kOEmpty = 14,
-                       kNumBars = 16;
+                       kSPEmpty = 8, kPSFull = 10, kPSEmpty = 12, kOFull = 14, kOEmpty = 16,
+                       kNumBars = 18;
   static constexpr uint32_t kMiscOff = kBarOff + 8u * kNumBars;
   static constexpr uint32_t kAlloc = kMiscOff + 16u + 1024u;
   static_assert(kQOff % 1024 == 0 && kPOff % 1024 == 0, "1 KB atoms");
@@ -590,7 +618,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < L::kNumBars; ++i) {
       uint32_t count = 1;
-      if (i == L::kSPEmpty || i == L::kSPEmpty + 1 || i == L::kPSFull) count = 8;
+      if (i == L::kSPEmpty || i == L::kSPEmpty + 1 || i == L::kPSFull || i == L::kPSFull + 1)
+        count = 8;
       if (i == L::kOEmpty || i == L::kOEmpty + 1) count = 4;
       if (i == L::kSPFull || i == L::kSPFull + 1) count = 2;
       mbar_init(bars + i, count);
@@ -701,12 +730,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t t = g0 + i - 1;
             const int st = (int)(t & 1);
             if (i == 1 && n >= 2 && !warp_wait(bars + L::kOEmpty + o, ((n - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-            if (!warp_wait(bars + L::kPSFull, t & 1, abort_flag, p.status)) { ok = false; break; }
+            if (!warp_wait(bars + L::kPSFull + st, (t >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after_sync();
             if (elect_one()) {
-              mma_pairT_mn<D>(tmem + 256u + 64u * o, sbase + L::kDOOff + st * L::kPair, sbase + L::kPOff, i > 1);
-              mma_pairT_mn<D>(tmem + 384u + 64u * o, sbase + L::kQOff + st * L::kPair, sbase + L::kSOff, i > 1);
-              umma_commit(bars + L::kPSEmpty);
+              mma_pairT_mn<D>(tmem + 256u + 64u * o, sbase + L::kDOOff + st * L::kPair,
+                              sbase + L::kPOff + st * 16384u, i > 1);
+              mma_pairT_mn<D>(tmem + 384u + 64u * o, sbase + L::kQOff + st * L::kPair,
+                              sbase + L::kSOff + st * 16384u, i > 1);
+              umma_commit(bars + L::kPSEmpty + st);
               umma_commit(bars + L::kQEmpty + st);
               if (i == np) {
                 umma_commit(bars + L::kOFull + o);
@@ -784,31 +815,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           pp[q] = pack_bf16x2(p0, p1);
           ps[q] = pack_bf16x2(d0, d1);
         }
-        // P and dS buffers are free once the products of step g - 1 are done
-        if (g >= 1) wwait(bars + L::kPSEmpty, (g - 1) & 1);
+        // this P / dS buffer pair is free once the products of step g - 2 are done
+        if (g >= 2) wwait(bars + L::kPSEmpty + st, ((g - 2) >> 1) & 1);
+        uint8_t* pbuf = smem + L::kPOff + st * 16384u;
+        uint8_t* sbuf = smem + L::kSOff + st * 16384u;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
-          *reinterpret_cast<uint4*>(smem + L::kPOff + sw128(row, 4 * grp + ch)) =
+          *reinterpret_cast<uint4*>(pbuf + sw128(row, 4 * grp + ch)) =
               make_uint4(pp[4 * ch], pp[4 * ch + 1], pp[4 * ch + 2], pp[4 * ch + 3]);
-          *reinterpret_cast<uint4*>(smem + L::kSOff + sw128(row, 4 * grp + ch)) =
+          *reinterpret_cast<uint4*>(sbuf + sw128(row, 4 * grp + ch)) =
               make_uint4(ps[4 * ch], ps[4 * ch + 1], ps[4 * ch + 2], ps[4 * ch + 3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bars + L::kPSFull);
+        if (lane == 0) mbar_arrive(bars + L::kPSFull + st);
       }
     }
   } else {
     regs_dec<kRegsEpilogue>();
     // ===================== epilogue: dV^T, scale * dK^T -> dv, dk rows =====================
+    // thread = head dim d (TMEM lane of dV^T / dK^T); rows straight from registers
     const int wq = warp & 3;
     const int d = wq * 32 + lane;
-    const int t128 = (warp - 12) * 32 + lane;
     const uint32_t t_lane = tmem + (uint32_t(wq * 32) << 16);
     const bool active = wq * 32 < D;
-    float* stage = reinterpret_cast<float*>(smem + L::kStageOff);
-    constexpr int kPerThread = 16 * D / 4 / 128;
-    const int d0 = (t128 % (D / 4)) * 4;
     uint32_t n = 0;
     for (long long it = it0; it < n_items; it += it_step, ++n) {
       const KvItem x = load_kv_item(p, it);
@@ -818,40 +848,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after_sync();
       for (int which = 0; which < 2; ++which) {
         const Strides3 st = which ? p.dk_st : p.dv_st;
-        __nv_bfloat16* base = (which ? p.dk : p.dv) + x.b * st.b + x.h * st.h + x.kv_tok * st.s + d0;
+        __nv_bfloat16* col = (which ? p.dk : p.dv) + x.b * st.b + x.h * st.h + x.kv_tok * st.s + d;
         const float mul = which ? p.scale : 1.f;
         for (int rnd = 0; rnd < 4; ++rnd) {
-          if (active) {
-            uint32_t ov[16];
-            if (x.num > 0) {
-              VSA_TMEM_LD16(t_lane + 256u + 128u * which + 64u * o + 16u * rnd, ov, 0);
-              asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-            } else {
+          uint32_t ov[16];
 #pragma unroll
-              for (int q = 0; q < 16; ++q) ov[q] = 0u;
-            }
-#pragma unroll
-            for (int q = 0; q < 16; ++q) stage[q * D + d] = __uint_as_float(ov[q]) * mul;
+          for (int q = 0; q < 16; ++q) ov[q] = 0u;
+          if (active && x.num > 0) {
+            VSA_TMEM_LD16(t_lane + 256u + 128u * which + 64u * o + 16u * rnd, ov, 0);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
           }
           if (which == 1 && rnd == 3) {
+            // the last read of this output buffer pair: hand it back
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars + L::kOEmpty + o);
           }
-          named_barrier_sync(5, 128);
+          if (active) {
+            float v[16];
 #pragma unroll
-          for (int k = 0; k < kPerThread; ++k) {
-            const int cidx = t128 + 128 * k;
-            const int rowi = cidx / (D / 4);
-            const int q = 16 * rnd + rowi;
-            const float4 v4 = *reinterpret_cast<const float4*>(stage + rowi * D + d0);
-            if (q < x.kv_len)
-              *reinterpret_cast<uint2*>(base + q * st.s) =
-                  make_uint2(pack_bf16x2(v4.x, v4.y), pack_bf16x2(v4.z, v4.w));
-            else if (!p.varlen)
-              *reinterpret_cast<uint2*>(base + q * st.s) = make_uint2(0u, 0u);
+            for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(ov[q]) * mul;
+            store_cols_t(col, st.s, v, 16 * rnd, x.kv_len, p.varlen != 0, lane);
           }
-          named_barrier_sync(5, 128);
         }
       }
     }
