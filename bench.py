@@ -361,9 +361,9 @@ def weak_scaling_value(world: int, flops_per_rank: float, ms_per_step: float) ->
 def a7_timing(wl: I.Workload, dev, vsa, reps: int = 20) -> dict:
     """a7 device token moves of the tiled workload, timed apart from the
     forward: q's tokens into the padded tile layout (gather) and back
-    (scatter), L2 flushed before each launch.  Algorithmic bytes: gather
-    reads the tokens and writes every slot, scatter reads and writes the
-    real tokens."""
+    (scatter), L2 flushed before each launch.
+    Algorithmic bytes: gather reads the tokens and writes every slot,
+    scatter reads and writes the real tokens."""
     meta = wl.extra["meta"]
     n_tok = int(sum(wl.q_block_sizes))
     G = wl.B * wl.H
@@ -380,6 +380,9 @@ def a7_timing(wl: I.Workload, dev, vsa, reps: int = 20) -> dict:
         total = 0.0
         for _ in range(reps):
             flush.fill_(1)
+            # keep the device busy while the host enqueues the call, so the
+            # events time the kernels and not the host's launch overhead
+            torch.cuda._sleep(400_000)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             fn()

@@ -809,7 +809,7 @@ int build_vsa_metadata(int T, int Hh, int W, int tT, int tH, int tW,
                        int64_t* slot_token, int32_t* n_tiles) {
   if (T <= 0 || Hh <= 0 || W <= 0 || tT <= 0 || tH <= 0 || tW <= 0) return VSA_ERR_INVALID_ARG;
   const int vol = tT * tH * tW;
-  if (vol > 128) return VSA_ERR_INVALID_ARG;
+  if (vol > 256) return VSA_ERR_INVALID_ARG;
   const int nT = (T + tT - 1) / tT, nH = (Hh + tH - 1) / tH, nW = (W + tW - 1) / tW;
   const long long ntiles = (long long)nT * nH * nW;
   if (ntiles > 0x7FFFFFFFLL) return VSA_ERR_UNSUPPORTED;

@@ -47,47 +47,56 @@ __global__ void rebase_kernel(const int32_t* q2k_idx, const int32_t* q2k_num,
   out[i] = v;
 }
 
-// One CTA per (SPB * kSlotsPerThread slots, group): thread t moves 16-byte
-// chunk t % (D / 8) of kSlotsPerThread slots spaced SPB apart.  The slot
-// indices are loaded first, then every data load, then every store, so a
-// gather's two dependent loads (index, then token row) overlap across slots.
-// 32-bit index arithmetic (every tensor here holds fewer than 2^31 16-byte
-// chunks per group).
+// One CTA per (SPB * kSlotsPerThread slots, kGroupsPerCta groups): thread t
+// moves 16-byte chunk t % (D / 8) of kSlotsPerThread slots spaced SPB apart,
+// for each of the CTA's groups.  The slot indices are loaded once for all
+// the groups, then every data load of the groups is issued, then every
+// store: a gather's two dependent loads (index, then token row) pay the
+// index latency once per kGroupsPerCta groups, with kSlotsPerThread *
+// kGroupsPerCta loads in flight per thread.
 constexpr int kSlotsPerThread = 4;
+constexpr int kGroupsPerCta = 4;
 
 template <bool SCATTER, int D>
 __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint4* src, uint4* dst,
                                                             const int64_t* slot_token,
-                                                            int n_tokens, int n_slots) {
+                                                            int n_tokens, int n_slots, int groups) {
   constexpr int CH = D / 8;             // 16-byte chunks per row
   constexpr int SPB = 256 / CH;         // slots per pass
   const int ch = (int)threadIdx.x % CH;
   const int s0 = blockIdx.x * SPB * kSlotsPerThread + (int)threadIdx.x / CH;
-  const long long g = blockIdx.y;
-  int64_t tok[kSlotsPerThread];
+  const int g0 = blockIdx.y * kGroupsPerCta;
+  int tok[kSlotsPerThread];
 #pragma unroll
   for (int i = 0; i < kSlotsPerThread; ++i) {
     const int s = s0 + i * SPB;
-    tok[i] = s < n_slots ? slot_token[s] : -1;
+    const int64_t t = s < n_slots ? slot_token[s] : -1;
+    tok[i] = (t >= 0 && t < n_tokens) ? (int)t : -1;  // -1: padding (or out of range)
   }
-  uint4 v[kSlotsPerThread];
+  uint4 v[kGroupsPerCta][kSlotsPerThread];
 #pragma unroll
-  for (int i = 0; i < kSlotsPerThread; ++i) {
-    const int s = s0 + i * SPB;
-    const bool real = tok[i] >= 0 && tok[i] < n_tokens;
-    v[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (s < n_slots && real)
-      v[i] = SCATTER ? __ldcs(src + (g * n_slots + s) * CH + ch)
-                     : __ldcs(src + (g * n_tokens + tok[i]) * CH + ch);
+  for (int k = 0; k < kGroupsPerCta; ++k) {
+    const long long g = g0 + k;
+    const uint4* sg = src + g * (SCATTER ? n_slots : n_tokens) * CH + ch;
+#pragma unroll
+    for (int i = 0; i < kSlotsPerThread; ++i) {
+      const int s = s0 + i * SPB;
+      v[k][i] = make_uint4(0u, 0u, 0u, 0u);
+      if (g < groups && s < n_slots && tok[i] >= 0)
+        v[k][i] = __ldcs(sg + (long long)(SCATTER ? s : tok[i]) * CH);
+    }
   }
 #pragma unroll
-  for (int i = 0; i < kSlotsPerThread; ++i) {
-    const int s = s0 + i * SPB;
-    if (s >= n_slots) continue;
-    if (!SCATTER) {
-      __stcs(dst + (g * n_slots + s) * CH + ch, v[i]);
-    } else if (tok[i] >= 0 && tok[i] < n_tokens) {
-      __stcs(dst + (g * n_tokens + tok[i]) * CH + ch, v[i]);
+  for (int k = 0; k < kGroupsPerCta; ++k) {
+    const long long g = g0 + k;
+    if (g >= groups) break;
+    uint4* dg = dst + g * (SCATTER ? n_tokens : n_slots) * CH + ch;
+#pragma unroll
+    for (int i = 0; i < kSlotsPerThread; ++i) {
+      const int s = s0 + i * SPB;
+      if (s >= n_slots) continue;
+      if (!SCATTER) __stcs(dg + (long long)s * CH, v[k][i]);
+      else if (tok[i] >= 0) __stcs(dg + (long long)tok[i] * CH, v[k][i]);
     }
   }
 }
@@ -289,16 +298,18 @@ int launch_gather_tokens(const void* src, void* dst, const int64_t* slot_token, 
   if (groups <= 0 || n_slots <= 0) return VSA_OK;
   if (n_tokens > 0x7FFFFFFFLL || n_slots > 0x7FFFFFFFLL || groups > 65535) return VSA_ERR_UNSUPPORTED;
   const int spb = D <= 2048 ? 256 / (D / 8) * kSlotsPerThread : 1;
-  const dim3 grid((unsigned)((n_slots + spb - 1) / spb), (unsigned)groups);
+  const dim3 grid((unsigned)((n_slots + spb - 1) / spb),
+                  (unsigned)((groups + kGroupsPerCta - 1) / kGroupsPerCta));
+  const int ng = (int)groups;
   const uint4* s4 = static_cast<const uint4*>(src);
   uint4* d4 = static_cast<uint4*>(dst);
   const int nt = (int)n_tokens, ns = (int)n_slots;
   if (D == 128) {
-    if (scatter) gather_tokens_kernel<true, 128><<<grid, 256, 0, stream>>>(s4, d4, slot_token, nt, ns);
-    else gather_tokens_kernel<false, 128><<<grid, 256, 0, stream>>>(s4, d4, slot_token, nt, ns);
+    if (scatter) gather_tokens_kernel<true, 128><<<grid, 256, 0, stream>>>(s4, d4, slot_token, nt, ns, ng);
+    else gather_tokens_kernel<false, 128><<<grid, 256, 0, stream>>>(s4, d4, slot_token, nt, ns, ng);
   } else if (D == 64) {
-    if (scatter) gather_tokens_kernel<true, 64><<<grid, 256, 0, stream>>>(s4, d4, slot_token, nt, ns);
-    else gather_tokens_kernel<false, 64><<<grid, 256, 0, stream>>>(s4, d4, slot_token, nt, ns);
+    if (scatter) gather_tokens_kernel<true, 64><<<grid, 256, 0, stream>>>(s4, d4, slot_token, nt, ns, ng);
+    else gather_tokens_kernel<false, 64><<<grid, 256, 0, stream>>>(s4, d4, slot_token, nt, ns, ng);
   } else {
     const dim3 g1((unsigned)n_slots, (unsigned)groups);
     if (scatter) gather_tokens_any_kernel<true><<<g1, 256, 0, stream>>>(s4, d4, slot_token, nt, ns, D / 8);

@@ -507,7 +507,8 @@ int block_sparse_attn_varlen_backward(
  *                                 each padded slot, -1 for padding
  * n_tiles                         int32 [1]
  * Returns VSA_ERR_INVALID_ARG for non-positive sizes or a tile volume above
- * 128 (64 for the 64-slot path, 128 for VSA-128 tiles such as 4 x 4 x 8).
+ * 256 (64 for the 64-slot path, 128 or 256 for VSA-128 / VSA-256 tiles such
+ * as 4 x 4 x 8 or 4 x 8 x 8).
  */
 int build_vsa_metadata(int T, int Hh, int W, int tT, int tH, int tW,
                        int64_t* tile_partition_indices, int64_t* reverse_tile_partition_indices,

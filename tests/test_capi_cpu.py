@@ -193,10 +193,13 @@ def test_metadata_matches_oracle(shape, tile):
 def test_metadata_rejects_bad_tiles():
     lib = _lib()
     n = ctypes.c_int32(0)
-    assert lib.build_vsa_metadata(4, 4, 4, 8, 4, 8, None, None, None, None, None,
-                                  ctypes.byref(n)) == 1          # tile volume 256 > 128
+    assert lib.build_vsa_metadata(8, 8, 8, 8, 8, 8, None, None, None, None, None,
+                                  ctypes.byref(n)) == 1          # tile volume 512 > 256
     assert lib.build_vsa_metadata(8, 4, 4, 8, 4, 4, None, None, None, None, None,
                                   ctypes.byref(n)) == 0          # 128-token tiles (VSA-128)
+    assert n.value == 1
+    assert lib.build_vsa_metadata(4, 8, 8, 4, 8, 8, None, None, None, None, None,
+                                  ctypes.byref(n)) == 0          # 256-token tiles (VSA-256)
     assert n.value == 1
     assert lib.build_vsa_metadata(0, 4, 4, 4, 4, 4, None, None, None, None, None,
                                   ctypes.byref(n)) == 1

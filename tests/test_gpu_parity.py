@@ -476,20 +476,22 @@ def test_varlen_variable_block_sizes():
 # a7: tile gather / scatter
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("D", [128, 64, 96, 8])
-@pytest.mark.parametrize("shape", [(9, 30, 52), (5, 5, 5)])
-def test_tile_gather_scatter(shape, D):
-    """Rows of 64 and 128 values take the 16-slots-per-CTA kernel, other
-    multiples of 8 the one-slot-per-CTA kernel; both give the tile layout
-    exactly and scatter back to the tokens."""
-    meta = vsa.build_vsa_metadata(*shape)
+@pytest.mark.parametrize("shape,tile", [((9, 30, 52), (4, 4, 4)), ((5, 5, 5), (4, 4, 4)),
+                                        ((6, 10, 20), (4, 8, 8))])
+def test_tile_gather_scatter(shape, tile, D):
+    """Rows of 64 and 128 values take the several-slots-per-thread kernel,
+    other multiples of 8 the one-slot-per-CTA kernel; both give the tile
+    layout exactly (64- and 256-token tiles) and scatter back to the tokens."""
+    meta = vsa.build_vsa_metadata(*shape, tile=tile)
     N = int(np.prod(shape))
     x = I.normal_bf16((2, 3, N, D), 3300, 0)
     slot = torch.from_numpy(meta["slot_token"]).to(DEV)
     xp = vsa.gather_tokens(x.reshape(6, N, D).to(DEV), slot)
-    want = O.tile_and_pad(P.to_np(x), O.build_vsa_metadata(*shape))
+    want = O.tile_and_pad(P.to_np(x), O.build_vsa_metadata(*shape, tile=tile))
     assert np.array_equal(P.to_np(xp).reshape(want.shape), want)
     back = vsa.scatter_tokens(xp, slot, N)
     assert torch.equal(back.cpu().reshape(x.shape), x)
+    vsa.check_device_status()
 
 
 # ---------------------------------------------------------------------------
