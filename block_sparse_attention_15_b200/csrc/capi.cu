@@ -16,6 +16,53 @@ namespace vsa {
 // Device status word: kernels record the first error of a launch sequence.
 __device__ int g_device_status = 0;
 
+// Page-locked staging of the small host tables some entries copy to the
+// device (varlen block tables, host block sizes): per device, a ring of
+// slots, each reused only after the copy that last read it has completed
+// (one event per slot).  The copies are then truly asynchronous, and the host
+// runs ahead of the stream by up to kStageSlots calls before it waits.
+namespace {
+constexpr int kStageSlots = 8;
+constexpr int kMaxDevices = 64;
+struct StageRing {
+  std::mutex mu;
+  void* buf[kStageSlots] = {};
+  size_t cap[kStageSlots] = {};
+  cudaEvent_t ev[kStageSlots] = {};
+  bool pending[kStageSlots] = {};
+  int next = 0;
+};
+StageRing g_stage[kMaxDevices];
+}  // namespace
+
+int stage_copy_h2d(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+  if (bytes == 0) return VSA_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return VSA_ERR_CUDA;
+  StageRing& r = g_stage[dev];
+  std::lock_guard<std::mutex> lock(r.mu);
+  const int i = r.next;
+  r.next = (i + 1) % kStageSlots;
+  if (r.pending[i] && cudaEventSynchronize(r.ev[i]) != cudaSuccess) return VSA_ERR_CUDA;
+  r.pending[i] = false;
+  if (!r.ev[i] && cudaEventCreateWithFlags(&r.ev[i], cudaEventDisableTiming) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  if (r.cap[i] < bytes) {
+    if (r.buf[i]) cudaFreeHost(r.buf[i]);
+    r.buf[i] = nullptr;
+    r.cap[i] = 0;
+    const size_t want = bytes < 16384 ? 16384 : bytes;
+    if (cudaMallocHost(&r.buf[i], want) != cudaSuccess) return VSA_ERR_CUDA;
+    r.cap[i] = want;
+  }
+  memcpy(r.buf[i], src, bytes);
+  if (cudaMemcpyAsync(dst, r.buf[i], bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaEventRecord(r.ev[i], st) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  r.pending[i] = true;
+  return VSA_OK;
+}
+
 // The address is looked up once per device and cached (under a lock, so
 // concurrent first calls from several host threads are safe).  The cache
 // assumes the device's context lives as long as the process: a
@@ -561,11 +608,9 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
     return VSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t* dtab = static_cast<int32_t*>(workspace);
-  // Pageable source: the runtime stages it before returning, so `table` may
-  // be released right after the call.
-  if (cudaMemcpyAsync(dtab, table.data(), sizeof(int32_t) * table.size(), cudaMemcpyHostToDevice,
-                      st) != cudaSuccess)
-    return VSA_ERR_CUDA;
+  // through the page-locked ring, so `table` may be released right after
+  if ((rc = stage_copy_h2d(dtab, table.data(), sizeof(int32_t) * table.size(), st)) != VSA_OK)
+    return rc;
   int* status = device_status_ptr();
   if (!status) return VSA_ERR_CUDA;
   const int32_t* d_qtok = dtab;
@@ -757,9 +802,8 @@ int block_sparse_attn_varlen_backward(
     return VSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t* dtab = static_cast<int32_t*>(workspace);
-  if (cudaMemcpyAsync(dtab, vt.table.data(), sizeof(int32_t) * vt.table.size(),
-                      cudaMemcpyHostToDevice, st) != cudaSuccess)
-    return VSA_ERR_CUDA;
+  if ((rc = stage_copy_h2d(dtab, vt.table.data(), sizeof(int32_t) * vt.table.size(), st)) != VSA_OK)
+    return rc;
   int* status = device_status_ptr();
   if (!status) return VSA_ERR_CUDA;
   const float sc = resolve_scale(scale, D);

@@ -150,10 +150,10 @@ extern "C" int vsa_forward_host(const void* q, const void* k, const void* v, con
   // workspace, for instance) comes first
   VSA_CK(cudaEventRecord(ev.start, st));
   VSA_CK(cudaStreamWaitEvent(s_in, ev.start, 0));
-  if (q_block_sizes)
-    VSA_CK(cudaMemcpyAsync(qbs_d, q_block_sizes, 4 * (size_t)nq, cudaMemcpyHostToDevice, s_in));
-  if (kv_block_sizes)
-    VSA_CK(cudaMemcpyAsync(kvbs_d, kv_block_sizes, 4 * (size_t)nkv, cudaMemcpyHostToDevice, s_in));
+  if (q_block_sizes && stage_copy_h2d(qbs_d, q_block_sizes, 4 * (size_t)nq, s_in) != VSA_OK)
+    return VSA_ERR_CUDA;
+  if (kv_block_sizes && stage_copy_h2d(kvbs_d, kv_block_sizes, 4 * (size_t)nkv, s_in) != VSA_OK)
+    return VSA_ERR_CUDA;
 
   const size_t sq = (size_t)Sq_pad, skv = (size_t)Skv_pad;
   const char* qh = static_cast<const char*>(q);

@@ -96,6 +96,10 @@ struct SparseParams {
   int* status;
 };
 
+// Host-to-device copy of a small host table through the library's per-device
+// page-locked staging ring (capi.cu): asynchronous on `st`; `src` may be
+// released as soon as the call returns.
+int stage_copy_h2d(void* dst, const void* src, size_t bytes, cudaStream_t st);
 int launch_pool(const PoolParams& p, int D, cudaStream_t stream);
 int launch_coarse_topk(const CoarseParams& p, int D, cudaStream_t stream);
 // q, k, v: strided [B, H, S, D] bf16 views with S = q_seq / kv_seq slots

@@ -32,10 +32,11 @@
  *   device on first use, kept for the process, and a few events per call.)
  * - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *   asynchronous on that stream and never synchronise it, except
- *   vsa_get_device_status, and except that block_sparse_attn_varlen (its
- *   block tables) and vsa_forward_host (the block sizes) copy a small table
- *   from pageable host memory with cudaMemcpyAsync, which the CUDA runtime
- *   may serialise with the stream.
+ *   vsa_get_device_status.  The varlen entries (their block tables) and
+ *   vsa_forward_host (the block sizes) copy a small host table through a
+ *   page-locked staging ring the library keeps per device (8 slots, grown on
+ *   first use): the host waits only when the slot it reuses, eight such
+ *   calls back, still has its copy in flight.
  * - Every call returns a vsa status code.  Argument problems detectable on
  *   the host are returned before anything is launched.  Problems found inside
  *   kernels (an out-of-range index, a bad block size, a barrier wait that ran
