@@ -80,6 +80,10 @@ constexpr uint32_t kTmemO = 256;
 // is exponentiated without a refresh: probabilities stay below 2^32, far from
 // fp32 / bf16 overflow in P^T, O^T and the row sums.
 constexpr float kOffsetLimit = 32.f;
+// Largest logit bound (log2 units) for which an item's vote-free steps skip
+// the exponential's lower clamp: every offset s*c - m is then >= -2 * bound
+// (s*c >= -bound and the running max m <= bound), so >= -120.
+constexpr float kNoClampBound = 60.f;
 
 template <int D>
 struct Layout {
@@ -243,13 +247,15 @@ __device__ __forceinline__ bool col_reduce32(const float (&v)[32], float* red, f
 // masked row), added to the row-sum partials and packed as bf16 pairs.  Three
 // column pairs in eight take the FMA-pipe exponential, the rest the MUFU one,
 // which balances the two units.
+// CLAMP = false where the offsets are known to be >= -120 (see kNoClampBound).
+template <bool CLAMP>
 __device__ __forceinline__ void compute_probs(const uint32_t (&x)[32], bool valid, float (&lp)[32],
                                               uint32_t (&pk)[16]) {
   if (valid) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const float x0 = __uint_as_float(x[2 * j]), x1 = __uint_as_float(x[2 * j + 1]);
-      const uint64_t pp = ((j & 7) < VSA_POLY8) ? exp2_fma2(x0, x1) : pk2(fast_exp2(x0), fast_exp2(x1));
+      const uint64_t pp = ((j & 7) < VSA_POLY8) ? exp2_fma2_t<CLAMP>(x0, x1) : pk2(fast_exp2(x0), fast_exp2(x1));
       upk2(fadd2(pk2(lp[2 * j], lp[2 * j + 1]), pp), lp[2 * j], lp[2 * j + 1]);
       float p0, p1;
       upk2(pp, p0, p1);
@@ -695,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (t128 < 32) {
             const float mn = (fin[t128] == -INFINITY) ? 0.f : -fin[t128];
             mns[t128] = mn;
-            fits = qk_bound + mn <= kOffsetLimit;
+            fits = qk_bound + mn <= kOffsetLimit && qk_bound <= kNoClampBound;
           }
           novote = bar_red_and(bar_red, 128, fits);
           VSA_TMEM_LD16(t_lane + s0_col, x0, 0);
@@ -760,8 +766,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the exponentials first, so that they overlap the PV products still
         // reading the P^T buffers
         uint32_t pk0[16], pk1[16];
-        compute_probs(x0, valid0, lp, pk0);
-        if (two) compute_probs(x1, valid1, lp, pk1);
+        compute_probs<vote>(x0, valid0, lp, pk0);
+        if (two) compute_probs<vote>(x1, valid1, lp, pk1);
         // the P^T buffers are free once the PV products of pairs g0 - kNP and
         // g0 + 1 - kNP are done; both are committed by one thread in order, so
         // the barrier of the later one covers both

@@ -431,11 +431,13 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // error on that interval (Remez exchange; block_sparse_attention_15_b200/
 // exp2_fit.py computes these float32 coefficients and models these steps:
 // max relative error 7.49e-5 over [-120, 32], far below the bf16 rounding of
-// the probabilities).  x is clamped to >= -120, where the result (2^-120) is
-// negligible next to the row maximum's 1.
-__device__ __forceinline__ uint64_t exp2_fma2(float x0, float x1) {
+// the probabilities).  With CLAMP, x is clamped to >= -120, where the result
+// (2^-120) is negligible next to the row maximum's 1; without it the caller
+// guarantees x >= -120 (below that the exponent field would wrap).
+template <bool CLAMP>
+__device__ __forceinline__ uint64_t exp2_fma2_t(float x0, float x1) {
   constexpr float kRound = 12582912.f;  // 1.5 * 2^23: adding it rounds to an integer
-  const uint64_t xx = pk2(fmaxf(x0, -120.f), fmaxf(x1, -120.f));
+  const uint64_t xx = CLAMP ? pk2(fmaxf(x0, -120.f), fmaxf(x1, -120.f)) : pk2(x0, x1);
   const uint64_t t = fadd2(xx, pk2(kRound, kRound));
   const uint64_t j = fadd2(t, pk2(-kRound, -kRound));
   const uint64_t f = ffma2(j, pk2(-1.f, -1.f), xx);
@@ -449,6 +451,9 @@ __device__ __forceinline__ uint64_t exp2_fma2(float x0, float x1) {
   const float r0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
   const float r1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
   return pk2(r0, r1);
+}
+__device__ __forceinline__ uint64_t exp2_fma2(float x0, float x1) {
+  return exp2_fma2_t<true>(x0, x1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
