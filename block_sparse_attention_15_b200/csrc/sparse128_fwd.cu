@@ -62,6 +62,10 @@ constexpr float kRefresh = 8.f;
 // the logit bound must rule out before an item's later tiles skip the max
 // exchange: probabilities then stay below 2^32 (bf16 and fp32 hold them).
 constexpr float kBoundLimit = 32.f;
+// Largest logit bound (log2 units) for which those tiles also skip the
+// FMA-pipe exponential's lower clamp: every offset s*c - m is then >= -2 *
+// bound (s*c >= -bound, the reference max m <= bound), so >= -120.
+constexpr float kNoClampBound = 60.f;
 #ifndef VSA128_POLY8
 #define VSA128_POLY8 3  // column pairs in eight whose exponential runs on the FMA pipe
 #endif
@@ -133,6 +137,11 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
 // rows of the block's 256 slots split in two, each selected KV block read as
 // two 128-key sub-tiles (the second empty when the block holds at most 128
 // real keys), so both halves see exactly the block's selected keys.
+template <bool B>
+struct ClampTag {
+  static constexpr bool value = B;
+};
+
 struct Item {
   int a;        // 128-row tile index in the sequence
   int ab;       // the caller's block index (a >> p.sub)
@@ -451,24 +460,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j == 0) {
           // the first tile fixed the row maxima: can the bound rule out a move
           // for every row of the item?  (m = -inf fails the test)
-          novote = bar_red_and(1, 256, qk_bound - m <= kBoundLimit);
+          novote = bar_red_and(1, 256, qk_bound - m <= kBoundLimit && qk_bound <= kNoClampBound);
         }
         }
         // probabilities 2^(s*c - m) as bf16 pairs, sums in fp32
         uint32_t pk[32];
-        if (full) {
-          // every key real (the common case): no per-element tests
+        // every key real (the common case): no per-element tests; the
+        // vote-free tiles of an item skip the exponential's clamp
+        auto full_tile = [&](auto clamp_tag) {
+          constexpr bool CLAMP = decltype(clamp_tag)::value;
           const uint64_t nm2 = pk2(-m, -m);
 #pragma unroll
           for (int q = 0; q < 32; ++q) {
             float a, b;
             upk2(ffma2(pk2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), cc, nm2), a, b);
-            const uint64_t pp = ((q & 7) < VSA128_POLY8) ? exp2_fma2(a, b) : pk2(fast_exp2(a), fast_exp2(b));
+            const uint64_t pp = ((q & 7) < VSA128_POLY8) ? exp2_fma2_t<CLAMP>(a, b)
+                                                          : pk2(fast_exp2(a), fast_exp2(b));
             upk2(fadd2(pk2(l0, l1), pp), l0, l1);
             float p0, p1;
             upk2(pp, p0, p1);
             pk[q] = pack_bf16x2(p0, p1);
           }
+        };
+        if (full && novote) {
+          full_tile(ClampTag<false>{});
+        } else if (full) {
+          full_tile(ClampTag<true>{});
         } else {
           // masked columns (s = -inf) give exactly 0; a row that has seen no
           // real key yet (m = -inf) too
