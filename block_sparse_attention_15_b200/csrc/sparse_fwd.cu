@@ -70,7 +70,7 @@ constexpr int kNS = 4;                 // S^T buffers in TMEM
 #define VSA_NP 2
 #endif
 #ifndef VSA_POLY8
-#define VSA_POLY8 3   // column pairs in eight whose exponential runs on the FMA pipe
+#define VSA_POLY8 2   // column pairs in eight whose exponential runs on the FMA pipe
 #endif
 constexpr int kNP = VSA_NP;            // P^T buffers in shared memory (even)
 static_assert(kNP >= 2 && kNP % 2 == 0, "two pairs per softmax step");
