@@ -30,8 +30,9 @@
 //   warps 4-7    softmax for query columns 0..31
 //   warps 8-11   softmax for query columns 32..63
 //   warps 12-15  epilogue: O^T / l, the gated combine, bf16 stores
-// The softmax takes two pairs per step; P^T is double-buffered in shared
-// memory, so a step waits for the PV products of the previous step.  The
+// The softmax takes two pairs per step; P^T has shared-memory buffers for
+// two steps, so a step waits for the PV products of the step before the
+// previous one (and the previous step's run while it computes).  The
 // running max per query column is exact after an item's first step (column
 // reduction across lanes) and refreshed only when a logit exceeds it by more
 // than kOffsetLimit (log2 units; barrier vote), then O^T and the partial sums
@@ -67,7 +68,7 @@ static_assert(128u * (kRegsProducer + 2u * kRegsSoftmax + kRegsEpilogue) <= 512u
 constexpr int kKLead = VSA_KLEAD;      // K requests run at most this many pairs ahead of V
 constexpr int kNS = 4;                 // S^T buffers in TMEM
 #ifndef VSA_NP
-#define VSA_NP 2
+#define VSA_NP 4
 #endif
 #ifndef VSA_POLY8
 #define VSA_POLY8 2   // column pairs in eight whose exponential runs on the FMA pipe
