@@ -66,7 +66,10 @@ static_assert(128u * (kRegsProducer + 2u * kRegsSoftmax + kRegsEpilogue) <= 512u
 #define VSA_KLEAD 6
 #endif
 constexpr int kKLead = VSA_KLEAD;      // K requests run at most this many pairs ahead of V
-constexpr int kNS = 4;                 // S^T buffers in TMEM
+#ifndef VSA_NS
+#define VSA_NS 4
+#endif
+constexpr int kNS = VSA_NS;            // S^T buffers in TMEM (64 columns each)
 #ifndef VSA_NP
 #define VSA_NP 4
 #endif
@@ -75,8 +78,9 @@ constexpr int kNS = 4;                 // S^T buffers in TMEM
 #endif
 constexpr int kNP = VSA_NP;            // P^T buffers in shared memory (even)
 static_assert(kNP >= 2 && kNP % 2 == 0, "two pairs per softmax step");
-constexpr uint32_t kTmemCols = 512;    // S^T buffers at 64*i (i < 4), O^T buffers at 256, 320
-constexpr uint32_t kTmemO = 256;
+constexpr uint32_t kTmemCols = 512;    // S^T buffers at 64*i (i < kNS), then the two O^T buffers
+constexpr uint32_t kTmemO = 64u * kNS;
+static_assert(kTmemO + 128u <= kTmemCols, "S^T and O^T buffers exceed TMEM");
 // Largest offset (log2 units) of a logit above its column's running max that
 // is exponentiated without a refresh: probabilities stay below 2^32, far from
 // fp32 / bf16 overflow in P^T, O^T and the row sums.
