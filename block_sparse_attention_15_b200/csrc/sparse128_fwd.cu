@@ -49,7 +49,18 @@ namespace vsa {
 namespace b128 {
 
 constexpr int kThreads = 512;
-constexpr uint32_t kRegsProducer = 56, kRegsSoftmax = 176, kRegsEpilogue = 104;
+// registers per thread of the producer / MMA, softmax and epilogue warpgroups
+#ifndef VSA128_REGS_P
+#define VSA128_REGS_P 48
+#endif
+#ifndef VSA128_REGS_S
+#define VSA128_REGS_S 184
+#endif
+#ifndef VSA128_REGS_E
+#define VSA128_REGS_E 96
+#endif
+constexpr uint32_t kRegsProducer = VSA128_REGS_P, kRegsSoftmax = VSA128_REGS_S,
+                   kRegsEpilogue = VSA128_REGS_E;
 constexpr uint32_t kLaunchRegs = 128;  // 512 x 128 = 65536
 static_assert(128u * (kRegsProducer + 2u * kRegsSoftmax + kRegsEpilogue) <= 512u * kLaunchRegs,
               "register split exceeds the launch's registers");
@@ -67,7 +78,7 @@ constexpr float kBoundLimit = 32.f;
 // bound (s*c >= -bound, the reference max m <= bound), so >= -120.
 constexpr float kNoClampBound = 60.f;
 #ifndef VSA128_POLY8
-#define VSA128_POLY8 3  // column pairs in eight whose exponential runs on the FMA pipe
+#define VSA128_POLY8 2  // column pairs in eight whose exponential runs on the FMA pipe
 #endif
 
 template <int D>

@@ -59,7 +59,17 @@ struct BoolTag {
 };
 
 constexpr int kThreads = 512;
-constexpr uint32_t kRegsProducer = 64, kRegsSoftmax = 192, kRegsEpilogue = 64;
+// registers per thread of the producer / MMA, softmax and epilogue warpgroups
+#ifndef VSA_REGS_P
+#define VSA_REGS_P 64
+#endif
+#ifndef VSA_REGS_S
+#define VSA_REGS_S 192
+#endif
+#ifndef VSA_REGS_E
+#define VSA_REGS_E 64
+#endif
+constexpr uint32_t kRegsProducer = VSA_REGS_P, kRegsSoftmax = VSA_REGS_S, kRegsEpilogue = VSA_REGS_E;
 static_assert(128u * (kRegsProducer + 2u * kRegsSoftmax + kRegsEpilogue) <= 512u * 128u,
               "register split exceeds the launch's 128 registers per thread");
 #ifndef VSA_KLEAD
