@@ -415,6 +415,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // max exchange (same results: the reference max would not move)
       const float qk_bound = p.qk_bound ? p.qk_bound[x.group * p.nq + x.ab] : INFINITY;
       bool novote = false;
+      if (qk_bound <= kNoClampBound) {
+        // the bound itself is the row's reference max: every offset s*c - m
+        // is then in [-2 * bound, 0], so no tile needs the row max, its
+        // exchange or the exponential's clamp (same results up to rounding:
+        // the row's probabilities share one scale factor)
+        m = qk_bound;
+        novote = true;
+      }
       for (int j = 0; j < x.num; ++j, ++g) {
         const int sb = (int)(g & 1);
         wwait(bars + L::kSFull + sb, (g >> 1) & 1);

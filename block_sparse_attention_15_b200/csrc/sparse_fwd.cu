@@ -661,6 +661,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       float lp[32];
 #pragma unroll
       for (int q = 0; q < 32; ++q) lp[q] = 0.f;
+      if (qk_bound <= kNoClampBound) {
+        // the bound itself is every column's reference max: each offset
+        // s*c - m is then in [-2 * bound, 0], so no step needs the exact
+        // maximum, a vote or the exponential's clamp (same results up to
+        // rounding: the probabilities of a column share one scale factor)
+        if (t128 < 32) mns[t128] = -qk_bound;
+        if (bar_red_or(bar_red, 128, aborted)) { ok = false; break; }
+        novote = true;
+      }
       // One step: two pairs (the second may be absent at the end of an
       // item), so the fixed cost of the handshakes is paid once per 4 KV
       // tiles.  The step is compiled for two pairs with the overflow vote, for

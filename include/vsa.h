@@ -313,10 +313,10 @@ int vsa_forward_host(const void* q, const void* k, const void* v, const void* ga
  *          its query norm times the largest key norm among the blocks it
  *          lists; where the bound shows no logit can exceed the first tile
  *          pair's maxima by 2^32, the sparse kernel skips its running-max
- *          check (fewer instructions; the same results at block size 64,
- *          and at 128 / 256 equal up to rounding where a later tile would
- *          have moved the running max).  Without it every step keeps the
- *          check.
+ *          check, and where the bound is at most 60 (log2 units) it serves
+ *          as the reference max from the first step on (fewer instructions;
+ *          the results equal those without the workspace up to the rounding
+ *          of the probabilities).  Without it every step keeps the check.
  * block_size  64, 128 or 256 (see vsa_forward_strided); n_q_blocks =
  *          Sq_pad / block_size
  * (ABI 2.0 added layout, block_size and workspace.)

@@ -79,10 +79,11 @@ def test_sparse256_from_indices(case):
     assert np.all(got[0, 0, BLK:BLK + qs[1]] == 0.0)   # the empty selection
 
 
-def test_sparse256_without_bound_pass_is_identical():
-    """The logit-bound pass only lets the kernel skip its max checks.  On
-    these N(0, 1) inputs no later sub-tile exceeds the first one's row maxima
-    by the refresh margin, so both runs take the same steps: the same bits."""
+def test_sparse256_without_bound_pass():
+    """With the logit-bound pass the bound becomes each row's reference max
+    (it is <= 60 log2 units on these N(0, 1) inputs), which changes the
+    probabilities only by a common factor per row: both runs agree up to
+    rounding and both match the oracle."""
     B, H, D = 1, 2, 128
     qs, ks = [256, 256, 130], [256, 90, 256, 256]
     q, k, v = (_padded(B, H, s, D, 760, i) for i, s in enumerate((qs, ks, ks)))
@@ -93,7 +94,13 @@ def test_sparse256_without_bound_pass_is_identical():
     o1 = vsa.block_sparse_attn_from_indices(*args, block=BLK)
     o2 = vsa.block_sparse_attn_from_indices(*args, block=BLK, logit_bound=False)
     vsa.check_device_status()
-    assert torch.equal(o1, o2)
+    a, b = o1.double(), o2.double()
+    assert ((a - b).norm() / b.norm()).item() <= 2e-3
+    want = O.block_sparse_attention(P.to_np(q), P.to_np(k), P.to_np(v), idx, num, qs, ks,
+                                    O.default_scale(D), block=BLK)
+    rr = _rows(qs)
+    for o in (o1, o2):
+        P.assert_outputs_close(P.to_np(o)[:, :, rr], want[:, :, rr], "sparse256 bound / no bound")
 
 
 def test_sparse256_peaked_logits_move_the_reference():

@@ -52,10 +52,22 @@ def test_bool_mask_matches_index_entry_and_oracle(D):
     assert np.all(got[0, 0, :64] == 0.0)
 
 
+def _within_rounding(a, b):
+    """Two bf16 results of the same attention computed with different
+    reference maxima: equal up to the rounding of the probabilities (a few
+    bf16 ulps), far inside the oracle tolerance."""
+    a, b = a.double(), b.double()
+    assert (a - b).abs().max().item() <= 2e-3 + 1e-2 * b.abs().max().item()
+    assert ((a - b).norm() / b.norm()).item() <= 2e-3
+
+
 @pytest.mark.parametrize("scale_q", [1.0, 6.0])
-def test_logit_bound_pass_changes_no_bit(scale_q):
-    """N(0,1) inputs: the bound lets items skip the running-max check;
-    peaked inputs (q x 6): it does not.  Either way the bits are the same."""
+def test_logit_bound_pass_changes_only_rounding(scale_q):
+    """N(0,1) inputs: the bound (<= 60 log2 units) becomes the reference max
+    and the items skip the running-max work, which changes the probabilities
+    only by a common factor per column (so the results only by rounding);
+    peaked inputs (q x 6): the bound is too loose and the kernel takes the
+    same steps with or without it (the same bits)."""
     B, H, D = 1, 4, 128
     qs, ks = [64] * 20, [64] * 30
     q = _bhsd(B, H, qs, D, 610, 0, scale=scale_q).to(DEV)
@@ -67,10 +79,14 @@ def test_logit_bound_pass_changes_no_bit(scale_q):
     with_bound = vsa.block_sparse_attn_from_indices(q, k, v, idx, num, logit_bound=True)
     without = vsa.block_sparse_attn_from_indices(q, k, v, idx, num, logit_bound=False)
     vsa.check_device_status()
-    assert torch.equal(with_bound, without)
+    if scale_q > 1.0:
+        assert torch.equal(with_bound, without)
+    else:
+        _within_rounding(with_bound, without)
     want = O.block_sparse_attention(P.to_np(q), P.to_np(k), P.to_np(v), P.to_np(idx), P.to_np(num),
                                     qs, ks, O.default_scale(D))
     P.assert_outputs_close(P.to_np(with_bound), want, "from indices with the bound")
+    P.assert_outputs_close(P.to_np(without), want, "from indices without the bound")
 
 
 @pytest.mark.parametrize("D,gated", [(128, True), (64, False)])
