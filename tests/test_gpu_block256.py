@@ -95,7 +95,7 @@ def test_sparse256_without_bound_pass():
     o2 = vsa.block_sparse_attn_from_indices(*args, block=BLK, logit_bound=False)
     vsa.check_device_status()
     a, b = o1.double(), o2.double()
-    assert ((a - b).norm() / b.norm()).item() <= 2e-3
+    assert ((a - b).norm() / b.norm()).item() <= 8e-3   # two bf16 ulps
     want = O.block_sparse_attention(P.to_np(q), P.to_np(k), P.to_np(v), idx, num, qs, ks,
                                     O.default_scale(D), block=BLK)
     rr = _rows(qs)

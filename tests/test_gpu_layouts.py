@@ -54,11 +54,12 @@ def test_bool_mask_matches_index_entry_and_oracle(D):
 
 def _within_rounding(a, b):
     """Two bf16 results of the same attention computed with different
-    reference maxima: equal up to the rounding of the probabilities (a few
-    bf16 ulps), far inside the oracle tolerance."""
+    reference maxima: equal up to rounding -- elements differ by a bf16 ulp
+    or two (relative 2^-8 each), so the relative RMS difference stays under
+    two ulps, inside the oracle tolerance."""
     a, b = a.double(), b.double()
     assert (a - b).abs().max().item() <= 2e-3 + 1e-2 * b.abs().max().item()
-    assert ((a - b).norm() / b.norm()).item() <= 2e-3
+    assert ((a - b).norm() / b.norm()).item() <= 8e-3
 
 
 @pytest.mark.parametrize("scale_q", [1.0, 6.0])
