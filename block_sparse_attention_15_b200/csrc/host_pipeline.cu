@@ -25,11 +25,14 @@ namespace {
 
 inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Heads per chunk: about eight chunks in all, at least one head.
+#ifndef VSA_HOST_CHUNKS
+#define VSA_HOST_CHUNKS 8
+#endif
+// Heads per chunk: about VSA_HOST_CHUNKS chunks in all, at least one head.
 int resolve_chunk_heads(int B, int H, int heads_per_chunk) {
   if (heads_per_chunk > 0) return heads_per_chunk < H ? heads_per_chunk : H;
-  if (B >= 8) return H;
-  const int per_batch = (8 + B - 1) / B;  // chunks wanted per batch entry
+  if (B >= VSA_HOST_CHUNKS) return H;
+  const int per_batch = (VSA_HOST_CHUNKS + B - 1) / B;  // chunks wanted per batch entry
   const int hc = (H + per_batch - 1) / per_batch;
   return hc < 1 ? 1 : hc;
 }
