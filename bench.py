@@ -82,10 +82,15 @@ def load_peaks():
 
 
 def sparse_source_hash() -> str:
+    """SHA-256 of the kernel sources' code: comments and blank lines are
+    dropped first, so that an edit of the comments alone keeps a capture's
+    record valid (the compiled kernel does not change)."""
     h = hashlib.sha256()
     for rel in SPARSE_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+        lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+        h.update("\n".join(ln for ln in lines if ln).encode())
     return h.hexdigest()
 
 

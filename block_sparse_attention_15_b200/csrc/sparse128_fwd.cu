@@ -26,10 +26,13 @@
 //   warp 1      TMEM owner; issues S(j) and PV(j-1) in that order
 //   warp 2      V tiles (2-stage ring)
 //   warps 4-11  softmax, two warpgroups splitting each row's key columns:
-//               S(j) -> P(j), row max with a lazy refresh (the reference max
-//               moves only when a logit exceeds it by more than kRefresh
-//               log2 units; then O is rescaled once the PV product before it
-//               is done), row sums
+//               S(j) -> P(j) and row sums.  The item's logit bound, where it
+//               is at most kNoClampBound, is the row's reference max from the
+//               first tile on; otherwise the row max takes a lazy refresh
+//               (the reference max moves only when a logit exceeds it by more
+//               than kRefresh log2 units; then O is rescaled once the PV
+//               product before it is done), with the tile max exchanged
+//               between the groups until the bound rules a move out
 //   warps 12-15 epilogue: O / l, out = out_c * gate + o (or out_c + o, or o),
 //               bf16 stores; double-buffered O lets it overlap the next item
 // Every wait is bounded and reports VSA_ERR_DEVICE_TIMEOUT.  The only named

@@ -32,16 +32,16 @@
 //   warps 12-15  epilogue: O^T / l, the gated combine, bf16 stores
 // The softmax takes two pairs per step; P^T has shared-memory buffers for
 // two steps, so a step waits for the PV products of the step before the
-// previous one (and the previous step's run while it computes).  The
+// previous one (and the previous step's run while it computes).  A
+// Cauchy-Schwarz bound on an item's logits (largest query row norm of the
+// block x largest key row norm of its selected blocks x scale), where it is
+// at most kNoClampBound, is every column's reference max from the first
+// step on: no step then needs a maximum, a vote or a rescale.  Otherwise the
 // running max per query column is exact after an item's first step (column
 // reduction across lanes) and refreshed only when a logit exceeds it by more
 // than kOffsetLimit (log2 units; barrier vote), then O^T and the partial sums
-// are rescaled.  Where a
-// Cauchy-Schwarz bound on an item's logits (largest query row norm of the
-// block x largest key row norm of the head x scale) already keeps every later
-// offset within the limit, the item's later steps run a copy of the step
-// without the vote.  Row sums are accumulated per lane and reduced across
-// lanes once per item.
+// are rescaled.  Row sums are accumulated per lane and reduced across lanes
+// once per item.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
