@@ -81,7 +81,7 @@ constexpr float kBoundLimit = 32.f;
 // bound (s*c >= -bound, the reference max m <= bound), so >= -120.
 constexpr float kNoClampBound = 60.f;
 #ifndef VSA128_POLY8
-#define VSA128_POLY8 2  // column pairs in eight whose exponential runs on the FMA pipe
+#define VSA128_POLY8 1  // column pairs in eight whose exponential runs on the FMA pipe
 #endif
 
 template <int D>
