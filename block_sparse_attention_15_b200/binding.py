@@ -84,6 +84,10 @@ SIGNATURES = {
     "block_sparse_attn_backward": (_c_int, [_c_void_p] * 10 + [_c_int] * 6 +
                                    [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                                     _c_size_t, _c_void_p]),
+    "block_sparse_attn_backward_ex_workspace_size": (_c_size_t, [_c_int] * 6),
+    "block_sparse_attn_backward_ex": (_c_int, [_c_void_p] * 10 + [_c_int] * 7 +
+                                      [_c_float, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                       _c_size_t, _c_void_p]),
     "block_sparse_attn_varlen_backward_workspace_size": (_c_size_t, [_c_int] * 5),
     "block_sparse_attn_varlen_backward": (_c_int, [_c_void_p] * 6 + [_P32] * 6 + [_c_int] * 3 +
                                           [_c_void_p, _c_void_p, _c_int, _c_float, _c_void_p,
@@ -436,10 +440,14 @@ def video_sparse_attn_bshd(q, k, v, gate=None, q_block_sizes=None, kv_block_size
 
 
 def block_sparse_attn_backward(q, k, v, out, dout, lse, q2k_idx, q2k_num, q_block_sizes=None,
-                               kv_block_sizes=None, *, scale: float | None = None, stream=None):
-    """dq, dk, dv of :func:`block_sparse_attn_from_indices` (64-slot blocks,
-    contiguous BHSD) for the output gradient ``dout``; ``out`` and ``lse``
-    come from that forward call (``return_lse=True``)."""
+                               kv_block_sizes=None, *, scale: float | None = None, block: int = 64,
+                               stream=None):
+    """dq, dk, dv of :func:`block_sparse_attn_from_indices` (contiguous BHSD)
+    for the output gradient ``dout``; ``out`` and ``lse`` come from that
+    forward call (``return_lse=True``), ``block`` is its block size.  Block
+    64 calls ``block_sparse_attn_backward``; 128 and 256 call
+    ``block_sparse_attn_backward_ex``, which rewrites the selection over
+    64-slot sub-blocks on the device first."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _require(t, torch.bfloat16, n)
     _require(lse, torch.float32, "lse")
@@ -447,21 +455,32 @@ def block_sparse_attn_backward(q, k, v, out, dout, lse, q2k_idx, q2k_num, q_bloc
     _require(q2k_num, torch.int32, "q2k_num")
     B, H, Sq, D = q.shape
     Skv = k.shape[2]
-    nq, nkv = Sq // 64, Skv // 64
+    nq, nkv = Sq // block, Skv // block
     if out.shape != q.shape or dout.shape != q.shape or lse.shape != (B, H, Sq):
         raise ValueError("out and dout must be shaped like q, lse [B, H, Sq_pad]")
+    if q2k_idx.dim() != 4 or q2k_idx.shape[:3] != (B, H, nq) or q2k_num.shape != (B, H, nq):
+        raise ValueError("q2k_idx must be [B, H, n_q_blocks, stride], q2k_num [B, H, n_q_blocks]")
     dev = q.device
     qbs = _block_sizes_tensor(q_block_sizes, nq, dev)
     kbs = _block_sizes_tensor(kv_block_sizes, nkv, dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     L = lib()
-    ws = torch.empty(max(L.block_sparse_attn_backward_workspace_size(B, H, Sq, nkv), 256),
-                     dtype=torch.uint8, device=dev)
-    _check("block_sparse_attn_backward", L.block_sparse_attn_backward(
+    sc = float(scale) if scale is not None else 0.0
+    width = q2k_idx.shape[3]
+    if block == 64:
+        ws = torch.empty(max(L.block_sparse_attn_backward_workspace_size(B, H, Sq, nkv), 256),
+                         dtype=torch.uint8, device=dev)
+        _check("block_sparse_attn_backward", L.block_sparse_attn_backward(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(q2k_idx),
+            _ptr(q2k_num), _ptr(qbs), _ptr(kbs), B, H, Sq, Skv, D, width, sc, _ptr(dq), _ptr(dk),
+            _ptr(dv), _ptr(ws), ws.numel(), _stream(stream)))
+        return dq, dk, dv
+    need = L.block_sparse_attn_backward_ex_workspace_size(B, H, Sq, Skv, int(block), width)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check("block_sparse_attn_backward_ex", L.block_sparse_attn_backward_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(q2k_idx), _ptr(q2k_num),
-        _ptr(qbs), _ptr(kbs), B, H, Sq, Skv, D, q2k_idx.shape[3],
-        float(scale) if scale is not None else 0.0, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
-        ws.numel(), _stream(stream)))
+        _ptr(qbs), _ptr(kbs), B, H, Sq, Skv, D, int(block), width, sc, _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(ws), ws.numel(), _stream(stream)))
     return dq, dk, dv
 
 

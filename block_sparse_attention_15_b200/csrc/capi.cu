@@ -293,7 +293,7 @@ const char* vsa_status_string(int status) {
   }
 }
 
-int vsa_abi_version(void) { return (2 << 16) | 0; }
+int vsa_abi_version(void) { return (2 << 16) | 1; }
 
 int vsa_get_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return VSA_ERR_CUDA;
@@ -397,7 +397,6 @@ static int sparse_from_indices(const void* q, const void* k, const void* v,
   const int nq = Sq_pad / block, nkv = Skv_pad / block;
   if (idx_stride > VSA_MAX_BLOCKS) return VSA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return VSA_ERR_INVALID_ARG;
-  if (lse && block != 64) return VSA_ERR_UNSUPPORTED;
   vsa_layout L;
   if (layout) L = *layout;
   else fill_layout(VSA_LAYOUT_BHSD, B, H, Sq_pad, Skv_pad, D, &L);
@@ -711,30 +710,15 @@ static void carve_bwd(BwdParams& bp, void* workspace, long long groups, long lon
   bp.k2q_num = reinterpret_cast<int32_t*>(ws);
 }
 
-int block_sparse_attn_backward(const void* q, const void* k, const void* v, const void* out,
-                               const void* dout, const float* lse, const int32_t* q2k_idx,
-                               const int32_t* q2k_num, const int32_t* q_block_sizes,
-                               const int32_t* kv_block_sizes, int B, int H, int Sq_pad,
-                               int Skv_pad, int D, int idx_stride, float scale, void* dq,
-                               void* dk, void* dv, void* workspace, size_t workspace_bytes,
-                               void* stream) {
-  if (!q || !k || !v || !out || !dout || !lse || !q2k_idx || !q2k_num || !dq || !dk || !dv)
-    return VSA_ERR_INVALID_ARG;
-  if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || idx_stride < 1 || !(scale == scale))
-    return VSA_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
-  if (Sq_pad % 64 || Skv_pad % 64) return VSA_ERR_SHAPE;
+// The 64-slot backward on checked arguments; `workspace` holds at least
+// block_sparse_attn_backward_workspace_size(B, H, Sq_pad, Skv_pad / 64) bytes.
+static int backward64(const void* q, const void* k, const void* v, const void* out,
+                      const void* dout, const float* lse, const int32_t* q2k_idx,
+                      const int32_t* q2k_num, const int32_t* q_block_sizes,
+                      const int32_t* kv_block_sizes, int B, int H, int Sq_pad, int Skv_pad, int D,
+                      int idx_stride, float scale, void* dq, void* dk, void* dv, void* workspace,
+                      int* status, cudaStream_t st) {
   const int nq = Sq_pad / 64, nkv = Skv_pad / 64;
-  if (idx_stride > VSA_MAX_BLOCKS || nq > VSA_MAX_BLOCKS || nkv > VSA_MAX_BLOCKS)
-    return VSA_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
-    return VSA_ERR_INVALID_ARG;
-  const size_t need = block_sparse_attn_backward_workspace_size(B, H, Sq_pad, nkv);
-  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-    return VSA_ERR_WORKSPACE;
-  int* status = device_status_ptr();
-  if (!status) return VSA_ERR_CUDA;
   const float sc = resolve_scale(scale, D);
   BwdParams bp;
   memset(&bp, 0, sizeof(bp));
@@ -763,7 +747,125 @@ int block_sparse_attn_backward(const void* q, const void* k, const void* v, cons
   bp.scale_log2 = sc * kLog2e;
   bp.status = status;
   carve_bwd(bp, workspace, (long long)B * H, Sq_pad, nq, nkv);
-  return launch_backward(bp, out, bhsd_strides(H, Sq_pad, D), D, static_cast<cudaStream_t>(stream));
+  return launch_backward(bp, out, bhsd_strides(H, Sq_pad, D), D, st);
+}
+
+// Argument checks shared by both backward entries (sizes in 64-slot units
+// after any expansion: n_q = Sq_pad / 64, n_kv = Skv_pad / 64, the expanded
+// index row width `stride64`).
+static int check_backward_args(const void* q, const void* k, const void* v, const void* out,
+                               const void* dout, const float* lse, const int32_t* q2k_idx,
+                               const int32_t* q2k_num, void* dq, void* dk, void* dv, int B, int H,
+                               int Sq_pad, int Skv_pad, int D, int block, int idx_stride,
+                               float scale) {
+  if (!q || !k || !v || !out || !dout || !lse || !q2k_idx || !q2k_num || !dq || !dk || !dv)
+    return VSA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || idx_stride < 1 || !(scale == scale))
+    return VSA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
+  if (block != 64 && block != 128 && block != 256) return VSA_ERR_UNSUPPORTED;
+  if (Sq_pad % block || Skv_pad % block) return VSA_ERR_SHAPE;
+  const long long stride64 = (long long)idx_stride * (block / 64);
+  if (stride64 > VSA_MAX_BLOCKS || Sq_pad / 64 > VSA_MAX_BLOCKS || Skv_pad / 64 > VSA_MAX_BLOCKS)
+    return VSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return VSA_ERR_INVALID_ARG;
+  return VSA_OK;
+}
+
+int block_sparse_attn_backward(const void* q, const void* k, const void* v, const void* out,
+                               const void* dout, const float* lse, const int32_t* q2k_idx,
+                               const int32_t* q2k_num, const int32_t* q_block_sizes,
+                               const int32_t* kv_block_sizes, int B, int H, int Sq_pad,
+                               int Skv_pad, int D, int idx_stride, float scale, void* dq,
+                               void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  int rc = check_backward_args(q, k, v, out, dout, lse, q2k_idx, q2k_num, dq, dk, dv, B, H, Sq_pad,
+                               Skv_pad, D, 64, idx_stride, scale);
+  if (rc != VSA_OK) return rc;
+  const size_t need = block_sparse_attn_backward_workspace_size(B, H, Sq_pad, Skv_pad / 64);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return VSA_ERR_WORKSPACE;
+  int* status = device_status_ptr();
+  if (!status) return VSA_ERR_CUDA;
+  return backward64(q, k, v, out, dout, lse, q2k_idx, q2k_num, q_block_sizes, kv_block_sizes, B, H,
+                    Sq_pad, Skv_pad, D, idx_stride, scale, dq, dk, dv, workspace, status,
+                    static_cast<cudaStream_t>(stream));
+}
+
+// Bytes of the 64-slot copy of a block-128/256 selection: index rows,
+// counts, query and key sub-block sizes.
+static size_t expand_bytes(long long groups, int nq, int nkv, int idx_stride, int shift) {
+  const size_t nq64 = (size_t)nq << shift, nkv64 = (size_t)nkv << shift;
+  return align256(sizeof(int32_t) * (size_t)groups * nq64 * ((size_t)idx_stride << shift)) +
+         align256(sizeof(int32_t) * (size_t)groups * nq64) + align256(sizeof(int32_t) * nq64) +
+         align256(sizeof(int32_t) * nkv64);
+}
+
+static int block_shift(int block) { return block == 256 ? 2 : (block == 128 ? 1 : 0); }
+
+size_t block_sparse_attn_backward_ex_workspace_size(int B, int H, int Sq_pad, int Skv_pad,
+                                                    int block_size, int idx_stride) {
+  if (B <= 0 || H <= 0 || Sq_pad <= 0 || Skv_pad <= 0 || idx_stride < 1) return 0;
+  if (block_size != 64 && block_size != 128 && block_size != 256) return 0;
+  if (Sq_pad % block_size || Skv_pad % block_size) return 0;
+  const int shift = block_shift(block_size);
+  const size_t base = block_sparse_attn_backward_workspace_size(B, H, Sq_pad, Skv_pad / 64);
+  if (!shift) return base;
+  return base + expand_bytes((long long)B * H, Sq_pad / block_size, Skv_pad / block_size,
+                             idx_stride, shift);
+}
+
+int block_sparse_attn_backward_ex(const void* q, const void* k, const void* v, const void* out,
+                                  const void* dout, const float* lse, const int32_t* q2k_idx,
+                                  const int32_t* q2k_num, const int32_t* q_block_sizes,
+                                  const int32_t* kv_block_sizes, int B, int H, int Sq_pad,
+                                  int Skv_pad, int D, int block_size, int idx_stride, float scale,
+                                  void* dq, void* dk, void* dv, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  int rc = check_backward_args(q, k, v, out, dout, lse, q2k_idx, q2k_num, dq, dk, dv, B, H, Sq_pad,
+                               Skv_pad, D, block_size, idx_stride, scale);
+  if (rc != VSA_OK) return rc;
+  const size_t need =
+      block_sparse_attn_backward_ex_workspace_size(B, H, Sq_pad, Skv_pad, block_size, idx_stride);
+  if (!workspace || !need || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return VSA_ERR_WORKSPACE;
+  int* status = device_status_ptr();
+  if (!status) return VSA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int shift = block_shift(block_size);
+  if (!shift)
+    return backward64(q, k, v, out, dout, lse, q2k_idx, q2k_num, q_block_sizes, kv_block_sizes, B,
+                      H, Sq_pad, Skv_pad, D, idx_stride, scale, dq, dk, dv, workspace, status, st);
+  // the selection over 64-slot sub-blocks, after the 64-slot scratch
+  ExpandParams e;
+  memset(&e, 0, sizeof(e));
+  e.q2k_idx = q2k_idx;
+  e.q2k_num = q2k_num;
+  e.q_bs = q_block_sizes;
+  e.kv_bs = kv_block_sizes;
+  e.groups = (long long)B * H;
+  e.nq = Sq_pad / block_size;
+  e.nkv = Skv_pad / block_size;
+  e.idx_stride = idx_stride;
+  e.shift = shift;
+  e.status = status;
+  char* ws = static_cast<char*>(workspace) +
+             block_sparse_attn_backward_workspace_size(B, H, Sq_pad, Skv_pad / 64);
+  const size_t nq64 = (size_t)e.nq << shift;
+  e.idx64 = reinterpret_cast<int32_t*>(ws);
+  ws += align256(sizeof(int32_t) * (size_t)e.groups * nq64 * ((size_t)idx_stride << shift));
+  e.num64 = reinterpret_cast<int32_t*>(ws);
+  ws += align256(sizeof(int32_t) * (size_t)e.groups * nq64);
+  e.q_bs64 = reinterpret_cast<int32_t*>(ws);
+  ws += align256(sizeof(int32_t) * nq64);
+  e.kv_bs64 = reinterpret_cast<int32_t*>(ws);
+  rc = launch_expand_selection(e, st);
+  if (rc != VSA_OK) return rc;
+  return backward64(q, k, v, out, dout, lse, e.idx64, e.num64, e.q_bs64, e.kv_bs64, B, H, Sq_pad,
+                    Skv_pad, D, idx_stride << shift, scale, dq, dk, dv, workspace, status, st);
 }
 
 size_t block_sparse_attn_varlen_backward_workspace_size(int n_seqs, int total_q_blocks,

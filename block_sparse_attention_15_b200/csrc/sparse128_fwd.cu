@@ -542,6 +542,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (half == 0) {
         const float lsum = xs[row] + xs[128 + row];
         inv_l[o * 128 + row] = lsum > 0.f ? 1.f / lsum : 0.f;
+        if (p.lse) {
+          // natural-log log-sum-exp of the row: reference max plus log2 of
+          // the sum (both in log2 units) times ln 2; -inf with no key
+          // selected, 0 on padding rows
+          const float v = row >= x.q_len ? 0.f
+                          : (lsum > 0.f ? (m + __log2f(lsum)) * 0.69314718055994531f : -INFINITY);
+          p.lse[x.group * p.lse_seq + 128LL * x.a + row] = v;
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + L::kLFull + o);

@@ -962,4 +962,80 @@ int launch_backward(const BwdParams& p_in, const void* out, Strides3 out_st, int
   return D == 128 ? launch_bwd_t<128>(p, mq, mk, mv, mdo, st) : launch_bwd_t<64>(p, mq, mk, mv, mdo, st);
 }
 
+
+// ---------------------------------------------------------------------------
+// Selection over 128- or 256-slot blocks -> the same selection over 64-slot
+// sub-blocks, so the 64-slot backward kernels serve the larger tiles.  One
+// warp per (group, query block) index row; the sub-block sizes are written
+// by a grid-stride loop over all threads first.
+// ---------------------------------------------------------------------------
+namespace bwd {
+
+__global__ void __launch_bounds__(256) expand_selection_kernel(ExpandParams e) {
+  const int r = 1 << e.shift, blk = 64 << e.shift;
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long n_threads = (long long)gridDim.x * blockDim.x;
+  const long long n_qsub = (long long)e.nq << e.shift;
+  const long long n_sub = n_qsub + ((long long)e.nkv << e.shift);
+  for (long long i = tid; i < n_sub; i += n_threads) {
+    const bool is_q = i < n_qsub;
+    const long long j = is_q ? i : i - n_qsub;
+    const int32_t* bs = is_q ? e.q_bs : e.kv_bs;
+    int len = bs ? bs[j >> e.shift] : blk;
+    len = (len < 1 ? 0 : (len > blk ? blk : len)) - 64 * (int)(j & (r - 1));
+    (is_q ? e.q_bs64 : e.kv_bs64)[j] = len < 0 ? 0 : (len > 64 ? 64 : len);
+  }
+  const long long w = tid >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= e.groups * e.nq) return;
+  const int a = (int)(w % e.nq);
+  int n = e.q2k_num[w];
+  if (n < 0 || n > e.idx_stride) {
+    if (lane == 0) set_status(e.status, VSA_ERR_INDEX_RANGE);
+    n = n < 0 ? 0 : e.idx_stride;
+  }
+  int ql = e.q_bs ? e.q_bs[a] : blk;
+  ql = ql < 1 ? 0 : (ql > blk ? blk : ql);
+  const int32_t* row = e.q2k_idx + w * (long long)e.idx_stride;
+  const long long stride64 = (long long)e.idx_stride << e.shift;
+  int32_t* out0 = e.idx64 + (w << e.shift) * stride64;  // sub-row i at out0 + i * stride64
+  int total = 0;
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    int c = 0, cnt = 0;
+    if (j < n) {
+      c = row[j];
+      if (c < 0 || c >= e.nkv) {
+        set_status(e.status, VSA_ERR_INDEX_RANGE);
+      } else {
+        int kl = e.kv_bs ? e.kv_bs[c] : blk;
+        kl = kl < 1 ? 0 : (kl > blk ? blk : kl);
+        cnt = (kl + 63) >> 6;                    // sub-blocks holding real keys
+      }
+    }
+    int inc = cnt;                               // inclusive prefix over the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    const int pos = total + inc - cnt;
+    for (int s = 0; s < cnt; ++s)
+      for (int i = 0; i < r; ++i)
+        if (ql > 64 * i) out0[i * stride64 + pos + s] = (c << e.shift) + s;
+    total += __shfl_sync(0xffffffffu, inc, 31);
+  }
+  if (lane < r) e.num64[(w << e.shift) + lane] = ql > 64 * lane ? total : 0;
+}
+
+}  // namespace bwd
+
+int launch_expand_selection(const ExpandParams& e, cudaStream_t st) {
+  if (e.groups <= 0 || e.nq <= 0 || e.nkv <= 0) return VSA_OK;
+  if (e.shift < 1 || e.shift > 2) return VSA_ERR_UNSUPPORTED;
+  const long long threads = e.groups * e.nq * 32;
+  bwd::expand_selection_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(e);
+  return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
 }  // namespace vsa

@@ -160,6 +160,26 @@ struct BwdParams {
 int launch_backward(const BwdParams& p, const void* out, Strides3 out_st, int D,
                     cudaStream_t stream);
 
+// A selection over blocks of 64 << shift slots rewritten as the same
+// selection over 64-slot sub-blocks (sparse_bwd.cu): sub-block 2^shift * c + i
+// holds slots 64 i .. 64 i + 63 of block c.  Every listed block becomes its
+// sub-blocks that hold real tokens, in order (same keys, same
+// multiplicities); query sub-blocks without real rows list nothing.
+struct ExpandParams {
+  const int32_t* q2k_idx;     // [groups, nq, idx_stride]
+  const int32_t* q2k_num;     // [groups, nq]
+  const int32_t* q_bs;        // [nq] or null (full blocks)
+  const int32_t* kv_bs;       // [nkv] or null
+  int32_t* idx64;             // [groups, nq << shift, idx_stride << shift]
+  int32_t* num64;             // [groups, nq << shift]
+  int32_t* q_bs64;            // [nq << shift]
+  int32_t* kv_bs64;           // [nkv << shift]
+  long long groups;
+  int nq, nkv, idx_stride, shift;
+  int* status;
+};
+int launch_expand_selection(const ExpandParams& e, cudaStream_t stream);
+
 // varlen / metadata helpers (vsa_varlen.cu)
 // Logit bound for the entries that take indices (same meaning as
 // CoarseParams::qk_bound): block row norms of q and k, then per (group,

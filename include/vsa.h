@@ -303,8 +303,8 @@ int vsa_forward_host(const void* q, const void* k, const void* v, const void* ga
  * lse      device fp32 [B, H, Sq_pad] or NULL: the natural-log
  *          log-sum-exp of each real query row's scaled logits over its
  *          selected keys (-inf where nothing is selected, 0 on padded rows),
- *          the softmax normaliser block_sparse_attn_backward takes.  Block
- *          size 64 only.
+ *          the softmax normaliser block_sparse_attn_backward(_ex) takes.
+ *          Any block size (ABI 2.1; 2.0 took it at block size 64 only).
  * layout   host, strides of q, k, v and out (gate unused), or NULL for
  *          contiguous BHSD
  * workspace  device, >= block_sparse_attn_from_indices_workspace_size(...)
@@ -458,6 +458,51 @@ int block_sparse_attn_backward(const void* q, const void* k, const void* v, cons
                                int Skv_pad, int D, int idx_stride, float scale, void* dq,
                                void* dk, void* dv, void* workspace, size_t workspace_bytes,
                                void* stream);
+
+/*
+ * Workspace bytes block_sparse_attn_backward_ex needs: those of
+ * block_sparse_attn_backward_workspace_size(B, H, Sq_pad, Skv_pad / 64),
+ * then for block_size 128 / 256 the selection rewritten over 64-slot
+ * sub-blocks: int32 index rows [B, H, Sq_pad / 64, idx_stride * r], counts
+ * [B, H, Sq_pad / 64], query and key sub-block sizes (r = block_size / 64).
+ * 0 for invalid arguments.  (ABI 2.1.)
+ */
+size_t block_sparse_attn_backward_ex_workspace_size(int B, int H, int Sq_pad, int Skv_pad,
+                                                    int block_size, int idx_stride);
+
+/*
+ * block_sparse_attn_backward_ex -- block_sparse_attn_backward for a forward
+ * call of any block size (64, 128 or 256; ABI 2.1).
+ *
+ * Defined by: PR #1319 "Summary" / "Backward correctness" as for
+ * block_sparse_attn_backward, at the tile sizes of release 0.3.0's 128/256
+ * tile fastpath ("Block-sparse / VSA attention improvements").  The gradients of attention over a list of blocks depend only on
+ * which key rows each query row sees, so a selection over blocks of
+ * 64 r slots equals the selection over their 64-slot sub-blocks: a first
+ * launch rewrites it on the device (every listed block c becomes its
+ * sub-blocks r c + i that hold real keys, i = 0 .. r - 1, in order, with the
+ * same multiplicity; each query sub-block with real rows lists them all,
+ * the others nothing), then the four launches of block_sparse_attn_backward
+ * run on it.  The results equal those of the 64-slot call on that rewritten
+ * selection bit for bit.
+ *
+ * Arguments as in block_sparse_attn_backward, plus
+ * block_size  64, 128 or 256: that of the forward call; q2k_idx, q2k_num,
+ *          q_block_sizes, kv_block_sizes are in its blocks (Sq_pad /
+ *          block_size query blocks, Skv_pad / block_size KV blocks)
+ * Limits: idx_stride * block_size / 64, Sq_pad / 64 and Skv_pad / 64 at most
+ * VSA_MAX_BLOCKS (else VSA_ERR_UNSUPPORTED).
+ * workspace  device, >= block_sparse_attn_backward_ex_workspace_size(...),
+ *          256-aligned
+ * Five launches on `stream` for block size 128 / 256, four for 64.
+ */
+int block_sparse_attn_backward_ex(const void* q, const void* k, const void* v, const void* out,
+                                  const void* dout, const float* lse, const int32_t* q2k_idx,
+                                  const int32_t* q2k_num, const int32_t* q_block_sizes,
+                                  const int32_t* kv_block_sizes, int B, int H, int Sq_pad,
+                                  int Skv_pad, int D, int block_size, int idx_stride, float scale,
+                                  void* dq, void* dk, void* dv, void* workspace,
+                                  size_t workspace_bytes, void* stream);
 
 /* Workspace bytes block_sparse_attn_varlen_backward needs: the block tables,
  * delta per packed query row [H, total_q] and the k2q index over the packed

@@ -686,6 +686,56 @@ def check_backward(O):
             assert np.all(k2q[0, h, c, len(want):] == -1)
 
 
+
+def check_backward_large_blocks(O):
+    """At 128- and 256-slot blocks: dq, dk, dv against torch autograd (fp64)
+    of the independently written forward at that block size, and lse against
+    torch's logsumexp, with partial query and key blocks (some holding fewer
+    than 64 real rows), duplicates and an empty selection."""
+    rng = _rng(43)
+    B, H, D = 1, 2, 8
+    for blk, q_sizes, kv_sizes in ((128, [128, 50, 100], [128, 30, 70, 128]),
+                                   (256, [256, 130], [200, 40, 256])):
+        nkv = len(kv_sizes)
+
+        def padded(sizes, pad_value=0.0):
+            x = np.full((B, H, blk * len(sizes), D), pad_value, dtype=np.float64)
+            for j, m in enumerate(sizes):
+                x[:, :, blk * j:blk * j + m] = _bf16_like(rng, (B, H, m, D))
+            return x
+
+        q, k, v, do = padded(q_sizes), padded(kv_sizes, 2.0), padded(kv_sizes, -2.0), padded(q_sizes)
+        width = 4
+        idx = np.full((B, H, len(q_sizes), width), -1, dtype=np.int32)
+        num = np.zeros((B, H, len(q_sizes)), dtype=np.int32)
+        for h, a in np.ndindex(H, len(q_sizes)):
+            if (h, a) == (1, 0):
+                continue                                  # empty selection
+            n = int(rng.integers(1, width + 1))
+            idx[0, h, a, :n] = rng.integers(0, nkv, size=n)   # duplicates allowed
+            num[0, h, a] = n
+        scale = 0.41
+        dq, dk, dv = O.block_sparse_attention_backward(q, k, v, do, idx, num, q_sizes, kv_sizes,
+                                                       scale, block=blk)
+        tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+        out = _torch_sparse_forward(tq, tk, tv, idx, num, q_sizes, kv_sizes, scale, block=blk)
+        out.backward(torch.tensor(do))
+        for got, want in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+            assert np.allclose(got, want.numpy(), atol=1e-12), blk
+        assert np.all(dq[0, 1, 0:blk] == 0.0)
+        lse = O.block_sparse_lse(q, k, idx, num, q_sizes, kv_sizes, scale, block=blk)
+        for h, a in np.ndindex(H, len(q_sizes)):
+            rows_q = slice(blk * a, blk * a + q_sizes[a])
+            if num[0, h, a] == 0:
+                assert np.all(np.isneginf(lse[0, h, rows_q]))
+                continue
+            rows = np.concatenate([np.arange(blk * int(c), blk * int(c) + kv_sizes[int(c)])
+                                   for c in idx[0, h, a, :num[0, h, a]]])
+            want = torch.logsumexp(scale * torch.tensor(q[0, h, rows_q]) @ torch.tensor(k[0, h, rows]).T,
+                                   dim=-1)
+            assert np.allclose(lse[0, h, rows_q], want.numpy(), atol=1e-12), (blk, h, a)
+            assert np.all(lse[0, h, blk * a + q_sizes[a]:blk * (a + 1)] == 0.0)
+
 ALL_CHECKS = [
     check_pool_closed_forms, check_coarse_special_cases, check_coarse_vs_library,
     check_topk_brute_force, check_topk_edge_cases, check_sparse_dense_equivalence,
@@ -693,4 +743,5 @@ ALL_CHECKS = [
     check_forward_dense_limit, check_varlen_pack_indices, check_varlen_equals_per_sequence,
     check_varlen_dense_vs_library, check_metadata, check_page_figures,
     check_block_map_to_indices, check_block128, check_block256, check_backward,
+    check_backward_large_blocks,
 ]

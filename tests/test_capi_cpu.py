@@ -251,3 +251,51 @@ def test_bool_mask_entry_argument_checks():
     assert call(Skv=64 * 4096) == 3
     assert call(block=96) == 3
     assert call(Sq=192, block=128) == 2
+
+
+def test_backward_ex_workspace_size():
+    """Block 64 needs the plain backward's bytes; 128 / 256 add the selection
+    rewritten over 64-slot sub-blocks (rows r times as many, r times as
+    wide, plus counts and sub-block sizes); bad sizes give 0."""
+    lib = _lib()
+    a = lambda x: (x + 255) // 256 * 256
+    B, H, Sq, Skv, stride = 1, 4, 128 * 10, 128 * 12, 5
+    base = lib.block_sparse_attn_backward_workspace_size(B, H, Sq, Skv // 64)
+    assert base > 0
+    assert lib.block_sparse_attn_backward_ex_workspace_size(B, H, Sq, Skv, 64, stride) == base
+    for blk in (128, 256):
+        Sq_b, Skv_b = blk * 5, blk * 6
+        r = blk // 64
+        nq, nkv = Sq_b // blk, Skv_b // blk
+        want = (lib.block_sparse_attn_backward_workspace_size(B, H, Sq_b, Skv_b // 64) +
+                a(4 * B * H * nq * r * stride * r) + a(4 * B * H * nq * r) + a(4 * nq * r) +
+                a(4 * nkv * r))
+        assert lib.block_sparse_attn_backward_ex_workspace_size(B, H, Sq_b, Skv_b, blk, stride) == want
+    assert lib.block_sparse_attn_backward_ex_workspace_size(B, H, 128 * 3 + 64, Skv, 128, 1) == 0
+    assert lib.block_sparse_attn_backward_ex_workspace_size(B, H, Sq, Skv, 96, 1) == 0
+    assert lib.block_sparse_attn_backward_ex_workspace_size(B, H, Sq, Skv, 128, 0) == 0
+
+
+def test_backward_ex_host_argument_checks():
+    """The block-size backward rejects bad arguments before any CUDA call."""
+    lib = _lib()
+    fake = 1 << 20
+    v = ctypes.c_void_p
+
+    def call(B=1, H=1, Sq=256, Skv=256, D=128, blk=128, stride=2, q=fake, ws=None, wsb=0):
+        return lib.block_sparse_attn_backward_ex(
+            v(q), v(fake), v(fake), v(fake), v(fake), v(fake), v(fake), v(fake), None, None, B, H,
+            Sq, Skv, D, blk, stride, 0.0, v(fake), v(fake), v(fake), None if ws is None else v(ws),
+            wsb, None)
+
+    assert call(q=None) == 1                                  # null input
+    assert call(D=96) == 3                                    # unsupported head dim
+    assert call(blk=96) == 3                                  # unsupported block size
+    assert call(Sq=128 + 64) == 2                             # not a multiple of the block
+    assert call(Sq=256 * 3, Skv=256 * 2, blk=256, stride=600) == 3   # 4 x 600 > VSA_MAX_BLOCKS
+    assert call(Skv=64 * 2050, Sq=128) == 3                   # Skv / 64 above VSA_MAX_BLOCKS
+    assert call(q=fake + 2) == 1                              # misaligned
+    assert call() == 7                                        # no workspace
+    need = lib.block_sparse_attn_backward_ex_workspace_size(1, 1, 256, 256, 128, 2)
+    assert call(ws=fake, wsb=need - 1) == 7                   # too small
+    assert call(ws=fake + 64, wsb=need) == 7                  # misaligned
