@@ -94,17 +94,20 @@ def sparse_source_hash() -> str:
     return h.hexdigest()
 
 
-def profiled_traffic():
-    """DRAM bytes per launch of the block-sparse kernel on the default workload,
-    from the committed record of an ncu capture (a JSON data file beside the
-    capture's summary), if the kernel sources still hash to what was
-    profiled; else None."""
+def profiled_traffic(wl):
+    """DRAM bytes per launch of the block-sparse kernel, from the committed
+    record of an ncu capture (a JSON data file beside the capture's summary),
+    if the workload has the recorded shape and the kernel sources still hash
+    to what was profiled; else None."""
     path = os.path.join(ROOT, "profiles", "sparse_fwd_h3_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
-    if rec.get("kernel_source_sha256") != sparse_source_hash():
+    shape = rec.get("shape", {})
+    ours = {"B": wl.B, "H": wl.H, "D": wl.D, "block": wl.block, "n_q_blocks": wl.nq,
+            "n_kv_blocks": wl.nkv, "topk": wl.topk}
+    if shape != ours or rec.get("kernel_source_sha256") != sparse_source_hash():
         return None
     return int(rec["traffic_bytes_per_launch"])
 
@@ -565,8 +568,9 @@ def run_ours(args, wl):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_of(wl, flush is not None),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": profiled_traffic(),
-                         "kernel": "sparse_fwd_kernel (block-sparse attention + fused gated combine)",
+                         "frac": achieved / peak, "traffic": profiled_traffic(wl),
+                         "kernel": ("sparse_fwd_kernel" if wl.block == 64 else "sparse128_fwd_kernel") +
+                                   " (block-sparse attention + fused combine)",
                          "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS)",
                          "frac_of_sustained": achieved / sustained},
             "kernels_ms": {"pool": k_pool, "coarse_topk": k_coarse, "sparse_combine": k_sparse,

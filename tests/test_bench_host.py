@@ -71,3 +71,14 @@ def test_forward_host_binding_rejects_bad_tensors():
         vsa.vsa_forward_host(q, k, k, torch.zeros((1, 128, 3, 64), dtype=torch.bfloat16), topk=1)
     with pytest.raises(ValueError):
         vsa.vsa_forward_host(q, k, k, topk=1, q_block_sizes=[64])     # 2 query blocks
+
+
+def test_traffic_record_applies_to_its_workload_only():
+    """The committed DRAM-traffic record is reported for the workload shape it
+    was captured on (with the kernel sources unchanged) and for no other."""
+    import dataclasses
+    h3 = bench.make_workload("h3")
+    assert bench.profiled_traffic(h3) == 1080151296
+    assert bench.profiled_traffic(bench.make_workload("vsa128")) is None
+    assert bench.profiled_traffic(bench.make_workload("long10")) is None
+    assert bench.profiled_traffic(dataclasses.replace(h3, H=16)) is None
