@@ -733,15 +733,19 @@ def run_entry(args, wl):
         # the backward of the sparse attention on the forward's selection:
         # algorithmic work 5 tile products (S recomputed, dP, dV, dK, dQ)
         # = 2.5 x the forward's per tile
-        if wl.block != 64:
-            raise SystemExit("the backward covers 64-slot blocks")
-        o_s, lse = vsa.block_sparse_attn_from_indices(q, k, v, idx, num, qbs, kbs, return_lse=True)
+        o_s, lse = vsa.block_sparse_attn_from_indices(q, k, v, idx, num, qbs, kbs, block=wl.block,
+                                                      return_lse=True)
         dout = I.normal_bf16(tuple(q.shape), wl.seed, 7).to(dev)
 
         def step():
-            vsa.block_sparse_attn_backward(q, k, v, o_s, dout, lse, idx, num, qbs, kbs)
-        what = "block_sparse_attn_backward (delta, k2q, dq pass, dk/dv pass) on the forward's selection"
-        launches = 4
+            vsa.block_sparse_attn_backward(q, k, v, o_s, dout, lse, idx, num, qbs, kbs, block=wl.block)
+        if wl.block == 64:
+            what = "block_sparse_attn_backward (delta, k2q, dq pass, dk/dv pass) on the forward's selection"
+            launches = 4
+        else:
+            what = ("block_sparse_attn_backward_ex (selection rewrite, delta, k2q, dq pass, dk/dv pass) "
+                    "on the forward's selection")
+            launches = 5
         flops = 2.5 * wl.flops
     elif args.entry == "ulysses":
         # the sequence-parallel wrapper over the ranks of the job (one rank:

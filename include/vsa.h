@@ -417,7 +417,8 @@ int block_sparse_attn_varlen(const void* q, const void* k, const void* v,
                              void* stream);
 
 /* ======================================================================== *
- * backward of the block-sparse attention (64-slot blocks)
+ * backward of the block-sparse attention (64-slot blocks; any block size
+ * through block_sparse_attn_backward_ex)
  * ======================================================================== */
 
 /*
