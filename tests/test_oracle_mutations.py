@@ -19,6 +19,13 @@ MUTATIONS = [
      "np.add.at(dk[b, h], rows, ds.T @ qa)"),
     ("backward dv ignores duplicates", "np.add.at(dv[b, h], rows, p.T @ da)",
      "dv[b, h][rows] += p.T @ da"),
+    ("backward query rows at 64-slot offsets", "qa = q[b, h, block * a:block * a + mq]\n",
+     "qa = q[b, h, BLOCK * a:BLOCK * a + mq]\n"),
+    ("backward dq written at 64-slot offsets",
+     "dq[b, h, block * a:block * a + mq] = scale * (ds @ k[b, h, rows])",
+     "dq[b, h, BLOCK * a:BLOCK * a + mq] = scale * (ds @ k[b, h, rows])"),
+    ("lse written at 64-slot offsets", "lse[b, h, block * a:block * a + mq] = m + np.log(",
+     "lse[b, h, BLOCK * a:BLOCK * a + mq] = m + np.log("),
     ("k2q drops multiplicities", "m = int(np.sum(idx[pos][a, :int(num[pos][a])] == c))",
      "m = int(np.any(idx[pos][a, :int(num[pos][a])] == c))"),
     ("block map rows not ascending", "idx[pos][:len(chosen)] = chosen",
