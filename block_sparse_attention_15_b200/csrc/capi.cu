@@ -750,9 +750,9 @@ static int backward64(const void* q, const void* k, const void* v, const void* o
   return launch_backward(bp, out, bhsd_strides(H, Sq_pad, D), D, st);
 }
 
-// Argument checks shared by both backward entries (sizes in 64-slot units
-// after any expansion: n_q = Sq_pad / 64, n_kv = Skv_pad / 64, the expanded
-// index row width `stride64`).
+// Argument checks shared by both backward entries.  The limits apply to the
+// 64-slot selection the passes run on: Sq_pad / 64 and Skv_pad / 64 blocks,
+// index rows idx_stride * block / 64 wide.
 static int check_backward_args(const void* q, const void* k, const void* v, const void* out,
                                const void* dout, const float* lse, const int32_t* q2k_idx,
                                const int32_t* q2k_num, void* dq, void* dk, void* dv, int B, int H,
